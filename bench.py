@@ -1,0 +1,326 @@
+#!/usr/bin/env python
+"""Benchmark of the SVDQuant W4A4 linear layer (NVFP4, rank 32, GELU) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload fc1_nvfp4]
+
+A step is one pass of the whole layer over one batch: the activation kernel
+(smooth + quantise + pack + down projection) and the 4-bit GEMM kernel (with
+the low-rank up projection, GELU and bf16 store), for the headline layer
+M=4608 tokens, K=3072, N=12288, r=32.  Inputs are seeded synthetic data
+already resident in HBM; L2 is flushed (a 256 MB write, outside the timed
+events) before every step.  Under torchrun each rank runs its own replica of
+the layer (the layer is token-parallel; no collective is on the data path),
+and the slowest rank's device time is reported.
+
+--impl reference times the CPU oracle (plain numpy) on the host cores on a
+bounded row sample per step, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4+rank-32 linear effective TFLOPS at M4608 K3072 N12288; % of FP4 TC roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="fc1_nvfp4")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "bit_diffusion_transformer_w4a4_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(f"{kernel}/{workload}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark(self, begin: bool):
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        loaded = [float(r[1]) for r in rows if float(r[3]) > 300.0] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(layer, pw, x_bits, nrows: int):
+    """The oracle, as it stands, on a row sample of the same workload."""
+    import numpy as np
+    from oracle import forward as O
+    rows = np.arange(nrows)
+    t = time.perf_counter()
+    O.linear_forward(x_bits, pw, rows=rows)
+    dt = time.perf_counter() - t
+    flops = 2.0 * nrows * layer.K * layer.N + 2.0 * nrows * layer.r * (layer.K + layer.N)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+            "sample": f"{nrows} of {layer.M} token rows of {layer.name} (numpy fp64), "
+                      f"{dt:.2f} s"}
+
+
+def run_reference(args, layer):
+    from bit_diffusion_transformer_w4a4_b200 import workloads as W
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    pw = W.synthetic_packed(layer)
+    x = W.activations(layer)
+    nrows = 64
+    for _ in range(min(args.warmup, 1)):
+        cpu_baseline(layer, pw, x, nrows)
+    times, t_start = [], time.perf_counter()
+    for _ in range(args.steps):
+        r = cpu_baseline(layer, pw, x, nrows)
+        times.append(r)
+        if time.perf_counter() - t_start > 120.0:
+            break
+    flops = 2.0 * nrows * layer.K * layer.N + 2.0 * nrows * layer.r * (layer.K + layer.N)
+    tflops = statistics.median(t["value"] for t in times)
+    ms = flops / (tflops * 1e12) * 1e3
+    line = {"metric": METRIC, "value": tflops, "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": len(times), "warmup": min(args.warmup, 1), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"{layer.name} M{layer.M} K{layer.K} N{layer.N} r{layer.r}"
+                                   f"{' GELU' if layer.gelu else ''} NVFP4",
+                       "step_sample_rows": nrows},
+            "cpu_baseline": {k: times[-1][k] for k in ("unit", "cores", "kind", "sample")}
+            | {"value": tflops},
+            "e2e": {"value": tflops, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, layer):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from bit_diffusion_transformer_w4a4_b200 import svdq
+    from bit_diffusion_transformer_w4a4_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    M, K, N, r = layer.M, layer.K, layer.N, layer.r
+    pw = W.synthetic_packed(layer, seed=rank)
+    x_bits = W.activations(layer, seed=rank)
+    h = svdq.SVDQWeights(pw, M)
+    x = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    codes, scales, t = h.alloc_act(M)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        flush.zero_()                      # L2 flush, outside the timed events
+        if ev is not None:
+            ev[0].record(stream)
+        h.quantize_act_lowrank_down(x, M, codes, scales, t)
+        if ev is not None:
+            ev[1].record(stream)
+        h.w4a4_gemm_lowrank_up(codes, scales, t, M, y)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = h.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {svdq.STATUS.get(st)} after warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    clocks.mark(True)
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    clocks.mark(False)
+    clk = clocks.stop()
+    st = h.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {svdq.STATUS.get(st)} in the timed region")
+    t_kq = [e[0].elapsed_time(e[1]) for e in evs]
+    t_kg = [e[1].elapsed_time(e[2]) for e in evs]
+    ms_step = statistics.mean(a + b for a, b in zip(t_kq, t_kg))
+    ms_kg = statistics.mean(t_kg)
+    ms_kq = statistics.mean(t_kq)
+    if world > 1:
+        tt = torch.tensor([ms_step, ms_kg, ms_kq], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_step, ms_kg, ms_kq = tt.tolist()
+
+    flops = layer.flops()
+    value = world * flops / (ms_step * 1e-3) / 1e12
+
+    # end to end through the host entry point (pinned buffers, copies timed)
+    xh = torch.from_numpy(x_bits.view(np.int16)).pin_memory()
+    yh = torch.empty((M, N), dtype=torch.int16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        h.linear_forward_host(xh, yh, M)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        h.linear_forward_host(xh, yh, M)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([ms_e2e], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_e2e = tt.item()
+    if h.device_status() != 0:
+        raise RuntimeError("device status error in the end-to-end loop")
+
+    pk, pk_src = peaks()
+    # dominant kernel: the 4-bit GEMM; FP4 dense peak = measured bf16 burst x 4 (9 / 2.25 PF nominal)
+    kg_flops = 2.0 * M * K * N + 2.0 * M * N * r
+    achieved = kg_flops / (ms_kg * 1e-3) / 1e12
+    peak = pk["bf16_tflops"] * 4.0
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": f"{layer.name} M{M} K{K} N{N} r{r}{' GELU' if layer.gelu else ''} "
+                               f"{W.VARIANT_NAME[layer.variant]}",
+                   "l2": "flushed before every step (256 MB write, outside the timed events)",
+                   "parallelism": f"replicas x{world}", "tokens_per_step": M * world},
+        "tokens_per_s": world * M / (ms_step * 1e-3),
+        "frac_of_fp4_roofline": None,
+        "kernels_ms": {"quantize_act_lowrank_down": ms_kq, "w4a4_gemm_lowrank_up": ms_kg},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic("w4a4_gemm_lowrank_up", args.workload),
+                     "peak_source": f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 4 (FP4:BF16 nominal 9:2.25)"},
+        "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS",
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    # whole-layer roofline: the slower of FP4 compute and the layer's HBM bytes
+    bytes_alg = (M * K * 2 + 2 * (M * K // 2) + 2 * (M * K // 16) + N * K // 2 + N * K // 16
+                 + K * r * 2 + r * N * 2 + 2 * M * r * 4 + M * N * 2)
+    t_star = max(flops / (peak * 1e12), bytes_alg / (pk["hbm_gbs"] * 1e9))
+    line["frac_of_fp4_roofline"] = t_star / (ms_step * 1e-3)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(layer, pw, x_bits, 1024)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    from bit_diffusion_transformer_w4a4_b200 import workloads as W
+    layer = W.workloads()[args.workload][0]
+    if args.impl == "reference":
+        run_reference(args, layer)
+    else:
+        run_ours(args, layer)
+
+
+if __name__ == "__main__":
+    main()

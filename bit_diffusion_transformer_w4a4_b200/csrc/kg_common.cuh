@@ -1,0 +1,123 @@
+// Pieces shared by the two GEMM kernels (NVFP4 and INT4): parameters, the
+// low-rank operand preparation and the output epilogue.
+//
+// The low-rank up projection T L2 ("Problemas do Nunchaku Qwen...",
+// apatero.com, section "O que e Nunchaku e como acelera modelos Qwen": the
+// up projection is fused into the 4-bit compute kernel) runs on the tensor
+// cores as extra bf16 k-steps into the same fp32 accumulator.  T arrives in
+// fp32; it is split into T_hi = bf16(T) and T_lo = bf16(T - T_hi) so that
+//   T L2 = [T_hi | T_lo] . [L2 ; L2]
+// keeps 16 significant bits of T (bf16 x bf16 products are exact in fp32).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace svdq {
+
+constexpr int KG_THREADS = 640;  // 4 control warps + 16 epilogue warps
+constexpr int KG_EPI_WARPS = 16;
+constexpr int KG_BM = 128;
+constexpr int KG_BN = 256;
+
+struct KGParams {
+  const uint8_t* sfa;   // NVFP4: tiled activation scales; INT4: bf16 [M x K/64]
+  const uint8_t* sfb;   // NVFP4: tiled weight scales; INT4: bf16 [K/64 x Npad]
+  const float* t;       // [M x R] fp32 (unused when R == 0)
+  const uint16_t* bias; // bf16 [N] or null
+  uint16_t* y;          // bf16 [M x N]
+  int M, N, K;
+  int num_m, num_n;
+  int gelu;
+  int* err;
+  uint32_t debug_mask;
+  uint64_t timeout_ns;
+};
+
+// GELU, tanh form: 0.5 x (1 + tanh(u)) = x / (1 + exp(-2u)),
+// u = sqrt(2/pi) (x + 0.044715 x^3).
+__device__ __forceinline__ float gelu_tanh(float x) {
+  const float u = __fmul_rn(__fmul_rn(x, __fmaf_rn(0.044715f * x, x, 1.0f)), 0.7978845608028654f);
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-2.8853900817779268f * u));
+  return __fdividef(x, 1.0f + e);
+}
+
+// Write [T_hi | T_lo] of rows m0..m0+127 into the A operand buffer of the
+// low-rank k-steps: 128 rows x (64 bf16 = 128 B) chunks, 128B swizzle.
+// Called by the 512 epilogue threads (etid = 0..511).
+template <int R>
+__device__ __forceinline__ void prep_lowrank_a(uint8_t* alr, const float* __restrict__ t, int m0,
+                                               int M, int etid) {
+  constexpr int SEG = R / 8;  // 8 values of T per item
+  for (int it = etid; it < 128 * SEG; it += KG_EPI_WARPS * 32) {
+    const int row = it / SEG;
+    const int seg = it % SEG;
+    const int gm = m0 + row;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (gm < M) {
+      const float4* src = reinterpret_cast<const float4*>(t + static_cast<size_t>(gm) * R + seg * 8);
+      a = __ldg(src);
+      b = __ldg(src + 1);
+    }
+    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+      const float h0 = __low2float(h), h1 = __high2float(h);
+      const __nv_bfloat162 l = __floats2bfloat162_rn(__fsub_rn(v[2 * j], h0), __fsub_rn(v[2 * j + 1], h1));
+      hi[j] = *reinterpret_cast<const uint32_t*>(&h);
+      lo[j] = *reinterpret_cast<const uint32_t*>(&l);
+    }
+    const int chi = seg * 8;      // logical bf16 column of T_hi
+    const int clo = R + seg * 8;  // logical bf16 column of T_lo
+    *reinterpret_cast<uint4*>(alr + (chi / 64) * 16384 + swz_off(row, (chi % 64) / 8, 128)) =
+        make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(alr + (clo / 64) * 16384 + swz_off(row, (clo % 64) / 8, 128)) =
+        make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
+// Store 64 fp32 accumulator columns of one row: + bias, GELU, bf16.
+__device__ __forceinline__ void store_row64(const KGParams& p, int gm, int n_base, const float* acc) {
+  if (gm >= p.M) return;
+  uint16_t* dst = p.y + static_cast<size_t>(gm) * p.N;
+#pragma unroll
+  for (int j8 = 0; j8 < 8; ++j8) {
+    const int n = n_base + 8 * j8;
+    if (n >= p.N) break;
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = acc[8 * j8 + e];
+    if (p.bias != nullptr) {
+      const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
+      const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = __fadd_rn(v[2 * e], bf16lo(bw[e]));
+        v[2 * e + 1] = __fadd_rn(v[2 * e + 1], bf16hi(bw[e]));
+      }
+    }
+    if (p.gelu) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = gelu_tanh(v[e]);
+    }
+    *reinterpret_cast<uint4*>(dst + n) =
+        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                   pack_bf16x2(v[6], v[7]));
+  }
+}
+
+// Wait for the producer's outstanding loads before the CTA exits (abort path).
+__device__ __forceinline__ void drain_loads(uint32_t bar_full, uint32_t issued, uint32_t issued_par,
+                                            int stages, uint64_t limit_ns) {
+  for (int s = 0; s < stages; ++s)
+    if (issued & (1u << s)) {
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bar_full + 8 * s, (issued_par >> s) & 1) &&
+             global_timer_ns() - t0 < limit_ns) {
+      }
+    }
+}
+
+}  // namespace svdq

@@ -1,0 +1,328 @@
+// Kernel 2, INT4 variant: the 4-bit GEMM on the packed residual with bf16
+// group scales (group 64 along K),
+//   acc[m,n] = sum_g s_x[m,g] s_w[n,g] P_g[m,n],  P_g = sum_{k in g} q_x q_w,
+// with P_g exact on the int8 tensor cores (tcgen05 kind::i8, s32 accumulate)
+// and the scale product applied per group in fp32 by the epilogue warps.
+// The low-rank up projection runs as bf16 MMAs into one more accumulator
+// buffer that the epilogue adds with weight 1.
+//
+// Method: "Nunchaku 1.3.0 for Python3.14.x & alpha" (note.com), section
+// "SVDQ-FP4 on Blackwell", part "1. INT4" (INT4 -8..+7, W ~ int4 * scale);
+// "Nunchaku Lite ... integrated into Diffusers" (axbrief.com), section "The
+// Mechanics of 4-Bit Efficiency and SVDQuant" (W4A4 residual + 16-bit
+// low-rank branch).
+//
+// Warp roles (640 threads):
+//   warp 0      TMA producer: packed activation codes (32B swizzle) and int8
+//               weight codes (64B swizzle) for one 64-group per stage
+//   warp 1      MMA issuer (two k-steps of 32 per group), tensor-memory owner
+//   warps 2-3   unpack activation nibbles to int8 in the MMA operand layout
+//   warps 4-19  epilogue: per-group rescale into fp32 registers, low-rank
+//               add, next tile's low-rank operand, bias + GELU + bf16 stores
+#pragma once
+
+#include "kg_common.cuh"
+
+namespace svdq {
+
+template <int R>
+struct KGI4Smem {
+  static constexpr int STAGES = R >= 128 ? 5 : 6;
+  static constexpr int APK_BYTES = KG_BM * 32;   // 128 rows x 32 B packed (64 codes)
+  static constexpr int A8_BYTES = KG_BM * 64;    // 128 rows x 64 int8
+  static constexpr int B_BYTES = KG_BN * 64;     // 256 rows x 64 int8
+  static constexpr int STAGE = APK_BYTES + A8_BYTES + B_BYTES;
+  static constexpr int LR_CHUNKS = R > 0 ? (2 * R + 63) / 64 : 0;
+  static constexpr int ALR_OFF = STAGES * STAGE;
+  static constexpr int BAR_OFF = ALR_OFF + LR_CHUNKS * 16384;
+  static constexpr int TOTAL = BAR_OFF + 512 + 1024;
+};
+
+// 8 two's-complement nibbles (element 0 in the low nibble) -> 8 int8 bytes.
+__device__ __forceinline__ uint2 unpack_s4x8(uint32_t w) {
+  uint32_t lo = w & 0x0F0F0F0Fu;          // elements 0, 2, 4, 6
+  uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;   // elements 1, 3, 5, 7
+  // per byte: n -> n - 16 when n >= 8 (no carries: every byte stays < 136)
+  lo = ((lo ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+  hi = ((hi ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+  uint2 r;
+  r.x = __byte_perm(lo, hi, 0x5140);
+  r.y = __byte_perm(lo, hi, 0x7362);
+  return r;
+}
+
+template <int R>
+__global__ void __launch_bounds__(KG_THREADS, 1)
+    kg_int4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                   const __grid_constant__ CUtensorMap tm_blr, KGParams p) {
+  using S = KGI4Smem<R>;
+  constexpr int NST = S::STAGES;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+  const uint32_t bar_full = smem_u32(bars);
+  const uint32_t bar_ready = smem_u32(bars + NST);
+  const uint32_t bar_empty = smem_u32(bars + 2 * NST);
+  const uint32_t bar_gfull = smem_u32(bars + 3 * NST);       // [2]
+  const uint32_t bar_gempty = smem_u32(bars + 3 * NST + 2);  // [2]
+  const uint32_t bar_lr_full = smem_u32(bars + 3 * NST + 4);
+  const uint32_t bar_drain = smem_u32(bars + 3 * NST + 5);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NST + 6);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Guard guard{p.err, abort_flag, p.timeout_ns};
+  const int num_tiles = p.num_m * p.num_n;
+  const int ng = p.K / 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_ready + 8 * s, 2);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_gfull + 8 * b, 1);
+      mbar_init(bar_gempty + 8 * b, KG_EPI_WARPS);
+    }
+    mbar_init(bar_lr_full, KG_EPI_WARPS);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_b);
+      if (R > 0) tma_prefetch_desc(&tm_blr);
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
+        const int mb = tile % p.num_m, nb = tile / p.num_m;
+        for (int g = 0; g < ng; ++g) {
+          if (!(ok = wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x301))) break;
+          issued &= ~(1u << s);
+          if (!((p.debug_mask & 1u) && j == 0 && g == 1)) {  // test hook: leave one stage empty
+            const uint32_t st = sbase + s * S::STAGE;
+            const uint32_t fb = bar_full + 8 * s;
+            mbar_expect_tx(fb, S::APK_BYTES + S::B_BYTES);
+            tma_load_2d(st, &tm_a, fb, g * 32, mb * KG_BM);
+            tma_load_2d(st + S::APK_BYTES + S::A8_BYTES, &tm_b, fb, g * 64, nb * KG_BN);
+            issued |= 1u << s;
+            issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          }
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+        for (int l = 0; l < R / 16 && ok; ++l) {
+          if (!(ok = wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x302))) break;
+          issued &= ~(1u << s);
+          const uint32_t fb = bar_full + 8 * s;
+          mbar_expect_tx(fb, KG_BN * 64);
+          tma_load_2d(sbase + s * S::STAGE + S::APK_BYTES + S::A8_BYTES, &tm_blr, fb, l * 32,
+                      nb * KG_BN);
+          issued |= 1u << s;
+          issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+      }
+      if (*abort_flag) drain_loads(bar_full, issued, issued_par, NST, p.timeout_ns);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t id_s8 = idesc_s8_s32(KG_BM, KG_BN);
+      constexpr uint32_t id_bf = idesc_bf16_f32(KG_BM, KG_BN);
+      const uint32_t alr = sbase + S::ALR_OFF;
+      int s = 0;
+      uint32_t ph = 0, gc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
+        for (int g = 0; g < ng; ++g, ++gc) {
+          const uint32_t b = gc & 1, use = gc >> 1;
+          if (!(ok = wait_bounded(bar_gempty + 8 * b, (use & 1) ^ 1, guard, 0x303))) break;
+          if (!(ok = wait_bounded(bar_ready + 8 * s, ph, guard, 0x304))) break;
+          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x305))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + s * S::STAGE;
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint64_t a = smem_desc(st + S::APK_BYTES + kk * 32, 16, 512, SWZ_64B);
+            const uint64_t bd = smem_desc(st + S::APK_BYTES + S::A8_BYTES + kk * 32, 16, 512, SWZ_64B);
+            mma_s8(tmem + b * 256, a, bd, id_s8, kk);
+          }
+          tc_commit(bar_empty + 8 * s);
+          tc_commit(bar_gfull + 8 * b);
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        if (R > 0) {
+          const uint32_t b = gc & 1, use = gc >> 1;
+          if (!(ok = wait_bounded(bar_gempty + 8 * b, (use & 1) ^ 1, guard, 0x306))) break;
+          if (!(ok = wait_bounded(bar_lr_full, j & 1, guard, 0x307))) break;
+          tc_fence_after();
+          for (int l = 0; l < R / 16; ++l) {
+            if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x308))) break;
+            tc_fence_after();
+            const uint32_t bst = sbase + s * S::STAGE + S::APK_BYTES + S::A8_BYTES;
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int kk = 2 * l + k2;
+              const uint64_t a = smem_desc(alr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, SWZ_128B);
+              const uint64_t bd = smem_desc(bst + k2 * 32, 16, 512, SWZ_64B);
+              mma_bf16(tmem + b * 256, a, bd, id_bf, kk != 0);
+            }
+            tc_commit(bar_empty + 8 * s);
+            if (++s == NST) { s = 0; ph ^= 1; }
+          }
+          if (!ok) break;
+          tc_commit(bar_gfull + 8 * b);
+          ++gc;
+        }
+      }
+      tc_commit(bar_drain);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < p.timeout_ns) {
+      }
+    }
+  } else if (warp < 4) {
+    // --------------------------------------------- nibble -> int8 transform
+    const int tt = threadIdx.x - 64;  // 0..63: rows tt and tt + 64
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int g = 0; g < ng; ++g) {
+        if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x309))) break;
+        const uint8_t* apk = smem + s * S::STAGE;
+        uint8_t* a8 = smem + s * S::STAGE + S::APK_BYTES;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int row = tt + 64 * h;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(apk + swz_off(row, c, 32));
+            const uint2 o0 = unpack_s4x8(v.x), o1 = unpack_s4x8(v.y);
+            const uint2 o2 = unpack_s4x8(v.z), o3 = unpack_s4x8(v.w);
+            *reinterpret_cast<uint4*>(a8 + swz_off(row, 2 * c, 64)) = make_uint4(o0.x, o0.y, o1.x, o1.y);
+            *reinterpret_cast<uint4*>(a8 + swz_off(row, 2 * c + 1, 64)) = make_uint4(o2.x, o2.y, o3.x, o3.y);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ready + 8 * s);
+        if (++s == NST) { s = 0; ph ^= 1; }
+      }
+      for (int l = 0; l < R / 16; ++l)
+        if (++s == NST) { s = 0; ph ^= 1; }
+    }
+  } else {
+    // ----------------------------------------------------------------- epilogue
+    const int e = warp - 4;
+    const int q = warp & 3;
+    const int cs = e >> 2;
+    const int row = q * 32 + lane;
+    const int etid = threadIdx.x - 128;
+    uint8_t* alr = smem + S::ALR_OFF;
+    const __nv_bfloat16* sx_all = reinterpret_cast<const __nv_bfloat16*>(p.sfa);
+    const float* sw_all = reinterpret_cast<const float*>(p.sfb);
+    const int npad = p.num_n * KG_BN;
+    if constexpr (R > 0) {
+      if (static_cast<int>(blockIdx.x) < num_tiles) {
+        prep_lowrank_a<R>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_lr_full);
+      }
+    }
+    uint32_t gc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
+      const int mb = tile % p.num_m, nb = tile / p.num_m;
+      const int gm = mb * KG_BM + row;
+      const int n_base = nb * KG_BN + cs * 64;
+      const __nv_bfloat16* sxr = sx_all + static_cast<size_t>(gm < p.M ? gm : 0) * ng;
+      float acc[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+      float sx_next = gm < p.M ? __bfloat162float(sxr[0]) : 0.0f;
+      for (int g = 0; g < ng; ++g, ++gc) {
+        const uint32_t b = gc & 1, use = gc >> 1;
+        const float sx = sx_next;
+        if (g + 1 < ng) sx_next = gm < p.M ? __bfloat162float(sxr[g + 1]) : 0.0f;
+        if (!(ok = wait_bounded(bar_gfull + 8 * b, use & 1, guard, 0x30a))) break;
+        tc_fence_after();
+        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * 256 + cs * 64;
+        const float4* swr = reinterpret_cast<const float4*>(sw_all + static_cast<size_t>(g) * npad + n_base);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          uint32_t v[16];
+          tmem_ld_x16(ta + 16 * h, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i4 = 0; i4 < 4; ++i4) {
+            const float4 w = __ldg(swr + 4 * h + i4);
+            const int i = 16 * h + 4 * i4;
+            acc[i] = __fmaf_rn(__int2float_rn(static_cast<int>(v[4 * i4])), sx * w.x, acc[i]);
+            acc[i + 1] = __fmaf_rn(__int2float_rn(static_cast<int>(v[4 * i4 + 1])), sx * w.y, acc[i + 1]);
+            acc[i + 2] = __fmaf_rn(__int2float_rn(static_cast<int>(v[4 * i4 + 2])), sx * w.z, acc[i + 2]);
+            acc[i + 3] = __fmaf_rn(__int2float_rn(static_cast<int>(v[4 * i4 + 3])), sx * w.w, acc[i + 3]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_gempty + 8 * b);
+      }
+      if (!ok) break;
+      if constexpr (R > 0) {
+        const uint32_t b = gc & 1, use = gc >> 1;
+        if (!(ok = wait_bounded(bar_gfull + 8 * b, use & 1, guard, 0x30b))) break;
+        tc_fence_after();
+        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * 256 + cs * 64;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          uint32_t v[16];
+          tmem_ld_x16(ta + 16 * h, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[16 * h + i] = __fadd_rn(acc[16 * h + i], __uint_as_float(v[i]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_gempty + 8 * b);
+        ++gc;
+        const int next = tile + gridDim.x;
+        if (next < num_tiles) {
+          // the low-rank MMAs of this tile have completed: reuse the operand buffer
+          prep_lowrank_a<R>(alr, p.t, (next % p.num_m) * KG_BM, p.M, etid);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_lr_full);
+        }
+      }
+      store_row64(p, gm, n_base, acc);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace svdq

@@ -1,0 +1,250 @@
+// Kernel 2, NVFP4 variant: the 4-bit GEMM on the packed residual,
+//   acc[m,n] = sum_g s_x[m,g] s_w[n,g] sum_{k in g} q_x[m,k] q_w[n,k]
+// on tcgen05 block-scaled MMA (kind::mxf4nvf4, E2M1 operands, one UE4M3 scale
+// per 16 elements), followed in the same tile by the low-rank up projection
+// (bf16 MMA into the same fp32 tensor-memory accumulator) and an epilogue
+// that adds the bias, applies GELU and stores bf16.
+//
+// Method: "Nunchaku Lite ... integrated into Diffusers" (axbrief.com),
+// section "The Mechanics of 4-Bit Efficiency and SVDQuant" (4-bit residual
+// branch with 4-bit activations, W4A4) and section "Hardware Specialization
+// and the Compression Workflow" (NVFP4 on Blackwell); "Problemas do Nunchaku
+// Qwen..." (apatero.com), section "O que e Nunchaku..." (up projection fused
+// into the 4-bit kernel).
+//
+// Persistent CTAs, one per SM, tile 128 x 256.  Warp roles (640 threads):
+//   warp 0      TMA producer: A/B code tiles (tensor maps, 64B swizzle) and
+//               the matching scale-factor atoms (bulk copies)
+//   warp 1      MMA issuer: scale factors shared->tensor memory, block-scaled
+//               MMAs, then the low-rank bf16 MMAs; owns tensor memory
+//   warps 4-19  epilogue: drain the accumulator, prepare the next tile's
+//               low-rank operand, bias + GELU + bf16 stores
+#pragma once
+
+#include "kg_common.cuh"
+
+namespace svdq {
+
+template <int R>
+struct KGF4Smem {
+  static constexpr int STAGES = R >= 128 ? 5 : 6;
+  static constexpr int A_BYTES = KG_BM * 64;   // 128 rows x 64 B (128 E2M1)
+  static constexpr int B_BYTES = KG_BN * 64;   // 256 rows x 64 B
+  static constexpr int SFA_BYTES = 2 * 512;    // 2 k-blocks x one 128-row atom
+  static constexpr int SFB_BYTES = 2 * 2 * 512;  // 2 atoms (256 rows) x 2 k-blocks
+  static constexpr int STAGE = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int LR_CHUNKS = R > 0 ? (2 * R + 63) / 64 : 0;
+  static constexpr int ALR_OFF = STAGES * STAGE;
+  static constexpr int BAR_OFF = ALR_OFF + LR_CHUNKS * 16384;
+  static constexpr int TOTAL = BAR_OFF + 256 + 1024;
+  // tensor memory columns
+  static constexpr int SFA_COL = 256;
+  static constexpr int SFB_COL = 256 + 8 * STAGES;
+};
+
+template <int R>
+__global__ void __launch_bounds__(KG_THREADS, 1)
+    kg_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                    const __grid_constant__ CUtensorMap tm_blr, KGParams p) {
+  using S = KGF4Smem<R>;
+  constexpr int NST = S::STAGES;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+  const uint32_t bar_full = smem_u32(bars);
+  const uint32_t bar_empty = smem_u32(bars + NST);
+  const uint32_t bar_acc_full = smem_u32(bars + 2 * NST);
+  const uint32_t bar_acc_empty = smem_u32(bars + 2 * NST + 1);
+  const uint32_t bar_lr_full = smem_u32(bars + 2 * NST + 2);
+  const uint32_t bar_drain = smem_u32(bars + 2 * NST + 3);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NST + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Guard guard{p.err, abort_flag, p.timeout_ns};
+  const int num_tiles = p.num_m * p.num_n;
+  const int nks = p.K / 128;          // pipeline stages per tile (128 K each)
+  const int kblk = p.K / 64;          // scale atoms along K
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_acc_full, 1);
+    mbar_init(bar_acc_empty, KG_EPI_WARPS);
+    mbar_init(bar_lr_full, KG_EPI_WARPS);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_b);
+      if (R > 0) tma_prefetch_desc(&tm_blr);
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
+        const int mb = tile % p.num_m, nb = tile / p.num_m;
+        for (int ks = 0; ks < nks; ++ks) {
+          if (!(ok = wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x201))) break;
+          issued &= ~(1u << s);
+          if (!((p.debug_mask & 1u) && j == 0 && ks == 1)) {  // test hook: leave one stage empty
+            const uint32_t st = sbase + s * S::STAGE;
+            const uint32_t fb = bar_full + 8 * s;
+            mbar_expect_tx(fb, S::STAGE);
+            tma_load_2d(st, &tm_a, fb, ks * 64, mb * KG_BM);
+            tma_load_2d(st + S::A_BYTES, &tm_b, fb, ks * 64, nb * KG_BN);
+            bulk_load(st + S::A_BYTES + S::B_BYTES,
+                      p.sfa + (static_cast<size_t>(mb) * kblk + 2 * ks) * 512, 1024, fb);
+            const uint8_t* sfb0 = p.sfb + (static_cast<size_t>(2 * nb) * kblk + 2 * ks) * 512;
+            bulk_load(st + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, sfb0, 1024, fb);
+            bulk_load(st + S::A_BYTES + S::B_BYTES + S::SFA_BYTES + 1024,
+                      sfb0 + static_cast<size_t>(kblk) * 512, 1024, fb);
+            issued |= 1u << s;
+            issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          }
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+        for (int l = 0; l < R / 16 && ok; ++l) {
+          if (!(ok = wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x202))) break;
+          issued &= ~(1u << s);
+          const uint32_t fb = bar_full + 8 * s;
+          mbar_expect_tx(fb, KG_BN * 64);
+          tma_load_2d(sbase + s * S::STAGE + S::A_BYTES, &tm_blr, fb, l * 32, nb * KG_BN);
+          issued |= 1u << s;
+          issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+      }
+      if (*abort_flag) drain_loads(bar_full, issued, issued_par, NST, p.timeout_ns);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t id_f4 = idesc_nvf4(KG_BM, KG_BN);
+      constexpr uint32_t id_bf = idesc_bf16_f32(KG_BM, KG_BN);
+      const uint32_t alr = sbase + S::ALR_OFF;
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
+        if (j > 0 && !(ok = wait_bounded(bar_acc_empty, (j - 1) & 1, guard, 0x203))) break;
+        tc_fence_after();
+        for (int ks = 0; ks < nks; ++ks) {
+          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x204))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + s * S::STAGE;
+          const uint32_t sfa_s = st + S::A_BYTES + S::B_BYTES;
+          const uint32_t sfb_s = sfa_s + S::SFA_BYTES;
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+            const uint32_t ca = S::SFA_COL + (2 * s + kb) * 4;
+            const uint32_t cb = S::SFB_COL + (2 * s + kb) * 8;
+            tmem_cp_32x128b_warpx4(tmem + ca, smem_desc(sfa_s + kb * 512, 0, 128, SWZ_NONE));
+            tmem_cp_32x128b_warpx4(tmem + cb, smem_desc(sfb_s + kb * 512, 0, 128, SWZ_NONE));
+            tmem_cp_32x128b_warpx4(tmem + cb + 4, smem_desc(sfb_s + 1024 + kb * 512, 0, 128, SWZ_NONE));
+          }
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+            const uint64_t a = smem_desc(st + kb * 32, 16, 512, SWZ_64B);
+            const uint64_t b = smem_desc(st + S::A_BYTES + kb * 32, 16, 512, SWZ_64B);
+            mma_nvf4(tmem, a, b, id_f4, tmem + S::SFA_COL + (2 * s + kb) * 4,
+                     tmem + S::SFB_COL + (2 * s + kb) * 8, (ks | kb) != 0);
+          }
+          tc_commit(bar_empty + 8 * s);
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        if (R > 0) {
+          if (!(ok = wait_bounded(bar_lr_full, j & 1, guard, 0x205))) break;
+          tc_fence_after();
+          for (int l = 0; l < R / 16; ++l) {
+            if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x206))) break;
+            tc_fence_after();
+            const uint32_t bst = sbase + s * S::STAGE + S::A_BYTES;
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int kk = 2 * l + k2;
+              const uint64_t a = smem_desc(alr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, SWZ_128B);
+              const uint64_t b = smem_desc(bst + k2 * 32, 16, 512, SWZ_64B);
+              mma_bf16(tmem, a, b, id_bf, 1);
+            }
+            tc_commit(bar_empty + 8 * s);
+            if (++s == NST) { s = 0; ph ^= 1; }
+          }
+          if (!ok) break;
+        }
+        tc_commit(bar_acc_full);
+      }
+      // drain: every MMA issued so far has completed before tensor memory is freed
+      tc_commit(bar_drain);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < p.timeout_ns) {
+      }
+    }
+  } else if (warp >= 4) {
+    // ----------------------------------------------------------------- epilogue
+    const int e = warp - 4;
+    const int q = warp & 3;        // tensor-memory lane group of this warp
+    const int cs = e >> 2;         // 64-column slice
+    const int row = q * 32 + lane;
+    const int etid = threadIdx.x - 128;
+    uint8_t* alr = smem + S::ALR_OFF;
+    if constexpr (R > 0) {
+      if (static_cast<int>(blockIdx.x) < num_tiles) {
+        prep_lowrank_a<R>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_lr_full);
+      }
+    }
+    for (int tile = blockIdx.x, j = 0; tile < num_tiles; tile += gridDim.x, ++j) {
+      const int mb = tile % p.num_m, nb = tile / p.num_m;
+      if (!wait_bounded(bar_acc_full, j & 1, guard, 0x207)) break;
+      tc_fence_after();
+      uint32_t v[64];
+      const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + cs * 64;
+      tmem_ld_x32(ta, v);
+      tmem_ld_x32(ta + 32, v + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acc_empty);
+      if constexpr (R > 0) {
+        const int next = tile + gridDim.x;
+        if (next < num_tiles) {
+          prep_lowrank_a<R>(alr, p.t, (next % p.num_m) * KG_BM, p.M, etid);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_lr_full);
+        }
+      }
+      store_row64(p, mb * KG_BM + row, nb * KG_BN + cs * 64, reinterpret_cast<const float*>(v));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace svdq

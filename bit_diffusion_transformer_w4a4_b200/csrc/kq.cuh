@@ -1,0 +1,398 @@
+// Kernel 1 of the layer: activation smoothing, per-token group quantisation
+// to 4 bits with packing, and the rank-r down projection T = X' L1 computed
+// from the same shared-memory tiles on the tensor cores.
+//
+// Method: "Problemas do Nunchaku Qwen e como corrigi-los em 2025"
+// (apatero.com), section "O que e Nunchaku e como acelera modelos Qwen" --
+// the down projection is fused with the quantisation kernel so both branches
+// share the activations; "Nunchaku Lite ... integrated into Diffusers"
+// (axbrief.com), section "The Mechanics of 4-Bit Efficiency and SVDQuant" --
+// activation outliers are divided out (moved into the weights) before the
+// 4-bit quantisation.
+//
+// CTA tile: 128 tokens x (K / ksplit) input channels.  The K range of a row
+// block is split over a cluster of `ksplit` CTAs so that a 4608-token layer
+// still fills the 148 SMs; their partial T tiles are summed through
+// distributed shared memory in a fixed order (deterministic).
+//
+// Warp roles (320 threads):
+//   warps 0-7  quantisers, one token row per thread; warp w covers rows
+//              32*(w%4).. and every second 64-column chunk (parity w/4)
+//   warp 8     TMA producer (X chunk [128 x 64] bf16 + L1^T chunk [r x 64])
+//   warp 9     tcgen05 MMA issuer and tensor-memory owner
+#pragma once
+
+#include "ptx.cuh"
+
+namespace svdq {
+
+constexpr int KQ_THREADS = 320;
+constexpr int KQ_QWARPS = 8;
+constexpr int KQ_STAGES = 4;
+constexpr int KQ_CHUNK = 64;  // columns per pipeline stage
+
+// Correctly rounded x / s for s > 0 finite: one correction step of
+// Markstein's division method (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 1990):
+// with y = RN(1/s), q0 = RN(x*y), the residual r = x - s*q0 is exact in one
+// fma and q1 = RN(q0 + r*y) is the correctly rounded quotient.  The kernels
+// only divide bf16 values by bf16 / E4M3 scales; the library's self-test
+// compares this routine against IEEE division over all such operand pairs.
+__device__ __forceinline__ float div_by_scale(float x, float s, float y) {
+  const float q0 = __fmul_rn(x, y);
+  const float r = __fmaf_rn(-q0, s, x);
+  return __fmaf_rn(r, y, q0);
+}
+
+// E4M3 (satfinite, RN) of a non-negative fp32, and its exact value.
+__device__ __forceinline__ uint32_t e4m3_rn(float v) {
+  uint16_t h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(v));
+  return h & 0xFFu;
+}
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  uint32_t h2;
+  const uint16_t c = static_cast<uint16_t>(code);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+// Eight fp32 -> eight E2M1 codes (RN, satfinite), element 0 in the low nibble.
+__device__ __forceinline__ uint32_t e2m1x8(const float* v) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return out;
+}
+// Round half to even to an integer in [-8, 7], two's complement nibble.
+__device__ __forceinline__ uint32_t int4_rn(float v) {
+  v = fminf(fmaxf(v, -8.0f), 7.0f);
+  // adding 1.5 * 2^23 leaves the rounded integer in the low mantissa bits
+  return __float_as_uint(__fadd_rn(v, 12582912.0f)) & 0xFu;
+}
+
+struct KQParams {
+  const float* inv_lam;  // [K]
+  uint8_t* codes;        // [M x K/2]
+  void* scales;          // INT4: bf16 [M x K/64]; NVFP4: tiled E4M3
+  float* t;              // [M x R]
+  int M, K, ksplit, chunks;  // chunks of 64 columns per CTA
+  int* err;
+  uint32_t debug_mask;
+  uint64_t timeout_ns;
+};
+
+template <int VARIANT, int R>
+struct KQSmem {
+  static constexpr int X_BYTES = 128 * KQ_CHUNK * 2;  // 16 KB
+  static constexpr int L_BYTES = R * KQ_CHUNK * 2;    // r x 128 B
+  static constexpr int STAGE = X_BYTES + L_BYTES;
+  static constexpr int TP_BYTES = R > 0 ? 128 * R * 4 : 0;  // partial T for the cluster sum
+  static constexpr int BAR_OFF = KQ_STAGES * STAGE + TP_BYTES;
+  static constexpr int TOTAL = BAR_OFF + 256 + 1024;  // barriers + slack for 1 KB alignment
+};
+
+// VARIANT 0 = INT4 (G 64, bf16 scale, amax/7); 1 = NVFP4 (G 16, E4M3 scale, amax/6)
+template <int VARIANT, int R>
+__global__ void __launch_bounds__(KQ_THREADS, 1)
+    kq_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1t,
+              KQParams p) {
+  using S = KQSmem<VARIANT, R>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+  // barrier indices
+  const uint32_t bar_full = smem_u32(bars + 0);               // [STAGES]
+  const uint32_t bar_ready = smem_u32(bars + KQ_STAGES);      // [STAGES] X' written
+  const uint32_t bar_empty = smem_u32(bars + 2 * KQ_STAGES);  // [STAGES]
+  const uint32_t bar_tfull = smem_u32(bars + 3 * KQ_STAGES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * KQ_STAGES + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ks = blockIdx.x;            // K-split index (= rank in the cluster)
+  const int m0 = blockIdx.y * 128;
+  const int kbase = ks * p.chunks * KQ_CHUNK;
+  const Guard guard{p.err, abort_flag, p.timeout_ns};
+  constexpr uint32_t TMEM_COLS = R <= 32 ? 32 : R;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < KQ_STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_ready + 8 * s, 4);
+      mbar_init(bar_empty + 8 * s, R > 0 ? 1 : 4);
+    }
+    mbar_init(bar_tfull, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (R > 0 && warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = R > 0 ? *tmem_slot : 0;
+
+  if (warp == 8) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_x);
+      if (R > 0) tma_prefetch_desc(&tm_l1t);
+      uint32_t issued = 0, issued_par = 0;  // per-stage outstanding loads
+      for (int c = 0; c < p.chunks; ++c) {
+        const int s = c % KQ_STAGES;
+        const uint32_t ph = (c / KQ_STAGES) & 1;
+        if (!wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x101)) break;
+        issued &= ~(1u << s);
+        if ((p.debug_mask & 2u) && c == 1) continue;  // test hook: never fill this stage
+        const uint32_t st = sbase + s * S::STAGE;
+        mbar_expect_tx(bar_full + 8 * s, S::STAGE);
+        tma_load_2d(st, &tm_x, bar_full + 8 * s, kbase + c * KQ_CHUNK, m0);
+        if (R > 0) tma_load_2d(st + S::X_BYTES, &tm_l1t, bar_full + 8 * s, kbase + c * KQ_CHUNK, 0);
+        issued |= 1u << s;
+        issued_par = (issued_par & ~(1u << s)) | (ph << s);
+      }
+      if (*abort_flag) {  // let copies still in flight land before the CTA exits
+        for (int s = 0; s < KQ_STAGES; ++s)
+          if (issued & (1u << s)) {
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar_full + 8 * s, (issued_par >> s) & 1) &&
+                   global_timer_ns() - t0 < p.timeout_ns) {
+            }
+          }
+      }
+    }
+  } else if (warp == 9) {
+    // --------------------------------------------------------------- MMA issue
+    if (R > 0 && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, R);
+      bool ok = true;
+      for (int c = 0; c < p.chunks && ok; ++c) {
+        const int s = c % KQ_STAGES;
+        const uint32_t ph = (c / KQ_STAGES) & 1;
+        ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x102) &&
+             wait_bounded(bar_ready + 8 * s, ph, guard, 0x103);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t st = sbase + s * S::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < KQ_CHUNK / 16; ++kk) {
+          const uint64_t a = smem_desc(st + kk * 32, 16, 1024, SWZ_128B);
+          const uint64_t b = smem_desc(st + S::X_BYTES + kk * 32, 16, 1024, SWZ_128B);
+          mma_bf16(tmem, a, b, idesc, (c | kk) != 0);
+        }
+        tc_commit(bar_empty + 8 * s);
+      }
+      tc_commit(bar_tfull);  // also serves as the drain point on the abort path
+      if (!ok) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar_tfull, 0) && global_timer_ns() - t0 < p.timeout_ns) {
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- quantise
+    const int q = warp & 3;
+    const int par = warp >> 2;
+    const int row = q * 32 + lane;
+    const int grow = m0 + row;
+    const bool live = grow < p.M;
+    const int kh = p.K / 2;
+    for (int c = par; c < p.chunks; c += 2) {
+      const int s = c % KQ_STAGES;
+      const uint32_t ph = (c / KQ_STAGES) & 1;
+      if (!wait_bounded(bar_full + 8 * s, ph, guard, 0x104)) break;
+      uint8_t* xt = smem + s * S::STAGE;
+      const int k0 = kbase + c * KQ_CHUNK;
+      // 64 bf16 of this row, de-swizzled
+      uint32_t w[32];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xt + swz_off(row, j, 128));
+        w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+      }
+      // x' = bf16(x * inv_lambda)
+      float xs[64];
+      const float4* il = reinterpret_cast<const float4*>(p.inv_lam + k0);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float4 f = __ldg(il + j);
+        const uint32_t w0 = w[2 * j], w1 = w[2 * j + 1];
+        const uint32_t o0 = pack_bf16x2(__fmul_rn(bf16lo(w0), f.x), __fmul_rn(bf16hi(w0), f.y));
+        const uint32_t o1 = pack_bf16x2(__fmul_rn(bf16lo(w1), f.z), __fmul_rn(bf16hi(w1), f.w));
+        w[2 * j] = o0;
+        w[2 * j + 1] = o1;
+        xs[4 * j] = bf16lo(o0); xs[4 * j + 1] = bf16hi(o0);
+        xs[4 * j + 2] = bf16lo(o1); xs[4 * j + 3] = bf16hi(o1);
+      }
+      if (R > 0) {
+        // X' replaces X in place: it is the A operand of the down projection
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(xt + swz_off(row, j, 128)) =
+              make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ready + 8 * s);
+      } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+      }
+      // group quantisation (all in registers)
+      uint32_t packed[8];
+      if (VARIANT == 1) {
+        uint32_t sc = 0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float a = 0.0f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(xs[16 * g + e]));
+          const uint32_t code = e4m3_rn(__fdiv_rn(a, 6.0f));
+          const float s_ = e4m3_value(code);
+          sc |= code << (8 * g);
+          float v[16];
+          if (s_ > 0.0f) {
+            const float y = __frcp_rn(s_);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = div_by_scale(xs[16 * g + e], s_, y);
+            packed[2 * g] = e2m1x8(v);
+            packed[2 * g + 1] = e2m1x8(v + 8);
+          } else {
+            packed[2 * g] = 0u;
+            packed[2 * g + 1] = 0u;
+          }
+        }
+        if (live) {
+          // tiled scale layout: 512-byte atom per (128-row block, 64-column block)
+          uint8_t* sp = reinterpret_cast<uint8_t*>(p.scales) +
+                        (static_cast<size_t>(blockIdx.y) * (p.K / 64) + (k0 / 64)) * 512 +
+                        (row & 31) * 16 + (row >> 5) * 4;
+          *reinterpret_cast<uint32_t*>(sp) = sc;
+        }
+      } else {
+        float a = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) a = fmaxf(a, fabsf(xs[e]));
+        const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(a, 7.0f));
+        const float s_ = __bfloat162float(sb);
+        if (s_ > 0.0f) {
+          const float y = __frcp_rn(s_);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint32_t pk = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              pk |= int4_rn(div_by_scale(xs[8 * j + e], s_, y)) << (4 * e);
+            packed[j] = pk;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) packed[j] = 0u;
+        }
+        if (live)
+          reinterpret_cast<__nv_bfloat16*>(p.scales)[static_cast<size_t>(grow) * (p.K / 64) +
+                                                     k0 / 64] = sb;
+      }
+      if (live) {
+        uint4* cp = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(grow) * kh + k0 / 2);
+        cp[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        cp[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      }
+    }
+  }
+
+  // ------------------------------------------------------- T = X' L1 epilogue
+  if constexpr (R > 0) {
+    float* tp = reinterpret_cast<float*>(smem + KQ_STAGES * S::STAGE);
+    const bool reader = warp < 4;  // one warp per 32-lane group of tensor memory
+    if (reader) {
+      const int row = warp * 32 + lane;
+      const bool ok = wait_bounded(bar_tfull, 0, guard, 0x105);
+      uint32_t v[R];
+      if (ok) {
+        tc_fence_after();
+        const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        if constexpr (R == 16) {
+          tmem_ld_x16(ta, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < R / 32; ++j) tmem_ld_x32(ta + 32 * j, v + 32 * j);
+        }
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int j = 0; j < R; ++j) v[j] = 0u;
+      }
+      if (p.ksplit == 1) {
+        const int grow = m0 + row;
+        if (ok && grow < p.M) {
+          float4* dst = reinterpret_cast<float4*>(p.t + static_cast<size_t>(grow) * R);
+#pragma unroll
+          for (int j = 0; j < R / 4; ++j)
+            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        }
+      } else {
+        // stage the partial tile; rotate the 16-byte column blocks per row to
+        // spread the shared-memory banks
+#pragma unroll
+        for (int j = 0; j < R / 4; ++j) {
+          const int jj = (j + row) % (R / 4);
+          reinterpret_cast<float4*>(tp + row * R)[jj] =
+              make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                          __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        }
+      }
+    }
+    if (p.ksplit > 1) {
+      // all CTAs of the cluster have their partial T in shared memory
+      asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                       : "memory");
+      // CTA `ks` sums rows [ks*rows_per, (ks+1)*rows_per) over the cluster, in rank order
+      const int rows_per = 128 / p.ksplit;
+      const int items = rows_per * (R / 4);
+      for (int it = threadIdx.x; it < items; it += KQ_THREADS) {
+        const int rr = ks * rows_per + it / (R / 4);
+        const int j = it % (R / 4);
+        const int jj = (j + rr) % (R / 4);
+        const uint32_t local = smem_u32(tp + rr * R + 4 * jj);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int src = 0; src < p.ksplit; ++src) {
+          uint32_t ra;
+          asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local), "r"(src));
+          float4 f;
+          asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w)
+                       : "r"(ra)
+                       : "memory");
+          acc.x += f.x; acc.y += f.y; acc.z += f.z; acc.w += f.w;
+        }
+        const int grow = m0 + rr;
+        if (grow < p.M && !*abort_flag)
+          reinterpret_cast<float4*>(p.t + static_cast<size_t>(grow) * R)[j] = acc;
+      }
+      // keep this CTA's shared memory alive until every peer has read it
+      asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                       : "memory");
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (R > 0 && warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace svdq

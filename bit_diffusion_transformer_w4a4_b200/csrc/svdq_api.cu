@@ -1,0 +1,562 @@
+// Host side of libsvdq: argument validation, weight re-tiling at load,
+// TMA tensor maps, kernel launches and device-status reporting.
+// The C declarations and their documentation live in include/svdq.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/svdq.h"
+#include "kg_int4.cuh"
+#include "kg_nvfp4.cuh"
+#include "kq.cuh"
+
+using namespace svdq;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+
+#define SVDQ_TRY(expr)                                              \
+  do {                                                              \
+    cudaError_t e_ = (expr);                                        \
+    if (e_ != cudaSuccess) return e_ == cudaErrorMemoryAllocation   \
+                               ? SVDQ_ERR_OOM : SVDQ_ERR_CUDA;      \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+svdq_status check_device(int* dev_out, int* sms_out) {
+  int dev = 0, n = 0;
+  if (cudaGetDeviceCount(&n) != cudaSuccess || n == 0) {
+    cudaGetLastError();
+    return SVDQ_ERR_UNSUPPORTED_DEVICE;
+  }
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+  int major = 0, minor = 0, sms = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // the 4-bit tensor-core kernels are built for sm_100a only
+  if (major != 10 || minor != 0) return SVDQ_ERR_UNSUPPORTED_DEVICE;
+  if (dev_out) *dev_out = dev;
+  if (sms_out) *sms_out = sms;
+  return SVDQ_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D tiled tensor map over a row-major [rows x cols] matrix.
+svdq_status make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_bytes,
+                      uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+                      CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return SVDQ_ERR_CUDA;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+template <class K>
+svdq_status set_smem(K kernel, int bytes) {
+  SVDQ_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+struct svdq_weights {
+  svdq_variant variant;
+  int64_t K, N, r, max_M, npad;
+  uint32_t flags;
+  int device, sms;
+  // device weights (library-owned)
+  float* inv_lam = nullptr;
+  uint16_t* l1t = nullptr;     // [r x K]
+  uint16_t* l2dup = nullptr;   // [N x 2r]
+  uint8_t* wcodes = nullptr;   // NVFP4 [N x K/2] packed; INT4 [N x K] int8
+  uint8_t* wscales = nullptr;  // NVFP4 tiled E4M3; INT4 fp32 [K/64 x npad]
+  uint16_t* bias = nullptr;
+  // forward workspace (sized for max_M)
+  uint8_t* ws_codes = nullptr;
+  uint8_t* ws_scales = nullptr;
+  float* ws_t = nullptr;
+  // host-call staging
+  void* x_dev = nullptr;
+  void* y_dev = nullptr;
+  int* err = nullptr;
+  uint32_t debug_mask = 0;
+  uint64_t timeout_ns = kDefaultTimeoutNs;
+  CUtensorMap tm_b, tm_blr, tm_l1t;
+  // per-call maps, cached by (pointer, M)
+  CUtensorMap tm_x, tm_a;
+  const void* tm_x_ptr = nullptr;
+  const void* tm_a_ptr = nullptr;
+  int64_t tm_x_M = -1, tm_a_M = -1;
+};
+
+namespace {
+
+int group_of(svdq_variant v) { return v == SVDQ_INT4_G64_BF16 ? 64 : 16; }
+
+size_t act_scale_bytes(const svdq_weights* h, int64_t M) {
+  if (h->variant == SVDQ_INT4_G64_BF16) return static_cast<size_t>(M) * (h->K / 64) * 2;
+  return static_cast<size_t>(cdiv(M, 128) * 128) * (h->K / 16);
+}
+
+void free_all(svdq_weights* h) {
+  void* ptrs[] = {h->inv_lam, h->l1t, h->l2dup, h->wcodes, h->wscales, h->bias, h->ws_codes,
+                  h->ws_scales, h->ws_t, h->x_dev, h->y_dev, h->err};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+}
+
+// ------------------------------------------------------------------ launches
+template <int V, int R>
+svdq_status launch_kq_t(svdq_weights* h, const CUtensorMap& tmx, int64_t M, uint8_t* codes,
+                        void* scales, float* t, cudaStream_t st) {
+  using S = KQSmem<V, R>;
+  static bool attr = false;
+  if (!attr) {
+    svdq_status s = set_smem(kq_kernel<V, R>, S::TOTAL);
+    if (s != SVDQ_OK) return s;
+    attr = true;
+  }
+  const int num_m = static_cast<int>(cdiv(M, 128));
+  const int kch = static_cast<int>(h->K / 64);
+  int ksplit = 1;
+  while (ksplit < 8 && num_m * ksplit * 2 <= h->sms && kch % (ksplit * 2) == 0) ksplit *= 2;
+  KQParams p;
+  p.inv_lam = h->inv_lam;
+  p.codes = codes;
+  p.scales = scales;
+  p.t = t;
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(h->K);
+  p.ksplit = ksplit;
+  p.chunks = kch / ksplit;
+  p.err = h->err;
+  p.debug_mask = h->debug_mask;
+  p.timeout_ns = h->timeout_ns;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ksplit, num_m, 1);
+  cfg.blockDim = dim3(KQ_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = S::TOTAL;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  if (R > 0 && ksplit > 1) {
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = ksplit;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+  }
+  SVDQ_TRY(cudaLaunchKernelEx(&cfg, kq_kernel<V, R>, tmx, h->tm_l1t, p));
+  return SVDQ_OK;
+}
+
+template <int V>
+svdq_status launch_kq_v(svdq_weights* h, const CUtensorMap& tmx, int64_t M, uint8_t* codes,
+                        void* scales, float* t, cudaStream_t st) {
+  switch (h->r) {
+    case 0: return launch_kq_t<V, 0>(h, tmx, M, codes, scales, t, st);
+    case 16: return launch_kq_t<V, 16>(h, tmx, M, codes, scales, t, st);
+    case 32: return launch_kq_t<V, 32>(h, tmx, M, codes, scales, t, st);
+    case 64: return launch_kq_t<V, 64>(h, tmx, M, codes, scales, t, st);
+    case 128: return launch_kq_t<V, 128>(h, tmx, M, codes, scales, t, st);
+  }
+  return SVDQ_ERR_SHAPE;
+}
+
+template <int V, int R>
+svdq_status launch_kg_t(svdq_weights* h, const CUtensorMap& tma, int64_t M, const uint8_t* sfa,
+                        const float* t, void* y, cudaStream_t st) {
+  const int smem = V == 1 ? KGF4Smem<R>::TOTAL : KGI4Smem<R>::TOTAL;
+  auto kern = V == 1 ? kg_nvfp4_kernel<R> : kg_int4_kernel<R>;
+  static bool attr = false;
+  if (!attr) {
+    svdq_status s = set_smem(kern, smem);
+    if (s != SVDQ_OK) return s;
+    attr = true;
+  }
+  KGParams p;
+  p.sfa = sfa;
+  p.sfb = h->wscales;
+  p.t = t;
+  p.bias = h->bias;
+  p.y = static_cast<uint16_t*>(y);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(h->N);
+  p.K = static_cast<int>(h->K);
+  p.num_m = static_cast<int>(cdiv(M, KG_BM));
+  p.num_n = static_cast<int>(cdiv(h->N, KG_BN));
+  p.gelu = (h->flags & SVDQ_EPI_GELU) ? 1 : 0;
+  p.err = h->err;
+  p.debug_mask = h->debug_mask;
+  p.timeout_ns = h->timeout_ns;
+  const int tiles = p.num_m * p.num_n;
+  const int grid = tiles < h->sms ? tiles : h->sms;
+  kern<<<grid, KG_THREADS, smem, st>>>(tma, h->tm_b, h->tm_blr, p);
+  SVDQ_TRY(cudaGetLastError());
+  return SVDQ_OK;
+}
+
+template <int V>
+svdq_status launch_kg_v(svdq_weights* h, const CUtensorMap& tma, int64_t M, const uint8_t* sfa,
+                        const float* t, void* y, cudaStream_t st) {
+  switch (h->r) {
+    case 0: return launch_kg_t<V, 0>(h, tma, M, sfa, t, y, st);
+    case 16: return launch_kg_t<V, 16>(h, tma, M, sfa, t, y, st);
+    case 32: return launch_kg_t<V, 32>(h, tma, M, sfa, t, y, st);
+    case 64: return launch_kg_t<V, 64>(h, tma, M, sfa, t, y, st);
+    case 128: return launch_kg_t<V, 128>(h, tma, M, sfa, t, y, st);
+  }
+  return SVDQ_ERR_SHAPE;
+}
+
+svdq_status get_tm_x(svdq_weights* h, const void* x, int64_t M) {
+  if (h->tm_x_ptr == x && h->tm_x_M == M) return SVDQ_OK;
+  svdq_status s = make_tmap(&h->tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->K, M, 64, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SVDQ_OK) return s;
+  h->tm_x_ptr = x;
+  h->tm_x_M = M;
+  return SVDQ_OK;
+}
+
+svdq_status get_tm_a(svdq_weights* h, const void* codes, int64_t M) {
+  if (h->tm_a_ptr == codes && h->tm_a_M == M) return SVDQ_OK;
+  svdq_status s =
+      h->variant == SVDQ_NVFP4_G16_E4M3
+          ? make_tmap(&h->tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h->K / 2, M, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_64B)
+          : make_tmap(&h->tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h->K / 2, M, 32, 128,
+                      CU_TENSOR_MAP_SWIZZLE_32B);
+  if (s != SVDQ_OK) return s;
+  h->tm_a_ptr = codes;
+  h->tm_a_M = M;
+  return SVDQ_OK;
+}
+
+svdq_status check_call(svdq_weights* h, int64_t M) {
+  if (!h) return SVDQ_ERR_INVALID_ARG;
+  if (M < 1 || M > h->max_M || M > (1ll << 30)) return SVDQ_ERR_SHAPE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (dev != h->device) return SVDQ_ERR_INVALID_ARG;
+  return SVDQ_OK;
+}
+
+// ------------------------------------------------------------- self-test
+// Exhaustive comparison of the quantiser's division routine against IEEE
+// division over every bf16 dividend and every positive finite scale of the
+// variant (E4M3: 126 values; bf16: 32639 values).
+__global__ void selftest_div_kernel(int variant, unsigned long long* mismatches) {
+  const uint32_t sidx = blockIdx.x + 1;  // 1 .. number of positive finite scales
+  float s;
+  if (variant == 1) s = e4m3_value(sidx);
+  else s = __uint_as_float(sidx << 16);
+  const float y = __frcp_rn(s);
+  unsigned long long bad = 0;
+  for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
+    const float x = __uint_as_float(xb << 16);
+    if (!isfinite(x)) continue;
+    const float a = div_by_scale(x, s, y);
+    const float b = __fdiv_rn(x, s);
+    if (__float_as_uint(a) != __float_as_uint(b)) ++bad;
+  }
+  if (bad) atomicAdd(mismatches, bad);
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* svdq_status_string(svdq_status s) {
+  switch (s) {
+    case SVDQ_OK: return "SVDQ_OK";
+    case SVDQ_ERR_INVALID_ARG: return "SVDQ_ERR_INVALID_ARG";
+    case SVDQ_ERR_SHAPE: return "SVDQ_ERR_SHAPE";
+    case SVDQ_ERR_ALIGNMENT: return "SVDQ_ERR_ALIGNMENT";
+    case SVDQ_ERR_UNSUPPORTED_DEVICE: return "SVDQ_ERR_UNSUPPORTED_DEVICE";
+    case SVDQ_ERR_OOM: return "SVDQ_ERR_OOM";
+    case SVDQ_ERR_CUDA: return "SVDQ_ERR_CUDA";
+    case SVDQ_ERR_DEVICE_TIMEOUT: return "SVDQ_ERR_DEVICE_TIMEOUT";
+  }
+  return "SVDQ_ERR_UNKNOWN";
+}
+
+const char* svdq_version(void) { return "svdq 0.1.0 sm_100a"; }
+
+svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, void* stream) {
+  if (!d || !out) return SVDQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (d->variant != SVDQ_INT4_G64_BF16 && d->variant != SVDQ_NVFP4_G16_E4M3) return SVDQ_ERR_INVALID_ARG;
+  if (d->flags & ~SVDQ_EPI_GELU) return SVDQ_ERR_INVALID_ARG;
+  const int64_t K = d->K, N = d->N, r = d->r;
+  if (K < 128 || K % 128 != 0 || K > (1 << 20)) return SVDQ_ERR_SHAPE;
+  if (N < 16 || N % 16 != 0 || N > (1 << 20)) return SVDQ_ERR_SHAPE;
+  if (!(r == 0 || r == 16 || r == 32 || r == 64 || r == 128)) return SVDQ_ERR_SHAPE;
+  if (d->max_M < 1 || d->max_M > (1ll << 30)) return SVDQ_ERR_SHAPE;
+  if (!d->lambda || !d->w_codes || !d->w_scales) return SVDQ_ERR_INVALID_ARG;
+  if (r > 0 && (!d->L1 || !d->L2)) return SVDQ_ERR_INVALID_ARG;
+  for (int64_t k = 0; k < K; ++k)
+    if (!(d->lambda[k] > 0.0f) || !(d->lambda[k] < INFINITY)) return SVDQ_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  svdq_status ds = check_device(&dev, &sms);
+  if (ds != SVDQ_OK) return ds;
+
+  svdq_weights* h = new (std::nothrow) svdq_weights();
+  if (!h) return SVDQ_ERR_OOM;
+  h->variant = d->variant;
+  h->K = K;
+  h->N = N;
+  h->r = r;
+  h->max_M = d->max_M;
+  h->npad = cdiv(N, 256) * 256;
+  h->flags = d->flags;
+  h->device = dev;
+  h->sms = sms;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = group_of(d->variant);
+
+  auto fail = [&](svdq_status s) {
+    cudaStreamSynchronize(st);
+    free_all(h);
+    delete h;
+    return s;
+  };
+  auto dmalloc = [&](void** p, size_t bytes) -> bool {
+    if (cudaMalloc(p, bytes < 256 ? 256 : bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    return true;
+  };
+
+  // ---- host-side re-layout (load time only)
+  std::vector<float> inv(K);
+  for (int64_t k = 0; k < K; ++k) inv[k] = 1.0f / d->lambda[k];  // IEEE fp32 division
+  std::vector<uint16_t> l1t(static_cast<size_t>(r) * K), l2dup(static_cast<size_t>(N) * 2 * r);
+  for (int64_t k = 0; k < K; ++k)
+    for (int64_t j = 0; j < r; ++j) l1t[j * K + k] = d->L1[k * r + j];
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t j = 0; j < r; ++j) {
+      const uint16_t v = d->L2[j * N + n];
+      l2dup[n * 2 * r + j] = v;
+      l2dup[n * 2 * r + r + j] = v;
+    }
+  std::vector<uint8_t> codes, scales;
+  if (d->variant == SVDQ_NVFP4_G16_E4M3) {
+    codes.assign(d->w_codes, d->w_codes + static_cast<size_t>(N) * (K / 2));
+    scales.assign(static_cast<size_t>(h->npad) * (K / 16), 0);
+    const uint8_t* sc = static_cast<const uint8_t*>(d->w_scales);
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t b = 0; b < K / 16; ++b) {
+        const size_t off = (static_cast<size_t>(n / 128) * (K / 64) + b / 4) * 512 +
+                           (n % 32) * 16 + ((n / 32) % 4) * 4 + (b % 4);
+        scales[off] = sc[n * (K / 16) + b];
+      }
+  } else {
+    codes.resize(static_cast<size_t>(N) * K);
+    for (size_t i = 0; i < static_cast<size_t>(N) * (K / 2); ++i) {
+      const uint8_t b = d->w_codes[i];
+      codes[2 * i] = static_cast<uint8_t>(static_cast<int8_t>(static_cast<uint8_t>(b << 4)) >> 4);
+      codes[2 * i + 1] = static_cast<uint8_t>(static_cast<int8_t>(b) >> 4);
+    }
+    scales.assign(static_cast<size_t>(K / 64) * h->npad * 4, 0);
+    float* sf = reinterpret_cast<float*>(scales.data());
+    const uint16_t* sc = static_cast<const uint16_t*>(d->w_scales);
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t g = 0; g < K / 64; ++g) {
+        const uint32_t bits = static_cast<uint32_t>(sc[n * (K / 64) + g]) << 16;
+        float f;
+        std::memcpy(&f, &bits, 4);
+        sf[g * h->npad + n] = f;
+      }
+  }
+
+  // ---- device allocations and copies
+  if (!dmalloc(reinterpret_cast<void**>(&h->inv_lam), K * 4) ||
+      !dmalloc(reinterpret_cast<void**>(&h->wcodes), codes.size()) ||
+      !dmalloc(reinterpret_cast<void**>(&h->wscales), scales.size()) ||
+      !dmalloc(reinterpret_cast<void**>(&h->err), 256) ||
+      !dmalloc(reinterpret_cast<void**>(&h->ws_codes), static_cast<size_t>(h->max_M) * (K / 2)) ||
+      !dmalloc(reinterpret_cast<void**>(&h->ws_scales), act_scale_bytes(h, h->max_M)))
+    return fail(SVDQ_ERR_OOM);
+  if (r > 0 && (!dmalloc(reinterpret_cast<void**>(&h->l1t), l1t.size() * 2) ||
+                !dmalloc(reinterpret_cast<void**>(&h->l2dup), l2dup.size() * 2) ||
+                !dmalloc(reinterpret_cast<void**>(&h->ws_t), static_cast<size_t>(h->max_M) * r * 4)))
+    return fail(SVDQ_ERR_OOM);
+  if (d->bias && !dmalloc(reinterpret_cast<void**>(&h->bias), N * 2)) return fail(SVDQ_ERR_OOM);
+
+  // synchronous copies: the host vectors go out of scope on return
+  if (cudaMemcpy(h->inv_lam, inv.data(), K * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(h->wcodes, codes.data(), codes.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(h->wscales, scales.data(), scales.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemset(h->err, 0, 256) != cudaSuccess)
+    return fail(SVDQ_ERR_CUDA);
+  if (r > 0 && (cudaMemcpy(h->l1t, l1t.data(), l1t.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess ||
+                cudaMemcpy(h->l2dup, l2dup.data(), l2dup.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess))
+    return fail(SVDQ_ERR_CUDA);
+  if (d->bias && cudaMemcpy(h->bias, d->bias, N * 2, cudaMemcpyHostToDevice) != cudaSuccess)
+    return fail(SVDQ_ERR_CUDA);
+
+  // ---- weight-side tensor maps
+  svdq_status s = d->variant == SVDQ_NVFP4_G16_E4M3
+                      ? make_tmap(&h->tm_b, h->wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N,
+                                  64, 256, CU_TENSOR_MAP_SWIZZLE_64B)
+                      : make_tmap(&h->tm_b, h->wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, 64,
+                                  256, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (s != SVDQ_OK) return fail(s);
+  if (r > 0) {
+    if ((s = make_tmap(&h->tm_blr, h->l2dup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * r, N, 32, 256,
+                       CU_TENSOR_MAP_SWIZZLE_64B)) != SVDQ_OK)
+      return fail(s);
+    if ((s = make_tmap(&h->tm_l1t, h->l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, r, 64,
+                       static_cast<uint32_t>(r), CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return fail(s);
+  } else {
+    h->tm_blr = h->tm_b;  // never read when r == 0
+    h->tm_l1t = h->tm_b;
+  }
+  (void)G;
+  *out = h;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_weights_free(svdq_weights_t h) {
+  if (!h) return SVDQ_OK;
+  cudaDeviceSynchronize();
+  free_all(h);
+  delete h;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_act_scales_bytes(svdq_weights_t h, int64_t M, size_t* bytes) {
+  if (!h || !bytes || M < 0) return SVDQ_ERR_INVALID_ARG;
+  *bytes = act_scale_bytes(h, M);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_quantize_act_lowrank_down(svdq_weights_t h, const void* x, int64_t M,
+                                           uint8_t* act_codes, void* act_scales, float* t,
+                                           void* stream) {
+  svdq_status s = check_call(h, M);
+  if (s != SVDQ_OK) return s;
+  if (!x || !act_codes || !act_scales || (h->r > 0 && !t)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(act_codes) || !aligned16(act_scales) || (t && !aligned16(t)))
+    return SVDQ_ERR_ALIGNMENT;
+  if ((s = get_tm_x(h, x, M)) != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return h->variant == SVDQ_NVFP4_G16_E4M3
+             ? launch_kq_v<1>(h, h->tm_x, M, act_codes, act_scales, t, st)
+             : launch_kq_v<0>(h, h->tm_x, M, act_codes, act_scales, t, st);
+}
+
+svdq_status svdq_w4a4_gemm_lowrank_up(svdq_weights_t h, const uint8_t* act_codes,
+                                      const void* act_scales, const float* t, int64_t M, void* y,
+                                      void* stream) {
+  svdq_status s = check_call(h, M);
+  if (s != SVDQ_OK) return s;
+  if (!act_codes || !act_scales || !y || (h->r > 0 && !t)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(y) || (t && !aligned16(t)))
+    return SVDQ_ERR_ALIGNMENT;
+  if ((s = get_tm_a(h, act_codes, M)) != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint8_t* sfa = static_cast<const uint8_t*>(act_scales);
+  return h->variant == SVDQ_NVFP4_G16_E4M3 ? launch_kg_v<1>(h, h->tm_a, M, sfa, t, y, st)
+                                           : launch_kg_v<0>(h, h->tm_a, M, sfa, t, y, st);
+}
+
+svdq_status svdq_linear_forward(svdq_weights_t h, const void* x, void* y, int64_t M, void* stream) {
+  svdq_status s = svdq_quantize_act_lowrank_down(h, x, M, h ? h->ws_codes : nullptr,
+                                                 h ? h->ws_scales : nullptr, h ? h->ws_t : nullptr,
+                                                 stream);
+  if (s != SVDQ_OK) return s;
+  return svdq_w4a4_gemm_lowrank_up(h, h->ws_codes, h->ws_scales, h->ws_t, M, y, stream);
+}
+
+svdq_status svdq_linear_forward_host(svdq_weights_t h, const void* x_host, void* y_host, int64_t M,
+                                     void* stream) {
+  svdq_status s = check_call(h, M);
+  if (s != SVDQ_OK) return s;
+  if (!x_host || !y_host) return SVDQ_ERR_INVALID_ARG;
+  if (!h->x_dev) {
+    if (cudaMalloc(&h->x_dev, static_cast<size_t>(h->max_M) * h->K * 2) != cudaSuccess ||
+        cudaMalloc(&h->y_dev, static_cast<size_t>(h->max_M) * h->N * 2) != cudaSuccess) {
+      cudaGetLastError();
+      return SVDQ_ERR_OOM;
+    }
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SVDQ_TRY(cudaMemcpyAsync(h->x_dev, x_host, static_cast<size_t>(M) * h->K * 2,
+                           cudaMemcpyHostToDevice, st));
+  if ((s = svdq_linear_forward(h, h->x_dev, h->y_dev, M, stream)) != SVDQ_OK) return s;
+  SVDQ_TRY(cudaMemcpyAsync(y_host, h->y_dev, static_cast<size_t>(M) * h->N * 2,
+                           cudaMemcpyDeviceToHost, st));
+  return SVDQ_OK;
+}
+
+svdq_status svdq_device_status(svdq_weights_t h, void* stream) {
+  if (!h) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SVDQ_ERR_CUDA;
+  int e = 0;
+  if (cudaMemcpy(&e, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (e != 0) {
+    cudaMemset(h->err, 0, sizeof(int));
+    return SVDQ_ERR_DEVICE_TIMEOUT;
+  }
+  return SVDQ_OK;
+}
+
+svdq_status svdq_debug_set_fault(svdq_weights_t h, uint32_t mask, uint32_t timeout_us) {
+  if (!h || (mask & ~3u)) return SVDQ_ERR_INVALID_ARG;
+  h->debug_mask = mask;
+  h->timeout_ns = timeout_us ? static_cast<uint64_t>(timeout_us) * 1000ull : kDefaultTimeoutNs;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_selftest_division(int variant, unsigned long long* mismatches) {
+  if (!mismatches || (variant != 0 && variant != 1)) return SVDQ_ERR_INVALID_ARG;
+  svdq_status ds = check_device(nullptr, nullptr);
+  if (ds != SVDQ_OK) return ds;
+  unsigned long long* d = nullptr;
+  SVDQ_TRY(cudaMalloc(&d, sizeof(unsigned long long)));
+  cudaMemset(d, 0, sizeof(unsigned long long));
+  // E4M3: codes 1..126 are the positive finite scales; bf16: 0x0001..0x7F7F
+  const int nscales = variant == 1 ? 126 : 0x7F7F;
+  selftest_div_kernel<<<nscales, 256>>>(variant, d);
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(mismatches, d, sizeof(unsigned long long), cudaMemcpyDeviceToHost);
+  cudaFree(d);
+  return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,205 @@
+"""Python binding of libsvdq (include/svdq.h) -- argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; this module only
+converts numpy / torch buffers into pointers, passes the current CUDA stream
+and raises on non-OK status codes.  There is no CPU fallback: if the shared
+library is missing or the device is not an sm_100 GPU, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+INT4 = 0
+NVFP4 = 1
+EPI_GELU = 1
+
+STATUS = {
+    0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_SHAPE", 3: "SVDQ_ERR_ALIGNMENT",
+    4: "SVDQ_ERR_UNSUPPORTED_DEVICE", 5: "SVDQ_ERR_OOM", 6: "SVDQ_ERR_CUDA",
+    7: "SVDQ_ERR_DEVICE_TIMEOUT",
+}
+
+EXPORTED = [
+    "svdq_weights_load", "svdq_weights_free", "svdq_act_scales_bytes",
+    "svdq_quantize_act_lowrank_down", "svdq_w4a4_gemm_lowrank_up", "svdq_linear_forward",
+    "svdq_linear_forward_host", "svdq_device_status", "svdq_debug_set_fault",
+    "svdq_selftest_division", "svdq_status_string", "svdq_version",
+]
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+class WeightDesc(ctypes.Structure):
+    _fields_ = [
+        ("variant", ctypes.c_int),
+        ("K", ctypes.c_int64), ("N", ctypes.c_int64), ("r", ctypes.c_int64),
+        ("max_M", ctypes.c_int64),
+        ("flags", ctypes.c_uint32),
+        ("lam", ctypes.c_void_p), ("L1", ctypes.c_void_p), ("L2", ctypes.c_void_p),
+        ("w_codes", ctypes.c_void_p), ("w_scales", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+    ]
+
+
+_LIB = None
+
+
+def lib(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libsvdq.so (building it first when absent or stale)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = _build.LIB
+    if build_if_missing and _build.stale():
+        _build.build()
+    if not os.path.exists(path):
+        raise OSError(f"libsvdq.so not found at {path}; run python -m "
+                      "bit_diffusion_transformer_w4a4_b200.build")
+    L = ctypes.CDLL(path)
+    vp, i64, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    L.svdq_weights_load.argtypes = [ctypes.POINTER(WeightDesc), ctypes.POINTER(vp), vp]
+    L.svdq_weights_free.argtypes = [vp]
+    L.svdq_act_scales_bytes.argtypes = [vp, i64, ctypes.POINTER(ctypes.c_size_t)]
+    L.svdq_quantize_act_lowrank_down.argtypes = [vp, vp, i64, vp, vp, vp, vp]
+    L.svdq_w4a4_gemm_lowrank_up.argtypes = [vp, vp, vp, vp, i64, vp, vp]
+    L.svdq_linear_forward.argtypes = [vp, vp, vp, i64, vp]
+    L.svdq_linear_forward_host.argtypes = [vp, vp, vp, i64, vp]
+    L.svdq_device_status.argtypes = [vp, vp]
+    L.svdq_debug_set_fault.argtypes = [vp, ctypes.c_uint32, ctypes.c_uint32]
+    L.svdq_selftest_division.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_ulonglong)]
+    L.svdq_status_string.argtypes = [st]
+    L.svdq_status_string.restype = ctypes.c_char_p
+    L.svdq_version.restype = ctypes.c_char_p
+    for name in EXPORTED:
+        f = getattr(L, name)
+        if f.restype is None or f.restype is ctypes.c_int:
+            f.restype = st
+    _LIB = L
+    return L
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise SvdqError(code, where)
+
+
+def _ptr(a) -> int:
+    """Device or host address of a torch tensor / numpy array (None -> 0)."""
+    if a is None:
+        return 0
+    if isinstance(a, np.ndarray):
+        return a.ctypes.data
+    return a.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        if not torch.cuda.is_available():
+            return 0            # the library itself reports the missing device
+        return torch.cuda.current_stream().cuda_stream
+    return int(stream)
+
+
+def selftest_division(variant: int) -> int:
+    n = ctypes.c_ulonglong(0)
+    _check(lib().svdq_selftest_division(variant, ctypes.byref(n)), "svdq_selftest_division")
+    return int(n.value)
+
+
+class SVDQWeights:
+    """A loaded layer: owns a library handle (``svdq_weights_t``)."""
+
+    def __init__(self, pw, max_M: int, stream=None):
+        """``pw`` has fields variant, K, N, r, lam, L1, L2, codes, scales, bias, gelu
+        (host numpy arrays in the formats of ``svdq_weight_desc``)."""
+        self._keep = [np.ascontiguousarray(pw.lam, dtype=np.float32),
+                      np.ascontiguousarray(pw.L1, dtype=np.uint16),
+                      np.ascontiguousarray(pw.L2, dtype=np.uint16),
+                      np.ascontiguousarray(pw.codes, dtype=np.uint8),
+                      np.ascontiguousarray(pw.scales),
+                      None if pw.bias is None else np.ascontiguousarray(pw.bias, dtype=np.uint16)]
+        lam, L1, L2, codes, scales, bias = self._keep
+        self.variant, self.K, self.N, self.r = int(pw.variant), int(pw.K), int(pw.N), int(pw.r)
+        self.max_M = int(max_M)
+        self.gelu = bool(pw.gelu)
+        d = WeightDesc(self.variant, self.K, self.N, self.r, self.max_M,
+                       EPI_GELU if self.gelu else 0,
+                       _ptr(lam), _ptr(L1) if self.r else 0, _ptr(L2) if self.r else 0,
+                       _ptr(codes), _ptr(scales), _ptr(bias))
+        h = ctypes.c_void_p(0)
+        self._lib = lib()
+        _check(self._lib.svdq_weights_load(ctypes.byref(d), ctypes.byref(h), _stream(stream)),
+               "svdq_weights_load")
+        self.handle = h
+
+    @property
+    def G(self) -> int:
+        return 64 if self.variant == INT4 else 16
+
+    def act_scales_bytes(self, M: int) -> int:
+        n = ctypes.c_size_t(0)
+        _check(self._lib.svdq_act_scales_bytes(self.handle, M, ctypes.byref(n)), "svdq_act_scales_bytes")
+        return int(n.value)
+
+    # --------------------------------------------------------------- the calls
+    def quantize_act_lowrank_down(self, x, M, act_codes, act_scales, t, stream=None):
+        _check(self._lib.svdq_quantize_act_lowrank_down(
+            self.handle, _ptr(x), int(M), _ptr(act_codes), _ptr(act_scales), _ptr(t),
+            _stream(stream)), "svdq_quantize_act_lowrank_down")
+
+    def w4a4_gemm_lowrank_up(self, act_codes, act_scales, t, M, y, stream=None):
+        _check(self._lib.svdq_w4a4_gemm_lowrank_up(
+            self.handle, _ptr(act_codes), _ptr(act_scales), _ptr(t), int(M), _ptr(y),
+            _stream(stream)), "svdq_w4a4_gemm_lowrank_up")
+
+    def linear_forward(self, x, y, M, stream=None):
+        _check(self._lib.svdq_linear_forward(self.handle, _ptr(x), _ptr(y), int(M), _stream(stream)),
+               "svdq_linear_forward")
+
+    def linear_forward_host(self, x_host, y_host, M, stream=None):
+        _check(self._lib.svdq_linear_forward_host(self.handle, _ptr(x_host), _ptr(y_host), int(M),
+                                                  _stream(stream)), "svdq_linear_forward_host")
+
+    def device_status(self, stream=None) -> int:
+        return int(self._lib.svdq_device_status(self.handle, _stream(stream)))
+
+    def debug_set_fault(self, mask: int, timeout_us: int) -> None:
+        _check(self._lib.svdq_debug_set_fault(self.handle, mask, timeout_us), "svdq_debug_set_fault")
+
+    # ------------------------------------------------------- torch conveniences
+    def alloc_act(self, M: int, device="cuda"):
+        """Allocate (codes, scales, t) device buffers for M tokens."""
+        import torch
+        codes = torch.empty((M, self.K // 2), dtype=torch.uint8, device=device)
+        scales = torch.empty(self.act_scales_bytes(M), dtype=torch.uint8, device=device)
+        t = torch.empty((M, max(self.r, 1)), dtype=torch.float32, device=device)
+        return codes, scales, t
+
+    def close(self) -> None:
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            self._lib.svdq_weights_free(self.handle)
+            self.handle = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def untile_nvfp4_scales(buf: np.ndarray, M: int, K: int) -> np.ndarray:
+    """Tensor-core tiled E4M3 activation scales -> canonical [M x K/16]."""
+    buf = np.asarray(buf, dtype=np.uint8)
+    m = np.arange(M)[:, None]
+    b = np.arange(K // 16)[None, :]
+    off = ((m // 128) * (K // 64) + b // 4) * 512 + (m % 32) * 16 + ((m // 32) % 4) * 4 + b % 4
+    return buf[off]

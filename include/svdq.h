@@ -1,0 +1,197 @@
+/*
+ * svdq.h -- C ABI of libsvdq, the SVDQuant W4A4 linear layer with its 16-bit
+ * low-rank branch, for NVIDIA B200 (sm_100a).
+ *
+ *     Y = (X diag(lambda)^-1) L1 L2  +  Q4(X diag(lambda)^-1) Q4(R),
+ *     R = diag(lambda) W - L1 L2.
+ *
+ * What the layer computes is described in "Nunchaku Lite: the 50% VRAM
+ * reduction now integrated into Diffusers" (axbrief.com), section "The
+ * Mechanics of 4-Bit Efficiency and SVDQuant": activation outliers are moved
+ * into the weights, the weight is split into a 16-bit low-rank branch and a
+ * 4-bit residual, and the residual branch runs with 4-bit weights and 4-bit
+ * activations (W4A4).  The two-call structure (down projection inside the
+ * activation quantiser, up projection inside the 4-bit GEMM, both sharing the
+ * activations) follows "Problemas do Nunchaku Qwen e como corrigi-los em
+ * 2025" (apatero.com), section "O que e Nunchaku e como acelera modelos Qwen".
+ * The capability gate follows the Nunchaku Lite article, section "Hardware
+ * Specialization and the Compression Workflow".
+ *
+ * Conventions for every call:
+ *   - Pointers named *_host are host memory; every other data pointer is
+ *     device memory owned by the caller, unless stated otherwise.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *   - Work is enqueued asynchronously on `stream`; the return value reports
+ *     host-side validation and launch errors only.  Device-side failures
+ *     (a bounded wait that timed out) are recorded in the handle and
+ *     reported by svdq_device_status().
+ *   - There is no CPU fallback: on a machine without an sm_100 GPU every
+ *     compute call returns SVDQ_ERR_UNSUPPORTED_DEVICE or SVDQ_ERR_CUDA.
+ *   - A handle must not be used on two streams at the same time.
+ *
+ * Shapes: M tokens, K in-features, N out-features, r rank.
+ *   K % 128 == 0, N % 16 == 0, r in {0, 16, 32, 64, 128}, 1 <= M <= max_M.
+ *   Rows beyond M inside the last 128-row tile are never written.
+ *
+ * Formats (all row-major, K contiguous):
+ *   bf16 values are passed as their 16-bit patterns (uint16_t).
+ *   4-bit codes: two per byte, element 2j in the low nibble.
+ *     INT4 : two's complement -8..7, group G = 64 along K, bf16 scales.
+ *     NVFP4: E2M1 (sign bit 3, magnitude index 0..7 = 0,0.5,1,1.5,2,3,4,6),
+ *            group G = 16 along K, E4M3 scale bytes.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* null pointer, bad enum, bad flag */
+  SVDQ_ERR_SHAPE = 2,              /* M/K/N/r outside the supported set */
+  SVDQ_ERR_ALIGNMENT = 3,          /* a device pointer is not 16-byte aligned */
+  SVDQ_ERR_UNSUPPORTED_DEVICE = 4, /* no CUDA device, or not compute capability 10.x */
+  SVDQ_ERR_OOM = 5,                /* device allocation failed */
+  SVDQ_ERR_CUDA = 6,               /* any other CUDA runtime / driver error */
+  SVDQ_ERR_DEVICE_TIMEOUT = 7      /* a kernel's bounded wait expired */
+} svdq_status;
+
+typedef enum {
+  SVDQ_INT4_G64_BF16 = 0,   /* INT4 codes, group 64, bf16 scales */
+  SVDQ_NVFP4_G16_E4M3 = 1   /* E2M1 codes, group 16, E4M3 scales */
+} svdq_variant;
+
+/* svdq_weight_desc.flags */
+#define SVDQ_EPI_GELU 1u    /* apply GELU (tanh form) in the GEMM epilogue */
+
+typedef struct svdq_weights* svdq_weights_t;   /* opaque, library-owned */
+
+/*
+ * Pre-packed layer weights, all HOST memory, read only during
+ * svdq_weights_load (the library copies what it needs).
+ *   lambda   fp32 [K]        smoothing factors (> 0); the library stores
+ *                            fp32(1 / lambda) for the runtime multiply
+ *   L1       bf16 [K x r]    low-rank down factor
+ *   L2       bf16 [r x N]    low-rank up factor
+ *   w_codes  u8   [N x K/2]  residual codes, one row per output feature
+ *   w_scales INT4: bf16 [N x K/64]; NVFP4: E4M3 bytes [N x K/16]
+ *   bias     bf16 [N] or NULL
+ * L1 / L2 may be NULL when r == 0.
+ */
+typedef struct {
+  svdq_variant variant;
+  int64_t K, N, r, max_M;
+  uint32_t flags;
+  const float* lambda;
+  const uint16_t* L1;
+  const uint16_t* L2;
+  const uint8_t* w_codes;
+  const void* w_scales;
+  const uint16_t* bias;
+} svdq_weight_desc;
+
+/*
+ * Copy and re-tile the weights into library-owned device memory on the
+ * current device and size the forward workspace for max_M tokens.
+ * The weight scales of the NVFP4 variant are re-tiled into the tensor-core
+ * scale-factor layout; the INT4 residual codes are additionally kept as int8
+ * for the int8 tensor-core path.  On error *out is left NULL and nothing is
+ * allocated.
+ */
+svdq_status svdq_weights_load(const svdq_weight_desc* desc, svdq_weights_t* out, void* stream);
+
+/* Free a handle (NULL is a no-op).  Synchronises the device first. */
+svdq_status svdq_weights_free(svdq_weights_t h);
+
+/*
+ * Size in bytes of the activation-scale buffer for M tokens:
+ *   INT4 : M * (K/64) * 2          canonical [M x K/64] bf16
+ *   NVFP4: ceil(M/128)*128 * (K/16) the tensor-core tiled layout (below)
+ */
+svdq_status svdq_act_scales_bytes(svdq_weights_t h, int64_t M, size_t* bytes);
+
+/*
+ * Kernel 1: smooth, quantise and pack the activations, and compute the
+ * rank-r down projection from the same tiles.
+ *   x          bf16 [M x K]
+ *   act_codes  u8   [M x K/2]  (written)
+ *   act_scales see svdq_act_scales_bytes (written).  NVFP4 layout: 128-row
+ *              tiles; inside tile b, K-block j (64 elements = 4 scales) of
+ *              row m sits at byte
+ *                b*(K/64)*512 + j*512 + (m%32)*16 + ((m/32)%4)*4 + (k/16)%4
+ *   t          fp32 [M x r]  T = X' L1 (written; untouched when r == 0)
+ * Per element (round to nearest even throughout):
+ *   x' = bf16(fp32(x) * inv_lambda);  a = max|x'| over the group;
+ *   INT4 s = bf16(a / 7), q = rint(x'/s);  NVFP4 s = e4m3_satfinite(a / 6),
+ *   q = e2m1_satfinite(x'/s);  s == 0 gives q = +0.  Divisions are IEEE
+ *   correctly rounded fp32.
+ */
+svdq_status svdq_quantize_act_lowrank_down(svdq_weights_t h, const void* x, int64_t M,
+                                           uint8_t* act_codes, void* act_scales, float* t,
+                                           void* stream);
+
+/*
+ * Kernel 2: the 4-bit GEMM on the packed residual with the low-rank up
+ * projection, optional bias and GELU fused into the epilogue.
+ *   act_codes, act_scales, t  as written by kernel 1 (t ignored when r == 0)
+ *   y  bf16 [M x N]  (written)
+ *   y = GELU?( sum_g s_x s_w sum_{k in g} q_x q_w  +  T L2  +  bias ),
+ *   accumulated in fp32, rounded once to bf16.
+ */
+svdq_status svdq_w4a4_gemm_lowrank_up(svdq_weights_t h, const uint8_t* act_codes,
+                                      const void* act_scales, const float* t, int64_t M,
+                                      void* y, void* stream);
+
+/* Both kernels back to back through the handle's workspace: y = layer(x). */
+svdq_status svdq_linear_forward(svdq_weights_t h, const void* x, void* y, int64_t M,
+                                void* stream);
+
+/*
+ * Same as svdq_linear_forward with HOST input and output (pinned memory is
+ * recommended): copies x_host to the device, runs the layer and copies y back
+ * on `stream`.  Returns after enqueueing; synchronise the stream before
+ * reading y_host.  Device staging buffers are owned by the handle.
+ */
+svdq_status svdq_linear_forward_host(svdq_weights_t h, const void* x_host, void* y_host,
+                                     int64_t M, void* stream);
+
+/*
+ * Synchronise `stream` and report device-side failures recorded by earlier
+ * calls on this handle (SVDQ_ERR_DEVICE_TIMEOUT), clearing the record.
+ */
+svdq_status svdq_device_status(svdq_weights_t h, void* stream);
+
+/*
+ * Test hook: make the next launches wait on a pipeline stage that is never
+ * filled (mask bit 0: GEMM producer skips one stage; bit 1: activation
+ * kernel producer skips one stage) and use `timeout_us` as the bounded-wait
+ * limit (0 restores the default of 2 s).  The kernels then return early and
+ * record SVDQ_ERR_DEVICE_TIMEOUT; no GPU fault is involved.
+ */
+svdq_status svdq_debug_set_fault(svdq_weights_t h, uint32_t mask, uint32_t timeout_us);
+
+/*
+ * Self-test of the activation quantiser's division: runs the kernels'
+ * correctly-rounded x / s routine against IEEE fp32 division for every bf16
+ * dividend and every positive finite scale of `variant` (0: bf16 scales,
+ * 1: E4M3 scales) on the current device, and stores the number of results
+ * that differ in *mismatches (0 expected).  Synchronises the device.
+ */
+svdq_status svdq_selftest_division(int variant, unsigned long long* mismatches);
+
+/* Human-readable name of a status code (static storage). */
+const char* svdq_status_string(svdq_status s);
+
+/* Library version, e.g. "svdq 0.1.0 sm_100a". */
+const char* svdq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

@@ -1,0 +1,96 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+symbol include/svdq.h declares, and host-side validation rejects bad calls
+before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from bit_diffusion_transformer_w4a4_b200 import svdq
+from bit_diffusion_transformer_w4a4_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "svdq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(svdq_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_header_symbol():
+    L = svdq.lib()
+    names = header_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(svdq.EXPORTED)
+
+
+def test_status_strings_and_version():
+    L = svdq.lib()
+    for code, name in svdq.STATUS.items():
+        assert L.svdq_status_string(code).decode() == name
+    assert b"sm_100a" in L.svdq_version()
+
+
+def _desc(**kw):
+    lay = W.Layer("t", M=64, K=256, N=128, r=16, variant=W.INT4, config_id=9)
+    pw = W.synthetic_packed(lay)
+    keep = [pw.lam, pw.L1, pw.L2, pw.codes, pw.scales]
+    d = svdq.WeightDesc(kw.get("variant", 0), kw.get("K", 256), kw.get("N", 128),
+                        kw.get("r", 16), kw.get("max_M", 64), kw.get("flags", 0),
+                        pw.lam.ctypes.data, pw.L1.ctypes.data, pw.L2.ctypes.data,
+                        pw.codes.ctypes.data, pw.scales.ctypes.data, 0)
+    return d, keep
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(variant=5), 1), (dict(flags=8), 1),
+    (dict(K=200), 2), (dict(K=64), 2), (dict(N=100), 2), (dict(r=24), 2), (dict(max_M=0), 2),
+])
+def test_load_validation(kw, code):
+    L = svdq.lib()
+    d, keep = _desc(**kw)
+    h = ctypes.c_void_p(0)
+    assert L.svdq_weights_load(ctypes.byref(d), ctypes.byref(h), None) == code
+    assert not h.value
+
+
+def test_null_arguments():
+    L = svdq.lib()
+    h = ctypes.c_void_p(0)
+    assert L.svdq_weights_load(None, ctypes.byref(h), None) == 1
+    d, keep = _desc()
+    assert L.svdq_weights_load(ctypes.byref(d), None, None) == 1
+    assert L.svdq_weights_free(None) == 0
+    assert L.svdq_linear_forward(None, None, None, 1, None) == 1
+    assert L.svdq_quantize_act_lowrank_down(None, None, 1, None, None, None, None) == 1
+    assert L.svdq_w4a4_gemm_lowrank_up(None, None, None, None, 1, None, None) == 1
+    assert L.svdq_device_status(None, None) == 1
+    assert L.svdq_debug_set_fault(None, 1, 10) == 1
+    n = ctypes.c_size_t(0)
+    assert L.svdq_act_scales_bytes(None, 1, ctypes.byref(n)) == 1
+
+
+def test_nonpositive_lambda_rejected():
+    L = svdq.lib()
+    d, keep = _desc()
+    keep[0][3] = 0.0
+    h = ctypes.c_void_p(0)
+    assert L.svdq_weights_load(ctypes.byref(d), ctypes.byref(h), None) == 1
+
+
+def test_no_gpu_no_fallback():
+    """Without an sm_100 device the library refuses; nothing runs on the CPU."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    L = svdq.lib()
+    d, keep = _desc()
+    h = ctypes.c_void_p(0)
+    assert L.svdq_weights_load(ctypes.byref(d), ctypes.byref(h), None) == 4
+    n = ctypes.c_ulonglong(0)
+    assert L.svdq_selftest_division(1, ctypes.byref(n)) == 4

@@ -1,0 +1,136 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle
+on the same seeded inputs.  Needs an sm_100 GPU (marked gpu)."""
+import numpy as np
+import pytest
+
+from bit_diffusion_transformer_w4a4_b200 import svdq
+from bit_diffusion_transformer_w4a4_b200 import workloads as W
+from oracle import forward as O
+from oracle import prep as P
+import parity as PT
+
+pytestmark = pytest.mark.gpu
+INT4, NVFP4 = W.INT4, W.NVFP4
+
+
+def _prepped(M, K, N, r, variant, gelu=False, with_bias=False, seed=0, cid=50):
+    lay = W.Layer("t", M=M, K=K, N=N, r=r, variant=variant, gelu=gelu, bias=with_bias,
+                  config_id=cid, layer_id=K // 64 + N + r)
+    x = W.activations(lay, seed)
+    w = W.weight(lay, seed)
+    pw = P.prepare(x, w, r, variant, bias_bits=W.bias(lay, seed), gelu=gelu)
+    return lay, x, pw
+
+
+@pytest.mark.parametrize("variant", [INT4, NVFP4])
+def test_division_selftest_exhaustive(variant):
+    assert svdq.selftest_division(variant) == 0
+
+
+@pytest.mark.parametrize("variant", [INT4, NVFP4])
+@pytest.mark.parametrize("r", [0, 16, 32, 64, 128])
+@pytest.mark.parametrize("M,K", [(200, 512), (64, 256), (1, 128), (384, 1024)])
+def test_activation_kernel(variant, r, M, K):
+    lay, x, pw = _prepped(M, K, 256, r, variant)
+    h = svdq.SVDQWeights(pw, M)
+    got = PT.gpu_forward(h, x, M)
+    inv = (np.float32(1) / pw.lam).astype(np.float32)
+    codes, scales, T = O.quantize_act_lowrank_down(x, inv, pw.L1, variant)
+    PT.check_act(got, {"codes": codes, "scales": scales, "T": T}, r=r, label=f"v{variant} r{r} M{M} K{K}")
+
+
+@pytest.mark.parametrize("variant", [INT4, NVFP4])
+@pytest.mark.parametrize("r", [0, 16, 32, 128])
+def test_gemm_isolated(variant, r):
+    """Kernel 2 alone, fed the oracle's activation codes / scales / T."""
+    import torch
+    M, K, N = 300, 512, 512
+    lay, x, pw = _prepped(M, K, N, r, variant)
+    inv = (np.float32(1) / pw.lam).astype(np.float32)
+    codes, scales, T = O.quantize_act_lowrank_down(x, inv, pw.L1, variant)
+    y_ref, Y_ref = O.gemm_lowrank_up(codes, scales, T, pw.codes, pw.scales, pw.L2, variant)
+    h = svdq.SVDQWeights(pw, M)
+    sc = PT.tile_nvfp4_scales(scales, M, K) if variant == NVFP4 else scales.view(np.uint8).reshape(-1)
+    tt = np.zeros((M, max(r, 1)), dtype=np.float32)
+    tt[:, :r] = T
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    h.w4a4_gemm_lowrank_up(PT.to_dev(codes), PT.to_dev(sc), PT.to_dev(tt), M, y)
+    torch.cuda.synchronize()
+    assert h.device_status() == 0
+    Yg = PT.from_dev(y.view(torch.int16)).view(np.uint16)
+    PT.check_y(Yg, y_ref, Y_ref, label=f"gemm v{variant} r{r}")
+
+
+@pytest.mark.parametrize("variant", [INT4, NVFP4])
+@pytest.mark.parametrize("gelu,with_bias", [(False, False), (True, True), (False, True)])
+@pytest.mark.parametrize("M,K,N,r", [(300, 512, 448, 32), (129, 1024, 272, 16), (513, 384, 768, 64)])
+def test_forward_small(variant, gelu, with_bias, M, K, N, r):
+    """Ragged M and N (partial tiles), several K tiles, bias and GELU."""
+    lay, x, pw = _prepped(M, K, N, r, variant, gelu=gelu, with_bias=with_bias)
+    h = svdq.SVDQWeights(pw, M)
+    got = PT.gpu_forward(h, x, M)
+    ref = O.linear_forward(x, pw)
+    PT.check_act(got, ref, r=r, label="fwd")
+    PT.check_y(got["Y"], ref["y"], ref["Y"], label=f"fwd v{variant} M{M} N{N}")
+    # the fused entry point runs the same kernels: identical bits
+    got2 = PT.gpu_forward(h, x, M, two_calls=False)
+    assert np.array_equal(got2["Y"], got["Y"])
+
+
+def test_quantizer_edge_values():
+    """All-zero groups, tiny values whose sign survives rounding to zero, huge
+    outliers that saturate E4M3 scales, and exact ties."""
+    M, K, N, r = 128, 256, 256, 16
+    for variant in (INT4, NVFP4):
+        lay = W.Layer("edge", M=M, K=K, N=N, r=r, variant=variant, config_id=60)
+        pw = W.synthetic_packed(lay)
+        pw.lam[:] = 1.0
+        x = W.bf16_bits_to_f32(W.activations(lay)).copy()
+        x[0, :] = 0.0                              # every group zero -> scale 0
+        x[1, :] *= 1e-30                           # subnormal-ish scales
+        x[2, :16] = [-0.0, 0.0, -1e-3, 1e-3] * 4   # signed zeros / tiny
+        x[3, :] = 5000.0                           # NVFP4 scale saturates at 448
+        x[4, :64] = np.arange(64) * 0.25 - 8.0     # many exact ties
+        xb = W.to_bf16_bits(x)
+        h = svdq.SVDQWeights(pw, M)
+        got = PT.gpu_forward(h, xb, M)
+        ref = O.linear_forward(xb, pw)
+        PT.check_act(got, ref, r=r, label=f"edge v{variant}")
+
+
+@pytest.mark.parametrize("variant", [INT4, NVFP4])
+def test_host_entry_point_matches_device(variant):
+    import torch
+    M, K, N, r = 256, 512, 512, 32
+    lay = W.Layer("host", M=M, K=K, N=N, r=r, variant=variant, config_id=61)
+    pw = W.synthetic_packed(lay)
+    x = W.activations(lay)
+    h = svdq.SVDQWeights(pw, M)
+    dev = PT.gpu_forward(h, x, M, two_calls=False)
+    xh = torch.from_numpy(x.view(np.int16)).pin_memory()
+    yh = torch.empty((M, N), dtype=torch.int16).pin_memory()
+    h.linear_forward_host(xh, yh, M)
+    torch.cuda.synchronize()
+    assert np.array_equal(yh.numpy().view(np.uint16), dev["Y"])
+
+
+@pytest.mark.parametrize("variant", [INT4, NVFP4])
+@pytest.mark.parametrize("mask", [1, 2])
+def test_bounded_wait_reports_timeout(variant, mask):
+    """A pipeline stage that is never filled: the kernel's bounded wait expires,
+    the call reports SVDQ_ERR_DEVICE_TIMEOUT and the context stays usable."""
+    M, K, N, r = 256, 1024, 512, 32
+    lay = W.Layer("fault", M=M, K=K, N=N, r=r, variant=variant, config_id=62)
+    pw = W.synthetic_packed(lay)
+    x = W.activations(lay)
+    h = svdq.SVDQWeights(pw, M)
+    ok = PT.gpu_forward(h, x, M)
+    h.debug_set_fault(mask, 20000)                 # 20 ms limit
+    import torch
+    xd = PT.to_dev(x.view(np.int16)).view(torch.bfloat16)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    h.linear_forward(xd, y, M)
+    assert h.device_status() == 7                 # SVDQ_ERR_DEVICE_TIMEOUT
+    h.debug_set_fault(0, 0)
+    again = PT.gpu_forward(h, x, M)
+    assert np.array_equal(again["Y"], ok["Y"])
