@@ -81,14 +81,14 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_ready + 8 * s, 2);
+      mbar_init(bar_ready + 8 * s, 64);   // the 64 transform threads
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_gfull + 8 * b, 1);
       mbar_init(bar_gempty + 8 * b, KG_EPI_WARPS);
     }
-    mbar_init(bar_lr_full, KG_EPI_WARPS);
+    mbar_init(bar_lr_full, KG_EPI_WARPS * 32);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           tc_fence_after();
           for (int l = 0; l < R / 16; ++l) {
             if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x308))) break;
+            if (!(ok = wait_bounded(bar_ready + 8 * s, ph, guard, 0x30d))) break;
             tc_fence_after();
             const uint32_t bst = sbase + s * S::STAGE + S::APK_BYTES + S::A8_BYTES;
 #pragma unroll
@@ -222,12 +223,16 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           }
         }
         fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_ready + 8 * s);
+        mbar_arrive(bar_ready + 8 * s);
         if (++s == NST) { s = 0; ph ^= 1; }
       }
-      for (int l = 0; l < R / 16; ++l)
+      // low-rank stages carry only the B operand; still pass each one through
+      // the ready barrier so its phase stays in step with the stage ring
+      for (int l = 0; l < R / 16 && ok; ++l) {
+        if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x30c))) break;
+        mbar_arrive(bar_ready + 8 * s);
         if (++s == NST) { s = 0; ph ^= 1; }
+      }
     }
   } else {
     // ----------------------------------------------------------------- epilogue
@@ -244,8 +249,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       if (static_cast<int>(blockIdx.x) < num_tiles) {
         prep_lowrank_a<R>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid);
         fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_lr_full);
+        mbar_arrive(bar_lr_full);
       }
     }
     uint32_t gc = 0;
@@ -309,8 +313,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           // the low-rank MMAs of this tile have completed: reuse the operand buffer
           prep_lowrank_a<R>(alr, p.t, (next % p.num_m) * KG_BM, p.M, etid);
           fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_lr_full);
+          mbar_arrive(bar_lr_full);
         }
       }
       store_row64(p, gm, n_base, acc);

@@ -12,9 +12,12 @@
 // Qwen..." (apatero.com), section "O que e Nunchaku..." (up projection fused
 // into the 4-bit kernel).
 //
-// Persistent CTAs, one per SM, tile 128 x 256.  Warp roles (640 threads):
-//   warp 0      TMA producer: A/B code tiles (tensor maps, 64B swizzle) and
-//               the matching scale-factor atoms (bulk copies)
+// Persistent CTAs, one per SM, tile 128 x 256.  A pipeline stage holds KB
+// k-blocks of 64 elements: KB = 4 (128-byte rows, 128B swizzle) when shared
+// memory allows, KB = 2 (64-byte rows, 64B swizzle) for rank 128, whose
+// low-rank operand is larger.  Warp roles (640 threads):
+//   warp 0      TMA producer: A/B code tiles (tensor maps) and the matching
+//               scale-factor atoms (bulk copies)
 //   warp 1      MMA issuer: scale factors shared->tensor memory, block-scaled
 //               MMAs, then the low-rank bf16 MMAs; owns tensor memory
 //   warps 4-19  epilogue: drain the accumulator, prepare the next tile's
@@ -27,19 +30,26 @@ namespace svdq {
 
 template <int R>
 struct KGF4Smem {
-  static constexpr int STAGES = R >= 128 ? 5 : 6;
-  static constexpr int A_BYTES = KG_BM * 64;   // 128 rows x 64 B (128 E2M1)
-  static constexpr int B_BYTES = KG_BN * 64;   // 256 rows x 64 B
-  static constexpr int SFA_BYTES = 2 * 512;    // 2 k-blocks x one 128-row atom
-  static constexpr int SFB_BYTES = 2 * 2 * 512;  // 2 atoms (256 rows) x 2 k-blocks
+  static constexpr int KB = R >= 128 ? 2 : 4;           // 64-element k-blocks per stage
+  static constexpr int ROWB = 32 * KB;                  // bytes per operand row per stage
+  static constexpr uint32_t SWZ = KB == 4 ? SWZ_128B : SWZ_64B;
+  static constexpr uint32_t SBO = 8 * ROWB;             // 8-row core-matrix group stride
+  static constexpr int STAGES = KB == 4 ? 3 : 5;
+  static constexpr int A_BYTES = KG_BM * ROWB;
+  static constexpr int B_BYTES = KG_BN * ROWB;
+  static constexpr int SFA_BYTES = KB * 512;            // one 128-row atom per k-block
+  static constexpr int SFB_BYTES = 2 * KB * 512;        // two atoms (256 rows) per k-block
   static constexpr int STAGE = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int LR_CHUNKS = R > 0 ? (2 * R + 63) / 64 : 0;
+  static constexpr int LR_STEPS = R / 8;                // bf16 k-steps of 16 over [T_hi | T_lo]
+  static constexpr int LR_STAGES = (LR_STEPS + KB - 1) / KB;  // a stage row holds KB k-steps
   static constexpr int ALR_OFF = STAGES * STAGE;
   static constexpr int BAR_OFF = ALR_OFF + LR_CHUNKS * 16384;
   static constexpr int TOTAL = BAR_OFF + 256 + 1024;
-  // tensor memory columns
+  // tensor memory columns: accumulator [0, 256), then scale factors
   static constexpr int SFA_COL = 256;
-  static constexpr int SFB_COL = 256 + 8 * STAGES;
+  static constexpr int SFB_COL = 256 + 4 * KB * STAGES;
+  static_assert(SFB_COL + 8 * KB * STAGES <= 512, "tensor memory columns");
 };
 
 template <int R>
@@ -48,6 +58,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_blr, KGParams p) {
   using S = KGF4Smem<R>;
   constexpr int NST = S::STAGES;
+  constexpr int KB = S::KB;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -66,8 +77,8 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   const int lane = threadIdx.x & 31;
   const Guard guard{p.err, abort_flag, p.timeout_ns};
   const int num_tiles = p.num_m * p.num_n;
-  const int nks = p.K / 128;          // pipeline stages per tile (128 K each)
-  const int kblk = p.K / 64;          // scale atoms along K
+  const int kblk = p.K / 64;                // 64-element k-blocks (scale atoms) along K
+  const int nks = (kblk + KB - 1) / KB;     // pipeline stages per tile; the last may be partial
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -76,7 +87,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     }
     mbar_init(bar_acc_full, 1);
     mbar_init(bar_acc_empty, KG_EPI_WARPS);
-    mbar_init(bar_lr_full, KG_EPI_WARPS);
+    mbar_init(bar_lr_full, KG_EPI_WARPS * 32);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -107,26 +118,28 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           if (!((p.debug_mask & 1u) && j == 0 && ks == 1)) {  // test hook: leave one stage empty
             const uint32_t st = sbase + s * S::STAGE;
             const uint32_t fb = bar_full + 8 * s;
-            mbar_expect_tx(fb, S::STAGE);
-            tma_load_2d(st, &tm_a, fb, ks * 64, mb * KG_BM);
-            tma_load_2d(st + S::A_BYTES, &tm_b, fb, ks * 64, nb * KG_BN);
+            // k-blocks present in this stage; code columns past K are zero-filled
+            const uint32_t kv = min(KB, kblk - KB * ks);
+            mbar_expect_tx(fb, S::A_BYTES + S::B_BYTES + 3 * kv * 512);
+            tma_load_2d(st, &tm_a, fb, ks * S::ROWB, mb * KG_BM);
+            tma_load_2d(st + S::A_BYTES, &tm_b, fb, ks * S::ROWB, nb * KG_BN);
             bulk_load(st + S::A_BYTES + S::B_BYTES,
-                      p.sfa + (static_cast<size_t>(mb) * kblk + 2 * ks) * 512, 1024, fb);
-            const uint8_t* sfb0 = p.sfb + (static_cast<size_t>(2 * nb) * kblk + 2 * ks) * 512;
-            bulk_load(st + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, sfb0, 1024, fb);
-            bulk_load(st + S::A_BYTES + S::B_BYTES + S::SFA_BYTES + 1024,
-                      sfb0 + static_cast<size_t>(kblk) * 512, 1024, fb);
+                      p.sfa + (static_cast<size_t>(mb) * kblk + KB * ks) * 512, kv * 512, fb);
+            const uint8_t* sfb0 = p.sfb + (static_cast<size_t>(2 * nb) * kblk + KB * ks) * 512;
+            bulk_load(st + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, sfb0, kv * 512, fb);
+            bulk_load(st + S::A_BYTES + S::B_BYTES + S::SFA_BYTES + KB * 512,
+                      sfb0 + static_cast<size_t>(kblk) * 512, kv * 512, fb);
             issued |= 1u << s;
             issued_par = (issued_par & ~(1u << s)) | (ph << s);
           }
           if (++s == NST) { s = 0; ph ^= 1; }
         }
-        for (int l = 0; l < R / 16 && ok; ++l) {
+        for (int l = 0; l < S::LR_STAGES && ok; ++l) {
           if (!(ok = wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x202))) break;
           issued &= ~(1u << s);
           const uint32_t fb = bar_full + 8 * s;
-          mbar_expect_tx(fb, KG_BN * 64);
-          tma_load_2d(sbase + s * S::STAGE + S::A_BYTES, &tm_blr, fb, l * 32, nb * KG_BN);
+          mbar_expect_tx(fb, S::B_BYTES);
+          tma_load_2d(sbase + s * S::STAGE + S::A_BYTES, &tm_blr, fb, l * (S::ROWB / 2), nb * KG_BN);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == NST) { s = 0; ph ^= 1; }
@@ -152,20 +165,23 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           const uint32_t st = sbase + s * S::STAGE;
           const uint32_t sfa_s = st + S::A_BYTES + S::B_BYTES;
           const uint32_t sfb_s = sfa_s + S::SFA_BYTES;
+          const int kv = min(KB, kblk - KB * ks);
 #pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
-            const uint32_t ca = S::SFA_COL + (2 * s + kb) * 4;
-            const uint32_t cb = S::SFB_COL + (2 * s + kb) * 8;
+          for (int kb = 0; kb < KB; ++kb) {
+            if (kb >= kv) break;
+            const uint32_t ca = S::SFA_COL + (KB * s + kb) * 4;
+            const uint32_t cb = S::SFB_COL + (KB * s + kb) * 8;
             tmem_cp_32x128b_warpx4(tmem + ca, smem_desc(sfa_s + kb * 512, 0, 128, SWZ_NONE));
             tmem_cp_32x128b_warpx4(tmem + cb, smem_desc(sfb_s + kb * 512, 0, 128, SWZ_NONE));
-            tmem_cp_32x128b_warpx4(tmem + cb + 4, smem_desc(sfb_s + 1024 + kb * 512, 0, 128, SWZ_NONE));
+            tmem_cp_32x128b_warpx4(tmem + cb + 4, smem_desc(sfb_s + KB * 512 + kb * 512, 0, 128, SWZ_NONE));
           }
 #pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
-            const uint64_t a = smem_desc(st + kb * 32, 16, 512, SWZ_64B);
-            const uint64_t b = smem_desc(st + S::A_BYTES + kb * 32, 16, 512, SWZ_64B);
-            mma_nvf4(tmem, a, b, id_f4, tmem + S::SFA_COL + (2 * s + kb) * 4,
-                     tmem + S::SFB_COL + (2 * s + kb) * 8, (ks | kb) != 0);
+          for (int kb = 0; kb < KB; ++kb) {
+            if (kb >= kv) break;
+            const uint64_t a = smem_desc(st + kb * 32, 16, S::SBO, S::SWZ);
+            const uint64_t b = smem_desc(st + S::A_BYTES + kb * 32, 16, S::SBO, S::SWZ);
+            mma_nvf4(tmem, a, b, id_f4, tmem + S::SFA_COL + (KB * s + kb) * 4,
+                     tmem + S::SFB_COL + (KB * s + kb) * 8, (ks | kb) != 0);
           }
           tc_commit(bar_empty + 8 * s);
           if (++s == NST) { s = 0; ph ^= 1; }
@@ -174,16 +190,18 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         if (R > 0) {
           if (!(ok = wait_bounded(bar_lr_full, j & 1, guard, 0x205))) break;
           tc_fence_after();
-          for (int l = 0; l < R / 16; ++l) {
+          for (int l = 0; l < S::LR_STAGES; ++l) {
             if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x206))) break;
             tc_fence_after();
             const uint32_t bst = sbase + s * S::STAGE + S::A_BYTES;
 #pragma unroll
-            for (int k2 = 0; k2 < 2; ++k2) {
-              const int kk = 2 * l + k2;
-              const uint64_t a = smem_desc(alr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, SWZ_128B);
-              const uint64_t b = smem_desc(bst + k2 * 32, 16, 512, SWZ_64B);
-              mma_bf16(tmem, a, b, id_bf, 1);
+            for (int k2 = 0; k2 < KB; ++k2) {
+              const int kk = KB * l + k2;  // k-step over [T_hi | T_lo]
+              if (kk < S::LR_STEPS) {
+                const uint64_t a = smem_desc(alr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, SWZ_128B);
+                const uint64_t b = smem_desc(bst + k2 * 32, 16, S::SBO, S::SWZ);
+                mma_bf16(tmem, a, b, id_bf, 1);
+              }
             }
             tc_commit(bar_empty + 8 * s);
             if (++s == NST) { s = 0; ph ^= 1; }
@@ -210,13 +228,12 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       if (static_cast<int>(blockIdx.x) < num_tiles) {
         prep_lowrank_a<R>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid);
         fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_lr_full);
+        mbar_arrive(bar_lr_full);
       }
     }
     for (int tile = blockIdx.x, j = 0; tile < num_tiles; tile += gridDim.x, ++j) {
       const int mb = tile % p.num_m, nb = tile / p.num_m;
-      if (!wait_bounded(bar_acc_full, j & 1, guard, 0x207)) break;
+      if (!wait_bounded(bar_acc_full, j & 1, guard, 0x207, 128)) break;
       tc_fence_after();
       uint32_t v[64];
       const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + cs * 64;
@@ -231,8 +248,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         if (next < num_tiles) {
           prep_lowrank_a<R>(alr, p.t, (next % p.num_m) * KG_BM, p.M, etid);
           fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_lr_full);
+          mbar_arrive(bar_lr_full);
         }
       }
       store_row64(p, mb * KG_BM + row, nb * KG_BN + cs * 64, reinterpret_cast<const float*>(v));

@@ -11,24 +11,25 @@
 // 4-bit quantisation.
 //
 // CTA tile: 128 tokens x (K / ksplit) input channels.  The K range of a row
-// block is split over a cluster of `ksplit` CTAs so that a 4608-token layer
-// still fills the 148 SMs; their partial T tiles are summed through
-// distributed shared memory in a fixed order (deterministic).
+// block is split over `ksplit` CTAs so that a 4608-token layer still fills
+// the 148 SMs in one wave; their partial T tiles go to a scratch buffer and
+// the last CTA of the row block to finish sums them in split order
+// (deterministic), with a per-block arrival counter that it resets.
 //
-// Warp roles (320 threads):
-//   warps 0-7  quantisers, one token row per thread; warp w covers rows
-//              32*(w%4).. and every second 64-column chunk (parity w/4)
-//   warp 8     TMA producer (X chunk [128 x 64] bf16 + L1^T chunk [r x 64])
-//   warp 9     tcgen05 MMA issuer and tensor-memory owner
+// Warp roles (576 threads):
+//   warps 0-15 quantisers, one token row per thread; warp w covers rows
+//              32*(w%4).. and every fourth 64-column chunk (group w/4)
+//   warp 16    TMA producer (X chunk [128 x 64] bf16, L1^T chunk [r x 64],
+//              1/lambda of the chunk)
+//   warp 17    tcgen05 MMA issuer and tensor-memory owner
 #pragma once
 
 #include "ptx.cuh"
 
 namespace svdq {
 
-constexpr int KQ_THREADS = 320;
-constexpr int KQ_QWARPS = 8;
-constexpr int KQ_STAGES = 4;
+constexpr int KQ_QWARPS = 16;  // quantiser warps: 4 chunk groups x 4 row quarters
+constexpr int KQ_THREADS = (KQ_QWARPS + 2) * 32;
 constexpr int KQ_CHUNK = 64;  // columns per pipeline stage
 
 // Correctly rounded x / s for s > 0 finite: one correction step of
@@ -38,10 +39,23 @@ constexpr int KQ_CHUNK = 64;  // columns per pipeline stage
 // fma and q1 = RN(q0 + r*y) is the correctly rounded quotient.  The kernels
 // only divide bf16 values by bf16 / E4M3 scales; the library's self-test
 // compares this routine against IEEE division over all such operand pairs.
+// The correction step can turn -0 into +0; the quotient's sign is x's sign
+// (s > 0), so it is put back explicitly.  The residual x - s*q0 must not
+// underflow and 1/s must be a normal number: the caller divides groups whose
+// scale lies outside [2^-90, 2^126) exactly instead.
 __device__ __forceinline__ float div_by_scale(float x, float s, float y) {
   const float q0 = __fmul_rn(x, y);
   const float r = __fmaf_rn(-q0, s, x);
-  return __fmaf_rn(r, y, q0);
+  const float q1 = __fmaf_rn(r, y, q0);
+  return __uint_as_float(__float_as_uint(q1) | (__float_as_uint(x) & 0x80000000u));
+}
+constexpr float kMinFastScale = 8.07793567e-28f;     // 2^-90: smallest scale of the fast path
+constexpr float kMaxFastScale = 8.50705917e+37f;  // 2^126: above it 1/s is subnormal
+
+// x / s as the quantiser computes it: the one-step method for normal s,
+// IEEE division when s is subnormal (its reciprocal would overflow).
+__device__ __forceinline__ float quant_div(float x, float s, float y) {
+  return (s >= kMinFastScale && s < kMaxFastScale) ? div_by_scale(x, s, y) : __fdiv_rn(x, s);
 }
 
 // E4M3 (satfinite, RN) of a non-negative fp32, and its exact value.
@@ -81,6 +95,8 @@ struct KQParams {
   uint8_t* codes;        // [M x K/2]
   void* scales;          // INT4: bf16 [M x K/64]; NVFP4: tiled E4M3
   float* t;              // [M x R]
+  float* tpart;          // scratch: partial T tiles [ksplit x num_m x 128 x R] (ksplit > 1)
+  int* counters;         // scratch: arrivals per 128-row block, zero between launches
   int M, K, ksplit, chunks;  // chunks of 64 columns per CTA
   int* err;
   uint32_t debug_mask;
@@ -89,13 +105,19 @@ struct KQParams {
 
 template <int VARIANT, int R>
 struct KQSmem {
+  static constexpr int STAGES = R <= 32 ? 8 : (R == 64 ? 7 : 6);
   static constexpr int X_BYTES = 128 * KQ_CHUNK * 2;  // 16 KB
   static constexpr int L_BYTES = R * KQ_CHUNK * 2;    // r x 128 B
-  static constexpr int STAGE = X_BYTES + L_BYTES;
-  static constexpr int TP_BYTES = R > 0 ? 128 * R * 4 : 0;  // partial T for the cluster sum
-  static constexpr int BAR_OFF = KQ_STAGES * STAGE + TP_BYTES;
-  static constexpr int TOTAL = BAR_OFF + 256 + 1024;  // barriers + slack for 1 KB alignment
+  static constexpr int IL_BYTES = KQ_CHUNK * 4;       // 1/lambda for the chunk
+  static constexpr int STAGE = X_BYTES + L_BYTES + 1024;  // 1/lambda padded to keep 1 KB alignment
+  static constexpr int BAR_OFF = STAGES * STAGE;
+  static constexpr int TOTAL = BAR_OFF + 512 + 1024;  // barriers + slack for 1 KB alignment
 };
+
+// 1/6 and 1/7 rounded to nearest: scale = amax / 6 (NVFP4) or amax / 7 (INT4)
+// is computed with the same one-step division as the codes.
+constexpr float kRcp6 = 0.16666667163372039794921875f;
+constexpr float kRcp7 = 0.14285714924335479736328125f;
 
 // VARIANT 0 = INT4 (G 64, bf16 scale, amax/7); 1 = NVFP4 (G 16, E4M3 scale, amax/6)
 template <int VARIANT, int R>
@@ -103,38 +125,40 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
     kq_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1t,
               KQParams p) {
   using S = KQSmem<VARIANT, R>;
+  constexpr int NST = S::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
-  // barrier indices
-  const uint32_t bar_full = smem_u32(bars + 0);               // [STAGES]
-  const uint32_t bar_ready = smem_u32(bars + KQ_STAGES);      // [STAGES] X' written
-  const uint32_t bar_empty = smem_u32(bars + 2 * KQ_STAGES);  // [STAGES]
-  const uint32_t bar_tfull = smem_u32(bars + 3 * KQ_STAGES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * KQ_STAGES + 1);
+  const uint32_t bar_full = smem_u32(bars + 0);          // [NST]
+  const uint32_t bar_ready = smem_u32(bars + NST);       // [NST] X' written
+  const uint32_t bar_empty = smem_u32(bars + 2 * NST);   // [NST]
+  const uint32_t bar_tfull = smem_u32(bars + 3 * NST);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NST + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ks = blockIdx.x;            // K-split index (= rank in the cluster)
+  const int ks = blockIdx.x;            // K-split index
   const int m0 = blockIdx.y * 128;
   const int kbase = ks * p.chunks * KQ_CHUNK;
   const Guard guard{p.err, abort_flag, p.timeout_ns};
   constexpr uint32_t TMEM_COLS = R <= 32 ? 32 : R;
+  constexpr int PRODUCER = KQ_QWARPS;      // warp index of the TMA producer
+  constexpr int MMA = KQ_QWARPS + 1;       // warp index of the MMA issuer
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < KQ_STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_ready + 8 * s, 4);
-      mbar_init(bar_empty + 8 * s, R > 0 ? 1 : 4);
+      mbar_init(bar_ready + 8 * s, 128);              // the 128 quantiser threads of a chunk
+      mbar_init(bar_empty + 8 * s, R > 0 ? 1 : 128);
     }
     mbar_init(bar_tfull, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (R > 0 && warp == 9) {
+  if (R > 0 && warp == MMA) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
@@ -143,27 +167,29 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = R > 0 ? *tmem_slot : 0;
 
-  if (warp == 8) {
+  if (warp == PRODUCER) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_x);
       if (R > 0) tma_prefetch_desc(&tm_l1t);
       uint32_t issued = 0, issued_par = 0;  // per-stage outstanding loads
       for (int c = 0; c < p.chunks; ++c) {
-        const int s = c % KQ_STAGES;
-        const uint32_t ph = (c / KQ_STAGES) & 1;
+        const int s = c % NST;
+        const uint32_t ph = (c / NST) & 1;
         if (!wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x101)) break;
         issued &= ~(1u << s);
         if ((p.debug_mask & 2u) && c == 1) continue;  // test hook: never fill this stage
         const uint32_t st = sbase + s * S::STAGE;
-        mbar_expect_tx(bar_full + 8 * s, S::STAGE);
-        tma_load_2d(st, &tm_x, bar_full + 8 * s, kbase + c * KQ_CHUNK, m0);
-        if (R > 0) tma_load_2d(st + S::X_BYTES, &tm_l1t, bar_full + 8 * s, kbase + c * KQ_CHUNK, 0);
+        const int k0 = kbase + c * KQ_CHUNK;
+        mbar_expect_tx(bar_full + 8 * s, S::X_BYTES + S::L_BYTES + S::IL_BYTES);
+        tma_load_2d(st, &tm_x, bar_full + 8 * s, k0, m0);
+        if (R > 0) tma_load_2d(st + S::X_BYTES, &tm_l1t, bar_full + 8 * s, k0, 0);
+        bulk_load(st + S::X_BYTES + S::L_BYTES, p.inv_lam + k0, S::IL_BYTES, bar_full + 8 * s);
         issued |= 1u << s;
         issued_par = (issued_par & ~(1u << s)) | (ph << s);
       }
       if (*abort_flag) {  // let copies still in flight land before the CTA exits
-        for (int s = 0; s < KQ_STAGES; ++s)
+        for (int s = 0; s < NST; ++s)
           if (issued & (1u << s)) {
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(bar_full + 8 * s, (issued_par >> s) & 1) &&
@@ -172,14 +198,14 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
           }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == MMA) {
     // --------------------------------------------------------------- MMA issue
     if (R > 0 && lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, R);
       bool ok = true;
       for (int c = 0; c < p.chunks && ok; ++c) {
-        const int s = c % KQ_STAGES;
-        const uint32_t ph = (c / KQ_STAGES) & 1;
+        const int s = c % NST;
+        const uint32_t ph = (c / NST) & 1;
         ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x102) &&
              wait_bounded(bar_ready + 8 * s, ph, guard, 0x103);
         if (!ok) break;
@@ -203,38 +229,32 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
   } else {
     // ---------------------------------------------------------------- quantise
     const int q = warp & 3;
-    const int par = warp >> 2;
+    const int grp = warp >> 2;              // chunk group: chunks c with c % 4 == grp
     const int row = q * 32 + lane;
     const int grow = m0 + row;
     const bool live = grow < p.M;
     const int kh = p.K / 2;
-    for (int c = par; c < p.chunks; c += 2) {
-      const int s = c % KQ_STAGES;
-      const uint32_t ph = (c / KQ_STAGES) & 1;
+    for (int c = grp; c < p.chunks; c += KQ_QWARPS / 4) {
+      const int s = c % NST;
+      const uint32_t ph = (c / NST) & 1;
       if (!wait_bounded(bar_full + 8 * s, ph, guard, 0x104)) break;
       uint8_t* xt = smem + s * S::STAGE;
+      const float4* il = reinterpret_cast<const float4*>(xt + S::X_BYTES + S::L_BYTES);
       const int k0 = kbase + c * KQ_CHUNK;
-      // 64 bf16 of this row, de-swizzled
+      // 64 bf16 of this row (de-swizzled), smoothed: x' = bf16(x * inv_lambda)
       uint32_t w[32];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const uint4 v = *reinterpret_cast<const uint4*>(xt + swz_off(row, j, 128));
-        w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+        const float4 f0 = il[2 * j], f1 = il[2 * j + 1];
+        w[4 * j] = pack_bf16x2(__fmul_rn(bf16lo(v.x), f0.x), __fmul_rn(bf16hi(v.x), f0.y));
+        w[4 * j + 1] = pack_bf16x2(__fmul_rn(bf16lo(v.y), f0.z), __fmul_rn(bf16hi(v.y), f0.w));
+        w[4 * j + 2] = pack_bf16x2(__fmul_rn(bf16lo(v.z), f1.x), __fmul_rn(bf16hi(v.z), f1.y));
+        w[4 * j + 3] = pack_bf16x2(__fmul_rn(bf16lo(v.w), f1.z), __fmul_rn(bf16hi(v.w), f1.w));
       }
-      // x' = bf16(x * inv_lambda)
-      float xs[64];
-      const float4* il = reinterpret_cast<const float4*>(p.inv_lam + k0);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float4 f = __ldg(il + j);
-        const uint32_t w0 = w[2 * j], w1 = w[2 * j + 1];
-        const uint32_t o0 = pack_bf16x2(__fmul_rn(bf16lo(w0), f.x), __fmul_rn(bf16hi(w0), f.y));
-        const uint32_t o1 = pack_bf16x2(__fmul_rn(bf16lo(w1), f.z), __fmul_rn(bf16hi(w1), f.w));
-        w[2 * j] = o0;
-        w[2 * j + 1] = o1;
-        xs[4 * j] = bf16lo(o0); xs[4 * j + 1] = bf16hi(o0);
-        xs[4 * j + 2] = bf16lo(o1); xs[4 * j + 3] = bf16hi(o1);
-      }
+      // Each thread orders its own shared-memory accesses of this stage before
+      // the async proxy (tensor core or the TMA refill) touches it again, and
+      // arrives itself.
       if (R > 0) {
         // X' replaces X in place: it is the A operand of the down projection
 #pragma unroll
@@ -242,11 +262,10 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
           *reinterpret_cast<uint4*>(xt + swz_off(row, j, 128)) =
               make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
         fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_ready + 8 * s);
+        mbar_arrive(bar_ready + 8 * s);
       } else {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+        fence_proxy_async_smem();
+        mbar_arrive(bar_empty + 8 * s);
       }
       // group quantisation (all in registers)
       uint32_t packed[8];
@@ -256,17 +275,24 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
         for (int g = 0; g < 4; ++g) {
           float a = 0.0f;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(xs[16 * g + e]));
-          const uint32_t code = e4m3_rn(__fdiv_rn(a, 6.0f));
+          for (int e = 0; e < 8; ++e)
+            a = fmaxf(a, fmaxf(fabsf(bf16lo(w[8 * g + e])), fabsf(bf16hi(w[8 * g + e]))));
+          const uint32_t code = e4m3_rn(div_by_scale(a, 6.0f, kRcp6));
           const float s_ = e4m3_value(code);
           sc |= code << (8 * g);
-          float v[16];
-          if (s_ > 0.0f) {
+          if (s_ > 0.0f) {           // E4M3 scales are >= 2^-9: 1/s is finite
             const float y = __frcp_rn(s_);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = div_by_scale(xs[16 * g + e], s_, y);
-            packed[2 * g] = e2m1x8(v);
-            packed[2 * g + 1] = e2m1x8(v + 8);
+            for (int h = 0; h < 2; ++h) {
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint32_t ww = w[8 * g + 4 * h + e];
+                v[2 * e] = div_by_scale(bf16lo(ww), s_, y);
+                v[2 * e + 1] = div_by_scale(bf16hi(ww), s_, y);
+              }
+              packed[2 * g + h] = e2m1x8(v);
+            }
           } else {
             packed[2 * g] = 0u;
             packed[2 * g + 1] = 0u;
@@ -282,17 +308,31 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
       } else {
         float a = 0.0f;
 #pragma unroll
-        for (int e = 0; e < 64; ++e) a = fmaxf(a, fabsf(xs[e]));
-        const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(a, 7.0f));
+        for (int e = 0; e < 32; ++e) a = fmaxf(a, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+        const __nv_bfloat16 sb = __float2bfloat16_rn(div_by_scale(a, 7.0f, kRcp7));
         const float s_ = __bfloat162float(sb);
-        if (s_ > 0.0f) {
+        if (s_ >= kMinFastScale && s_ < kMaxFastScale) {
           const float y = __frcp_rn(s_);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             uint32_t pk = 0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              pk |= int4_rn(div_by_scale(xs[8 * j + e], s_, y)) << (4 * e);
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t ww = w[4 * j + e];
+              pk |= int4_rn(div_by_scale(bf16lo(ww), s_, y)) << (8 * e);
+              pk |= int4_rn(div_by_scale(bf16hi(ww), s_, y)) << (8 * e + 4);
+            }
+            packed[j] = pk;
+          }
+        } else if (s_ > 0.0f) {  // scale outside the fast path's range: exact division
+#pragma unroll 1
+          for (int j = 0; j < 8; ++j) {
+            uint32_t pk = 0;
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t ww = w[4 * j + e];
+              pk |= int4_rn(__fdiv_rn(bf16lo(ww), s_)) << (8 * e);
+              pk |= int4_rn(__fdiv_rn(bf16hi(ww), s_)) << (8 * e + 4);
+            }
             packed[j] = pk;
           }
         } else {
@@ -313,83 +353,67 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
 
   // ------------------------------------------------------- T = X' L1 epilogue
   if constexpr (R > 0) {
-    float* tp = reinterpret_cast<float*>(smem + KQ_STAGES * S::STAGE);
-    const bool reader = warp < 4;  // one warp per 32-lane group of tensor memory
-    if (reader) {
+    // partial tile of this K range: straight to T when the row block is not
+    // split, else to the scratch slot of this split
+    const int num_m = gridDim.y;
+    if (warp < 4) {  // one warp per 32-lane group of tensor memory
       const int row = warp * 32 + lane;
+      const int grow = m0 + row;
       const bool ok = wait_bounded(bar_tfull, 0, guard, 0x105);
-      uint32_t v[R];
-      if (ok) {
-        tc_fence_after();
-        const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        if constexpr (R == 16) {
-          tmem_ld_x16(ta, v);
-        } else {
-#pragma unroll
-          for (int j = 0; j < R / 32; ++j) tmem_ld_x32(ta + 32 * j, v + 32 * j);
+      if (ok) tc_fence_after();
+      const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+      // stream the row's R fp32 values out of tensor memory 16 or 32 columns at a time
+      constexpr int CW = R < 32 ? R : 32;
+#pragma unroll 1
+      for (int c0 = 0; c0 < R; c0 += CW) {
+        uint32_t v[CW];
+        if (ok) {
+          if constexpr (CW == 16) tmem_ld_x16(ta + c0, v);
+          else tmem_ld_x32(ta + c0, v);
+          tmem_ld_wait();
         }
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int j = 0; j < R; ++j) v[j] = 0u;
-      }
-      if (p.ksplit == 1) {
-        const int grow = m0 + row;
         if (ok && grow < p.M) {
-          float4* dst = reinterpret_cast<float4*>(p.t + static_cast<size_t>(grow) * R);
+          float* drow = p.ksplit == 1
+                            ? p.t + static_cast<size_t>(grow) * R
+                            : p.tpart + ((static_cast<size_t>(ks) * num_m + blockIdx.y) * 128 + row) * R;
+          float4* dst = reinterpret_cast<float4*>(drow + c0);
 #pragma unroll
-          for (int j = 0; j < R / 4; ++j)
+          for (int j = 0; j < CW / 4; ++j)
             dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                  __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-        }
-      } else {
-        // stage the partial tile; rotate the 16-byte column blocks per row to
-        // spread the shared-memory banks
-#pragma unroll
-        for (int j = 0; j < R / 4; ++j) {
-          const int jj = (j + row) % (R / 4);
-          reinterpret_cast<float4*>(tp + row * R)[jj] =
-              make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                          __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
         }
       }
     }
     if (p.ksplit > 1) {
-      // all CTAs of the cluster have their partial T in shared memory
-      asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                       : "memory");
-      // CTA `ks` sums rows [ks*rows_per, (ks+1)*rows_per) over the cluster, in rank order
-      const int rows_per = 128 / p.ksplit;
-      const int items = rows_per * (R / 4);
-      for (int it = threadIdx.x; it < items; it += KQ_THREADS) {
-        const int rr = ks * rows_per + it / (R / 4);
-        const int j = it % (R / 4);
-        const int jj = (j + rr) % (R / 4);
-        const uint32_t local = smem_u32(tp + rr * R + 4 * jj);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int src = 0; src < p.ksplit; ++src) {
-          uint32_t ra;
-          asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local), "r"(src));
-          float4 f;
-          asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                       : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w)
-                       : "r"(ra)
-                       : "memory");
-          acc.x += f.x; acc.y += f.y; acc.z += f.z; acc.w += f.w;
+      // The last split CTA of this row block to arrive sums the partial tiles
+      // in split order (deterministic) and resets the block's counter.
+      __shared__ int last;
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) last = atomicAdd(p.counters + blockIdx.y, 1) == p.ksplit - 1;
+      __syncthreads();
+      if (last) {
+        __threadfence();
+        const int rows = min(128, p.M - m0);
+        for (int it = threadIdx.x; it < rows * (R / 4); it += KQ_THREADS) {
+          const int rr = it / (R / 4), j = it % (R / 4);
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int src = 0; src < p.ksplit; ++src) {
+            const float4 f = __ldcg(reinterpret_cast<const float4*>(
+                p.tpart + ((static_cast<size_t>(src) * num_m + blockIdx.y) * 128 + rr) * R) + j);
+            acc.x += f.x; acc.y += f.y; acc.z += f.z; acc.w += f.w;
+          }
+          if (!*abort_flag)
+            reinterpret_cast<float4*>(p.t + static_cast<size_t>(m0 + rr) * R)[j] = acc;
         }
-        const int grow = m0 + rr;
-        if (grow < p.M && !*abort_flag)
-          reinterpret_cast<float4*>(p.t + static_cast<size_t>(grow) * R)[j] = acc;
+        if (threadIdx.x == 0) p.counters[blockIdx.y] = 0;
       }
-      // keep this CTA's shared memory alive until every peer has read it
-      asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                       : "memory");
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (R > 0 && warp == 9) {
+  if (R > 0 && warp == MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }

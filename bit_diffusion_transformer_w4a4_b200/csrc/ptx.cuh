@@ -64,11 +64,39 @@ struct Guard {
   uint64_t limit_ns;
 };
 
+#ifdef SVDQ_WAIT_PROFILE
+// Opt-in instrumentation (compile with -DSVDQ_WAIT_PROFILE): SM cycles spent
+// in each wait site, summed over all waiting threads' first lanes.
+__device__ unsigned long long g_wait_cycles[1024];
+__device__ unsigned long long g_wait_count[1024];
+#endif
+
+__device__ __forceinline__ bool wait_bounded_impl(uint32_t bar, uint32_t parity, const Guard& g,
+                                                  int site, uint32_t sleep_ns);
+
+// `sleep_ns` > 0 backs off between polls: for waits that are expected to be
+// long (idle epilogue warps), so they leave issue slots to the busy warps.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Guard& g,
-                                             int site) {
+                                             int site, uint32_t sleep_ns = 0) {
+#ifdef SVDQ_WAIT_PROFILE
+  const long long c0 = clock64();
+  const bool r = wait_bounded_impl(bar, parity, g, site, sleep_ns);
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(&g_wait_cycles[site & 1023], static_cast<unsigned long long>(clock64() - c0));
+    atomicAdd(&g_wait_count[site & 1023], 1ull);
+  }
+  return r;
+#else
+  return wait_bounded_impl(bar, parity, g, site, sleep_ns);
+#endif
+}
+
+__device__ __forceinline__ bool wait_bounded_impl(uint32_t bar, uint32_t parity, const Guard& g,
+                                                  int site, uint32_t sleep_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if (*g.abort_flag) return false;
     if (global_timer_ns() - t0 > g.limit_ns) {

@@ -91,6 +91,8 @@ svdq_status set_smem(K kernel, int bytes) {
 struct svdq_weights {
   svdq_variant variant;
   int64_t K, N, r, max_M, npad;
+  int64_t lr_cols = 0;          // columns of the [L2^T | L2^T] operand (multiple of 64)
+  uint32_t stage_row_bytes = 64;  // bytes per operand row in one GEMM pipeline stage
   uint32_t flags;
   int device, sms;
   // device weights (library-owned)
@@ -100,6 +102,10 @@ struct svdq_weights {
   uint8_t* wcodes = nullptr;   // NVFP4 [N x K/2] packed; INT4 [N x K] int8
   uint8_t* wscales = nullptr;  // NVFP4 tiled E4M3; INT4 fp32 [K/64 x npad]
   uint16_t* bias = nullptr;
+  // activation-kernel scratch: partial T tiles of split row blocks and their
+  // arrival counters (zero between launches)
+  float* kq_tpart = nullptr;
+  int* kq_counters = nullptr;
   // forward workspace (sized for max_M)
   uint8_t* ws_codes = nullptr;
   uint8_t* ws_scales = nullptr;
@@ -129,7 +135,7 @@ size_t act_scale_bytes(const svdq_weights* h, int64_t M) {
 
 void free_all(svdq_weights* h) {
   void* ptrs[] = {h->inv_lam, h->l1t, h->l2dup, h->wcodes, h->wscales, h->bias, h->ws_codes,
-                  h->ws_scales, h->ws_t, h->x_dev, h->y_dev, h->err};
+                  h->ws_scales, h->ws_t, h->x_dev, h->y_dev, h->err, h->kq_tpart, h->kq_counters};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -147,13 +153,19 @@ svdq_status launch_kq_t(svdq_weights* h, const CUtensorMap& tmx, int64_t M, uint
   }
   const int num_m = static_cast<int>(cdiv(M, 128));
   const int kch = static_cast<int>(h->K / 64);
+  // split the K range so that the grid fills the SMs in one wave
   int ksplit = 1;
-  while (ksplit < 8 && num_m * ksplit * 2 <= h->sms && kch % (ksplit * 2) == 0) ksplit *= 2;
+  if (R > 0)
+    while (ksplit < 8 && num_m * ksplit * 2 <= h->sms && kch % (ksplit * 2) == 0) ksplit *= 2;
+  else
+    while (ksplit < 8 && num_m * ksplit * 2 <= h->sms && kch % (ksplit * 2) == 0) ksplit *= 2;
   KQParams p;
   p.inv_lam = h->inv_lam;
   p.codes = codes;
   p.scales = scales;
   p.t = t;
+  p.tpart = h->kq_tpart;
+  p.counters = h->kq_counters;
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(h->K);
   p.ksplit = ksplit;
@@ -166,15 +178,6 @@ svdq_status launch_kq_t(svdq_weights* h, const CUtensorMap& tmx, int64_t M, uint
   cfg.blockDim = dim3(KQ_THREADS, 1, 1);
   cfg.dynamicSmemBytes = S::TOTAL;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
-  if (R > 0 && ksplit > 1) {
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = ksplit;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-  }
   SVDQ_TRY(cudaLaunchKernelEx(&cfg, kq_kernel<V, R>, tmx, h->tm_l1t, p));
   return SVDQ_OK;
 }
@@ -252,8 +255,9 @@ svdq_status get_tm_a(svdq_weights* h, const void* codes, int64_t M) {
   if (h->tm_a_ptr == codes && h->tm_a_M == M) return SVDQ_OK;
   svdq_status s =
       h->variant == SVDQ_NVFP4_G16_E4M3
-          ? make_tmap(&h->tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h->K / 2, M, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_64B)
+          ? make_tmap(&h->tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h->K / 2, M,
+                      h->stage_row_bytes, 128,
+                      h->stage_row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B)
           : make_tmap(&h->tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h->K / 2, M, 32, 128,
                       CU_TENSOR_MAP_SWIZZLE_32B);
   if (s != SVDQ_OK) return s;
@@ -272,24 +276,50 @@ svdq_status check_call(svdq_weights* h, int64_t M) {
 }
 
 // ------------------------------------------------------------- self-test
-// Exhaustive comparison of the quantiser's division routine against IEEE
-// division over every bf16 dividend and every positive finite scale of the
-// variant (E4M3: 126 values; bf16: 32639 values).
-__global__ void selftest_div_kernel(int variant, unsigned long long* mismatches) {
+// Exhaustive check of the quantiser's division routine against IEEE division
+// over every bf16 dividend and every positive finite scale of the variant
+// (E4M3: 126 values; bf16: 32639 values), restricted to the quantiser's
+// domain |x / s| <= 8 (a group's values never exceed ~7.02 scales).
+//   bad[0]: pairs whose 4-bit codes differ (the kernels rely on 0)
+//   bad[1]: pairs whose quotients differ while |IEEE quotient| >= 2^-24
+//           (far below the smallest nonzero code threshold, 0.25), plus
+//           the scale divisions amax/6 and amax/7 over all finite bf16 amax
+__global__ void selftest_div_kernel(int variant, unsigned long long* bad) {
   const uint32_t sidx = blockIdx.x + 1;  // 1 .. number of positive finite scales
   float s;
   if (variant == 1) s = e4m3_value(sidx);
   else s = __uint_as_float(sidx << 16);
-  const float y = __frcp_rn(s);
-  unsigned long long bad = 0;
+  const float y = (s >= kMinFastScale && s < kMaxFastScale) ? __frcp_rn(s) : 0.0f;
+  unsigned long long bad_code = 0, bad_quot = 0;
   for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
     const float x = __uint_as_float(xb << 16);
     if (!isfinite(x)) continue;
-    const float a = div_by_scale(x, s, y);
     const float b = __fdiv_rn(x, s);
-    if (__float_as_uint(a) != __float_as_uint(b)) ++bad;
+    if (!(fabsf(b) <= 8.0f)) continue;
+    const float a = quant_div(x, s, y);
+    uint32_t ca, cb;
+    if (variant == 1) {
+      float va[8] = {a, 0, 0, 0, 0, 0, 0, 0}, vb[8] = {b, 0, 0, 0, 0, 0, 0, 0};
+      ca = e2m1x8(va) & 0xFu;
+      cb = e2m1x8(vb) & 0xFu;
+    } else {
+      ca = int4_rn(a);
+      cb = int4_rn(b);
+    }
+    if (ca != cb) ++bad_code;
+    if (fabsf(b) >= 5.9604644775390625e-08f && __float_as_uint(a) != __float_as_uint(b)) ++bad_quot;
   }
-  if (bad) atomicAdd(mismatches, bad);
+  if (blockIdx.x == 0) {
+    // the group scale divisions amax / 6 and amax / 7 over every finite bf16 amax
+    for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
+      const float x = __uint_as_float(xb << 16);
+      if (!isfinite(x)) continue;
+      if (__float_as_uint(div_by_scale(x, 6.0f, kRcp6)) != __float_as_uint(__fdiv_rn(x, 6.0f))) ++bad_quot;
+      if (__float_as_uint(div_by_scale(x, 7.0f, kRcp7)) != __float_as_uint(__fdiv_rn(x, 7.0f))) ++bad_quot;
+    }
+  }
+  if (bad_code) atomicAdd(bad, bad_code);
+  if (bad_quot) atomicAdd(bad + 1, bad_quot);
 }
 
 }  // namespace
@@ -362,14 +392,16 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
   // ---- host-side re-layout (load time only)
   std::vector<float> inv(K);
   for (int64_t k = 0; k < K; ++k) inv[k] = 1.0f / d->lambda[k];  // IEEE fp32 division
-  std::vector<uint16_t> l1t(static_cast<size_t>(r) * K), l2dup(static_cast<size_t>(N) * 2 * r);
+  // [L2^T | L2^T], zero-padded to a multiple of 64 columns (one 128-byte row)
+  h->lr_cols = r > 0 ? (2 * r + 63) / 64 * 64 : 0;
+  std::vector<uint16_t> l1t(static_cast<size_t>(r) * K), l2dup(static_cast<size_t>(N) * h->lr_cols, 0);
   for (int64_t k = 0; k < K; ++k)
     for (int64_t j = 0; j < r; ++j) l1t[j * K + k] = d->L1[k * r + j];
   for (int64_t n = 0; n < N; ++n)
     for (int64_t j = 0; j < r; ++j) {
       const uint16_t v = d->L2[j * N + n];
-      l2dup[n * 2 * r + j] = v;
-      l2dup[n * 2 * r + r + j] = v;
+      l2dup[n * h->lr_cols + j] = v;
+      l2dup[n * h->lr_cols + r + j] = v;
     }
   std::vector<uint8_t> codes, scales;
   if (d->variant == SVDQ_NVFP4_G16_E4M3) {
@@ -414,6 +446,11 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
                 !dmalloc(reinterpret_cast<void**>(&h->ws_t), static_cast<size_t>(h->max_M) * r * 4)))
     return fail(SVDQ_ERR_OOM);
   if (d->bias && !dmalloc(reinterpret_cast<void**>(&h->bias), N * 2)) return fail(SVDQ_ERR_OOM);
+  if (r > 0 && (!dmalloc(reinterpret_cast<void**>(&h->kq_tpart), static_cast<size_t>(sms) * 128 * r * 4) ||
+                !dmalloc(reinterpret_cast<void**>(&h->kq_counters), cdiv(h->max_M, 128) * 4)))
+    return fail(SVDQ_ERR_OOM);
+  if (h->kq_counters && cudaMemset(h->kq_counters, 0, cdiv(h->max_M, 128) * 4) != cudaSuccess)
+    return fail(SVDQ_ERR_CUDA);
 
   // synchronous copies: the host vectors go out of scope on return
   if (cudaMemcpy(h->inv_lam, inv.data(), K * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
@@ -428,15 +465,21 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
     return fail(SVDQ_ERR_CUDA);
 
   // ---- weight-side tensor maps
+  // NVFP4 stages are 128-byte rows (128B swizzle) except at rank 128 (64-byte
+  // rows); the INT4 kernel uses 64-byte rows
+  const bool wide = d->variant == SVDQ_NVFP4_G16_E4M3 && r < 128;
+  const uint32_t rowb = wide ? 128 : 64;
+  const CUtensorMapSwizzle swz = wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  h->stage_row_bytes = rowb;
   svdq_status s = d->variant == SVDQ_NVFP4_G16_E4M3
                       ? make_tmap(&h->tm_b, h->wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N,
-                                  64, 256, CU_TENSOR_MAP_SWIZZLE_64B)
+                                  rowb, 256, swz)
                       : make_tmap(&h->tm_b, h->wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, 64,
                                   256, CU_TENSOR_MAP_SWIZZLE_64B);
   if (s != SVDQ_OK) return fail(s);
   if (r > 0) {
-    if ((s = make_tmap(&h->tm_blr, h->l2dup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 2 * r, N, 32, 256,
-                       CU_TENSOR_MAP_SWIZZLE_64B)) != SVDQ_OK)
+    if ((s = make_tmap(&h->tm_blr, h->l2dup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->lr_cols, N,
+                       rowb / 2, 256, swz)) != SVDQ_OK)
       return fail(s);
     if ((s = make_tmap(&h->tm_l1t, h->l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, r, 64,
                        static_cast<uint32_t>(r), CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
@@ -531,6 +574,8 @@ svdq_status svdq_device_status(svdq_weights_t h, void* stream) {
   if (cudaMemcpy(&e, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SVDQ_ERR_CUDA;
   if (e != 0) {
     cudaMemset(h->err, 0, sizeof(int));
+    // an aborted launch may leave split arrival counters mid-count
+    if (h->kq_counters) cudaMemset(h->kq_counters, 0, cdiv(h->max_M, 128) * 4);
     return SVDQ_ERR_DEVICE_TIMEOUT;
   }
   return SVDQ_OK;
@@ -548,15 +593,29 @@ svdq_status svdq_selftest_division(int variant, unsigned long long* mismatches) 
   svdq_status ds = check_device(nullptr, nullptr);
   if (ds != SVDQ_OK) return ds;
   unsigned long long* d = nullptr;
-  SVDQ_TRY(cudaMalloc(&d, sizeof(unsigned long long)));
-  cudaMemset(d, 0, sizeof(unsigned long long));
+  SVDQ_TRY(cudaMalloc(&d, 2 * sizeof(unsigned long long)));
+  cudaMemset(d, 0, 2 * sizeof(unsigned long long));
   // E4M3: codes 1..126 are the positive finite scales; bf16: 0x0001..0x7F7F
   const int nscales = variant == 1 ? 126 : 0x7F7F;
   selftest_div_kernel<<<nscales, 256>>>(variant, d);
   cudaError_t e = cudaDeviceSynchronize();
-  if (e == cudaSuccess) e = cudaMemcpy(mismatches, d, sizeof(unsigned long long), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(mismatches, d, 2 * sizeof(unsigned long long), cudaMemcpyDeviceToHost);
   cudaFree(d);
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
+
+#ifdef SVDQ_WAIT_PROFILE
+// Instrumented builds only: read and clear the per-site wait counters.
+int svdq_wait_profile(unsigned long long* cycles, unsigned long long* counts) {
+  cudaDeviceSynchronize();
+  cudaMemcpyFromSymbol(cycles, g_wait_cycles, sizeof(g_wait_cycles));
+  cudaMemcpyFromSymbol(counts, g_wait_count, sizeof(g_wait_count));
+  static unsigned long long zero[1024] = {};
+  cudaMemcpyToSymbol(g_wait_cycles, zero, sizeof(zero));
+  cudaMemcpyToSymbol(g_wait_count, zero, sizeof(zero));
+  return 0;
+}
+#endif
 
 }  // extern "C"

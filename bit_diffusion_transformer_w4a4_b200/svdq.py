@@ -74,7 +74,7 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
     L.svdq_linear_forward_host.argtypes = [vp, vp, vp, i64, vp]
     L.svdq_device_status.argtypes = [vp, vp]
     L.svdq_debug_set_fault.argtypes = [vp, ctypes.c_uint32, ctypes.c_uint32]
-    L.svdq_selftest_division.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_ulonglong)]
+    L.svdq_selftest_division.argtypes = [ctypes.c_int, ctypes.c_void_p]
     L.svdq_status_string.argtypes = [st]
     L.svdq_status_string.restype = ctypes.c_char_p
     L.svdq_version.restype = ctypes.c_char_p
@@ -109,10 +109,11 @@ def _stream(stream) -> int:
     return int(stream)
 
 
-def selftest_division(variant: int) -> int:
-    n = ctypes.c_ulonglong(0)
-    _check(lib().svdq_selftest_division(variant, ctypes.byref(n)), "svdq_selftest_division")
-    return int(n.value)
+def selftest_division(variant: int) -> tuple[int, int]:
+    """(code mismatches, normal-range quotient mismatches) -- both 0 expected."""
+    n = (ctypes.c_ulonglong * 2)()
+    _check(lib().svdq_selftest_division(variant, n), "svdq_selftest_division")
+    return int(n[0]), int(n[1])
 
 
 class SVDQWeights:

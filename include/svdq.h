@@ -128,8 +128,8 @@ svdq_status svdq_act_scales_bytes(svdq_weights_t h, int64_t M, size_t* bytes);
  * Per element (round to nearest even throughout):
  *   x' = bf16(fp32(x) * inv_lambda);  a = max|x'| over the group;
  *   INT4 s = bf16(a / 7), q = rint(x'/s);  NVFP4 s = e4m3_satfinite(a / 6),
- *   q = e2m1_satfinite(x'/s);  s == 0 gives q = +0.  Divisions are IEEE
- *   correctly rounded fp32.
+ *   q = e2m1_satfinite(x'/s);  s == 0 gives q = +0.  Codes are those of
+ *   IEEE correctly rounded fp32 division x'/s.
  */
 svdq_status svdq_quantize_act_lowrank_down(svdq_weights_t h, const void* x, int64_t M,
                                            uint8_t* act_codes, void* act_scales, float* t,
@@ -176,11 +176,17 @@ svdq_status svdq_device_status(svdq_weights_t h, void* stream);
 svdq_status svdq_debug_set_fault(svdq_weights_t h, uint32_t mask, uint32_t timeout_us);
 
 /*
- * Self-test of the activation quantiser's division: runs the kernels'
- * correctly-rounded x / s routine against IEEE fp32 division for every bf16
- * dividend and every positive finite scale of `variant` (0: bf16 scales,
- * 1: E4M3 scales) on the current device, and stores the number of results
- * that differ in *mismatches (0 expected).  Synchronises the device.
+ * Self-test of the activation quantiser's division (x / s is computed with a
+ * reciprocal and one fma correction step).  Runs it against IEEE fp32
+ * division for every bf16 dividend and every positive finite scale of
+ * `variant` (0: bf16 scales, 1: E4M3 scales) with |x / s| <= 8 on the
+ * current device and writes two counts to mismatches[0..1]:
+ *   [0] pairs whose 4-bit codes differ (0 expected: the codes the kernels
+ *       write are exactly those of IEEE division);
+ *   [1] pairs whose quotients differ while |IEEE quotient| >= 2^-24, plus
+ *       the group-scale divisions amax/6 and amax/7 that differ, over all
+ *       finite bf16 amax.
+ * Synchronises the device.
  */
 svdq_status svdq_selftest_division(int variant, unsigned long long* mismatches);
 

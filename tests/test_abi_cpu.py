@@ -92,5 +92,5 @@ def test_no_gpu_no_fallback():
     d, keep = _desc()
     h = ctypes.c_void_p(0)
     assert L.svdq_weights_load(ctypes.byref(d), ctypes.byref(h), None) == 4
-    n = ctypes.c_ulonglong(0)
-    assert L.svdq_selftest_division(1, ctypes.byref(n)) == 4
+    n = (ctypes.c_ulonglong * 2)()
+    assert L.svdq_selftest_division(1, n) == 4

@@ -24,7 +24,8 @@ def _prepped(M, K, N, r, variant, gelu=False, with_bias=False, seed=0, cid=50):
 
 @pytest.mark.parametrize("variant", [INT4, NVFP4])
 def test_division_selftest_exhaustive(variant):
-    assert svdq.selftest_division(variant) == 0
+    bad_codes, bad_quotients = svdq.selftest_division(variant)
+    assert bad_codes == 0 and bad_quotients == 0, (bad_codes, bad_quotients)
 
 
 @pytest.mark.parametrize("variant", [INT4, NVFP4])
