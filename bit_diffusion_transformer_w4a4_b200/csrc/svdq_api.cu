@@ -322,6 +322,90 @@ __global__ void selftest_div_kernel(int variant, unsigned long long* bad) {
   if (bad_quot) atomicAdd(bad + 1, bad_quot);
 }
 
+// ------------------------------------------------- allocation-free variant
+// Scratch of svdq_quantize_act_lowrank_down_static, in the library's own
+// static device memory (every GPU that loads the library holds it until the
+// process exits): split partial T tiles, then one arrival counter per
+// 128-row block, then a fallback error word.
+constexpr size_t kStaticTpartBytes = 10u << 20;   // 10 MiB of partial T tiles
+constexpr int kStaticMaxRowBlocks = 4096;          // M <= 4096 * 128 tokens
+constexpr size_t kStaticScratchBytes = kStaticTpartBytes + kStaticMaxRowBlocks * 4 + 256;
+static __device__ __align__(256) unsigned char g_kq_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+void* g_static_ptr[64] = {};  // device address of the scratch, per device ordinal
+
+// Once per device, with that device current: the scratch's device address.
+svdq_status static_scratch(int dev, unsigned char** out) {
+  if (dev < 0 || dev >= 64) return SVDQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_kq_static_scratch) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
+    g_static_ptr[dev] = ptr;
+  }
+  *out = static_cast<unsigned char*>(g_static_ptr[dev]);
+  return SVDQ_OK;
+}
+
+template <int V, int R>
+svdq_status launch_kq_static(const CUtensorMap& tmx, const CUtensorMap& tml, const float* inv_lam,
+                             int64_t M, int64_t K, int sms, uint8_t* codes, void* scales, float* t,
+                             unsigned char* scratch, int* err, cudaStream_t st) {
+  using S = KQSmem<V, R>;
+  static bool attr = false;
+  if (!attr) {
+    svdq_status s = set_smem(kq_kernel<V, R>, S::TOTAL);
+    if (s != SVDQ_OK) return s;
+    attr = true;
+  }
+  const int num_m = static_cast<int>(cdiv(M, 128));
+  const int kch = static_cast<int>(K / 64);
+  int ksplit = 1;  // same split rule as the handle-based entry point
+  while (ksplit < 8 && num_m * ksplit * 2 <= sms && kch % (ksplit * 2) == 0) ksplit *= 2;
+  if (R > 0 && ksplit > 1 &&
+      static_cast<size_t>(ksplit) * num_m * 128 * R * 4 > kStaticTpartBytes)
+    return SVDQ_ERR_SHAPE;
+  int* counters = reinterpret_cast<int*>(scratch + kStaticTpartBytes);
+  if (R > 0 && ksplit > 1)  // arrival counters must start at zero
+    SVDQ_TRY(cudaMemsetAsync(counters, 0, static_cast<size_t>(num_m) * 4, st));
+  KQParams p;
+  p.inv_lam = inv_lam;
+  p.codes = codes;
+  p.scales = scales;
+  p.t = t;
+  p.tpart = reinterpret_cast<float*>(scratch);
+  p.counters = counters;
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(K);
+  p.ksplit = ksplit;
+  p.chunks = kch / ksplit;
+  p.err = err;
+  p.debug_mask = 0;
+  p.timeout_ns = kDefaultTimeoutNs;
+  kq_kernel<V, R><<<dim3(ksplit, num_m, 1), KQ_THREADS, S::TOTAL, st>>>(tmx, tml, p);
+  SVDQ_TRY(cudaGetLastError());
+  return SVDQ_OK;
+}
+
+template <int V>
+svdq_status launch_kq_static_v(int64_t r, const CUtensorMap& tmx, const CUtensorMap& tml,
+                               const float* inv_lam, int64_t M, int64_t K, int sms, uint8_t* codes,
+                               void* scales, float* t, unsigned char* scratch, int* err,
+                               cudaStream_t st) {
+  switch (r) {
+    case 0: return launch_kq_static<V, 0>(tmx, tml, inv_lam, M, K, sms, codes, scales, t, scratch, err, st);
+    case 16: return launch_kq_static<V, 16>(tmx, tml, inv_lam, M, K, sms, codes, scales, t, scratch, err, st);
+    case 32: return launch_kq_static<V, 32>(tmx, tml, inv_lam, M, K, sms, codes, scales, t, scratch, err, st);
+    case 64: return launch_kq_static<V, 64>(tmx, tml, inv_lam, M, K, sms, codes, scales, t, scratch, err, st);
+    case 128: return launch_kq_static<V, 128>(tmx, tml, inv_lam, M, K, sms, codes, scales, t, scratch, err, st);
+  }
+  return SVDQ_ERR_SHAPE;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -586,6 +670,44 @@ svdq_status svdq_debug_set_fault(svdq_weights_t h, uint32_t mask, uint32_t timeo
   h->debug_mask = mask;
   h->timeout_ns = timeout_us ? static_cast<uint64_t>(timeout_us) * 1000ull : kDefaultTimeoutNs;
   return SVDQ_OK;
+}
+
+svdq_status svdq_quantize_act_lowrank_down_static(svdq_variant variant, int64_t K, int64_t r,
+                                                  const float* inv_lambda, const uint16_t* l1t,
+                                                  const void* x, int64_t M, uint8_t* act_codes,
+                                                  void* act_scales, float* t, int* device_error,
+                                                  void* stream) {
+  if (variant != SVDQ_INT4_G64_BF16 && variant != SVDQ_NVFP4_G16_E4M3) return SVDQ_ERR_INVALID_ARG;
+  if (K < 128 || K % 128 != 0 || K > (1 << 20)) return SVDQ_ERR_SHAPE;
+  if (!(r == 0 || r == 16 || r == 32 || r == 64 || r == 128)) return SVDQ_ERR_SHAPE;
+  if (M < 1 || cdiv(M, 128) > kStaticMaxRowBlocks) return SVDQ_ERR_SHAPE;
+  if (!inv_lambda || !x || !act_codes || !act_scales || (r > 0 && (!l1t || !t)))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(inv_lambda) || !aligned16(x) || !aligned16(act_codes) || !aligned16(act_scales) ||
+      (r > 0 && (!aligned16(l1t) || !aligned16(t))))
+    return SVDQ_ERR_ALIGNMENT;
+  int dev = 0, sms = 0;
+  svdq_status s = check_device(&dev, &sms);
+  if (s != SVDQ_OK) return s;
+  unsigned char* scratch = nullptr;
+  if ((s = static_scratch(dev, &scratch)) != SVDQ_OK) return s;
+  int* err = device_error ? device_error
+                          : reinterpret_cast<int*>(scratch + kStaticTpartBytes + kStaticMaxRowBlocks * 4);
+  CUtensorMap tmx, tml;
+  if ((s = make_tmap(&tmx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+    return s;
+  if (r > 0) {
+    if ((s = make_tmap(&tml, l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, r, 64,
+                       static_cast<uint32_t>(r), CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return s;
+  } else {
+    tml = tmx;  // never read when r == 0
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return variant == SVDQ_NVFP4_G16_E4M3
+             ? launch_kq_static_v<1>(r, tmx, tml, inv_lambda, M, K, sms, act_codes, act_scales, t, scratch, err, st)
+             : launch_kq_static_v<0>(r, tmx, tml, inv_lambda, M, K, sms, act_codes, act_scales, t, scratch, err, st);
 }
 
 svdq_status svdq_selftest_division(int variant, unsigned long long* mismatches) {

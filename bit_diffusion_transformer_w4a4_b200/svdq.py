@@ -29,6 +29,7 @@ EXPORTED = [
     "svdq_quantize_act_lowrank_down", "svdq_w4a4_gemm_lowrank_up", "svdq_linear_forward",
     "svdq_linear_forward_host", "svdq_device_status", "svdq_debug_set_fault",
     "svdq_selftest_division", "svdq_status_string", "svdq_version",
+    "svdq_quantize_act_lowrank_down_static",
 ]
 
 
@@ -75,6 +76,7 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
     L.svdq_device_status.argtypes = [vp, vp]
     L.svdq_debug_set_fault.argtypes = [vp, ctypes.c_uint32, ctypes.c_uint32]
     L.svdq_selftest_division.argtypes = [ctypes.c_int, ctypes.c_void_p]
+    L.svdq_quantize_act_lowrank_down_static.argtypes = [st, i64, i64, vp, vp, vp, i64, vp, vp, vp, vp, vp]
     L.svdq_status_string.argtypes = [st]
     L.svdq_status_string.restype = ctypes.c_char_p
     L.svdq_version.restype = ctypes.c_char_p

@@ -161,6 +161,38 @@ svdq_status svdq_linear_forward_host(svdq_weights_t h, const void* x_host, void*
                                      int64_t M, void* stream);
 
 /*
+ * Kernel 1 for callers that cannot allocate device memory: the same
+ * smoothing, quantisation, packing and down projection as
+ * svdq_quantize_act_lowrank_down, but with no weights handle and no call to
+ * cudaMalloc or any other allocating routine, at load time or per call.
+ * Code that runs inside a CUDA-graph capture, a runtime that owns every
+ * device allocation (a fixed memory pool of an inference server, an
+ * embedding plugin host), or a process with a hard device-memory budget
+ * cannot let a library allocate; it passes every buffer itself:
+ *   inv_lambda  device fp32 [K]      1 / lambda (the caller divides)
+ *   l1t         device bf16 [r x K]  L1 transposed (NULL when r == 0)
+ *   x, act_codes, act_scales, t      as for svdq_quantize_act_lowrank_down
+ *   device_error device int, set to a nonzero wait-site code if a bounded
+ *               wait expires (never cleared by the library); may be NULL
+ * The split-K scratch (partial T tiles and per-row-block arrival counters)
+ * lives in a static device array of the library: 10 MiB of partial tiles
+ * plus counters for M <= 524288 tokens, held by every GPU that loads the
+ * library until the process exits.  Calls whose split needs more, or with
+ * M > 524288, return SVDQ_ERR_SHAPE before any work is enqueued.  The first
+ * call on a device looks up the array's device address (once per device,
+ * that device current); make that first call before any stream capture.
+ * Every call shares the one array: the counters are cleared on `stream`
+ * before each launch, and calls that overlap on the GPU (two streams, two
+ * threads) race on it and must be serialised by the caller.
+ * The paper has no counterpart to this entry point.
+ */
+svdq_status svdq_quantize_act_lowrank_down_static(svdq_variant variant, int64_t K, int64_t r,
+                                                  const float* inv_lambda, const uint16_t* l1t,
+                                                  const void* x, int64_t M, uint8_t* act_codes,
+                                                  void* act_scales, float* t, int* device_error,
+                                                  void* stream);
+
+/*
  * Synchronise `stream` and report device-side failures recorded by earlier
  * calls on this handle (SVDQ_ERR_DEVICE_TIMEOUT), clearing the record.
  */
