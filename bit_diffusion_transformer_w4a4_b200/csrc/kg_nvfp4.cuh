@@ -152,7 +152,14 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t id_f4 = idesc_nvf4(KG_BM, KG_BN);
       constexpr uint32_t id_bf = idesc_bf16_f32(KG_BM, KG_BN);
-      const uint32_t alr = sbase + S::ALR_OFF;
+      // Descriptors are built once; a start address moves in 16-byte units in
+      // the low bits, so per-stage / per-k-block offsets are plain additions.
+      const uint64_t dA0 = smem_desc(sbase, 16, S::SBO, S::SWZ);
+      const uint64_t dB0 = smem_desc(sbase + S::A_BYTES, 16, S::SBO, S::SWZ);
+      const uint64_t dSFA0 = smem_desc(sbase + S::A_BYTES + S::B_BYTES, 0, 128, SWZ_NONE);
+      const uint64_t dSFB0 = smem_desc(sbase + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, 0, 128, SWZ_NONE);
+      const uint64_t dLRA0 = smem_desc(sbase + S::ALR_OFF, 16, 1024, SWZ_128B);
+      constexpr uint64_t kStage = S::STAGE >> 4;
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -162,26 +169,22 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         for (int ks = 0; ks < nks; ++ks) {
           if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x204))) break;
           tc_fence_after();
-          const uint32_t st = sbase + s * S::STAGE;
-          const uint32_t sfa_s = st + S::A_BYTES + S::B_BYTES;
-          const uint32_t sfb_s = sfa_s + S::SFA_BYTES;
+          const uint64_t so = kStage * s;
           const int kv = min(KB, kblk - KB * ks);
+          const uint32_t ca = tmem + S::SFA_COL + KB * 4 * s;
+          const uint32_t cb = tmem + S::SFB_COL + KB * 8 * s;
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) {
             if (kb >= kv) break;
-            const uint32_t ca = S::SFA_COL + (KB * s + kb) * 4;
-            const uint32_t cb = S::SFB_COL + (KB * s + kb) * 8;
-            tmem_cp_32x128b_warpx4(tmem + ca, smem_desc(sfa_s + kb * 512, 0, 128, SWZ_NONE));
-            tmem_cp_32x128b_warpx4(tmem + cb, smem_desc(sfb_s + kb * 512, 0, 128, SWZ_NONE));
-            tmem_cp_32x128b_warpx4(tmem + cb + 4, smem_desc(sfb_s + KB * 512 + kb * 512, 0, 128, SWZ_NONE));
+            tmem_cp_32x128b_warpx4(ca + 4 * kb, dSFA0 + so + 32 * kb);
+            tmem_cp_32x128b_warpx4(cb + 8 * kb, dSFB0 + so + 32 * kb);
+            tmem_cp_32x128b_warpx4(cb + 8 * kb + 4, dSFB0 + so + 32 * (KB + kb));
           }
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) {
             if (kb >= kv) break;
-            const uint64_t a = smem_desc(st + kb * 32, 16, S::SBO, S::SWZ);
-            const uint64_t b = smem_desc(st + S::A_BYTES + kb * 32, 16, S::SBO, S::SWZ);
-            mma_nvf4(tmem, a, b, id_f4, tmem + S::SFA_COL + (KB * s + kb) * 4,
-                     tmem + S::SFB_COL + (KB * s + kb) * 8, (ks | kb) != 0);
+            mma_nvf4(tmem, dA0 + so + 2 * kb, dB0 + so + 2 * kb, id_f4, ca + 4 * kb, cb + 8 * kb,
+                     (ks | kb) != 0);
           }
           tc_commit(bar_empty + 8 * s);
           if (++s == NST) { s = 0; ph ^= 1; }
@@ -193,15 +196,12 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           for (int l = 0; l < S::LR_STAGES; ++l) {
             if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x206))) break;
             tc_fence_after();
-            const uint32_t bst = sbase + s * S::STAGE + S::A_BYTES;
+            const uint64_t so = kStage * s;
 #pragma unroll
             for (int k2 = 0; k2 < KB; ++k2) {
               const int kk = KB * l + k2;  // k-step over [T_hi | T_lo]
-              if (kk < S::LR_STEPS) {
-                const uint64_t a = smem_desc(alr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, SWZ_128B);
-                const uint64_t b = smem_desc(bst + k2 * 32, 16, S::SBO, S::SWZ);
-                mma_bf16(tmem, a, b, id_bf, 1);
-              }
+              if (kk < S::LR_STEPS)
+                mma_bf16(tmem, dLRA0 + (kk / 4) * 1024 + (kk % 4) * 2, dB0 + so + 2 * k2, id_bf, 1);
             }
             tc_commit(bar_empty + 8 * s);
             if (++s == NST) { s = 0; ph ^= 1; }
