@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         const uint32_t b = gc & 1, use = gc >> 1;
         const float sx = sx_next;
         if (g + 1 < ng) sx_next = gm < p.M ? __bfloat162float(sxr[g + 1]) : 0.0f;
-        if (!(ok = wait_bounded(bar_gfull + 8 * b, use & 1, guard, 0x30a))) break;
+        if (!(ok = __all_sync(0xffffffffu, wait_bounded(bar_gfull + 8 * b, use & 1, guard, 0x30a)))) break;
         tc_fence_after();
         const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * 256 + cs * 64;
         const float4* swr = reinterpret_cast<const float4*>(sw_all + static_cast<size_t>(g) * npad + n_base);
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       if (!ok) break;
       if constexpr (R > 0) {
         const uint32_t b = gc & 1, use = gc >> 1;
-        if (!(ok = wait_bounded(bar_gfull + 8 * b, use & 1, guard, 0x30b))) break;
+        if (!(ok = __all_sync(0xffffffffu, wait_bounded(bar_gfull + 8 * b, use & 1, guard, 0x30b)))) break;
         tc_fence_after();
         const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * 256 + cs * 64;
 #pragma unroll
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           mbar_arrive(bar_lr_full);
         }
       }
-      store_row64(p, gm, n_base, acc);
+      store_rows64_coalesced(p, mb * KG_BM + q * 32, n_base, acc, lane);
     }
   }
 

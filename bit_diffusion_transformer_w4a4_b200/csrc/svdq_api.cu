@@ -15,6 +15,7 @@
 #include "../../include/svdq.h"
 #include "kg_int4.cuh"
 #include "kg_nvfp4.cuh"
+#include "kg_nvfp4_pair.cuh"
 #include "kq.cuh"
 
 using namespace svdq;
@@ -117,11 +118,16 @@ struct svdq_weights {
   uint32_t debug_mask = 0;
   uint64_t timeout_ns = kDefaultTimeoutNs;
   CUtensorMap tm_b, tm_blr, tm_l1t;
+  // NVFP4 CTA-pair GEMM: 128-row boxes of codes and L2, scale atoms as rows
+  // of 128 32-bit words
+  CUtensorMap tm_b2, tm_blr2, tm_sfb2;
   // per-call maps, cached by (pointer, M)
-  CUtensorMap tm_x, tm_a;
+  CUtensorMap tm_x, tm_a, tm_a2, tm_sfa2;
   const void* tm_x_ptr = nullptr;
   const void* tm_a_ptr = nullptr;
-  int64_t tm_x_M = -1, tm_a_M = -1;
+  const void* tm_a2_ptr = nullptr;
+  const void* tm_sfa2_ptr = nullptr;
+  int64_t tm_x_M = -1, tm_a_M = -1, tm_a2_M = -1, tm_sfa2_M = -1;
 };
 
 namespace {
@@ -228,9 +234,117 @@ svdq_status launch_kg_t(svdq_weights* h, const CUtensorMap& tma, int64_t M, cons
   return SVDQ_OK;
 }
 
+// Clusters of two CTAs that fit on the device at once for this kernel
+// (0 if the pair kernel cannot be resident).
+template <int R>
+int pair_clusters(svdq_weights* h) {
+  using S = KGF4PairSmem<R>;
+  static int clusters = -1;
+  if (clusters >= 0) return clusters;
+  clusters = 0;
+  if (set_smem(kg_nvfp4_pair_kernel<R>, S::TOTAL) != SVDQ_OK) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (h->sms / 2));
+  cfg.blockDim = dim3(KG_THREADS);
+  cfg.dynamicSmemBytes = S::TOTAL;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kg_nvfp4_pair_kernel<R>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  clusters = n;
+  return clusters;
+}
+
+template <int R>
+svdq_status launch_kg_pair_t(svdq_weights* h, int64_t M, const uint8_t* sfa, const float* t,
+                             void* y, int clusters, cudaStream_t st) {
+  using S = KGF4PairSmem<R>;
+  KGParams p;
+  p.sfa = sfa;
+  p.sfb = h->wscales;
+  p.t = t;
+  p.bias = h->bias;
+  p.y = static_cast<uint16_t*>(y);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(h->N);
+  p.K = static_cast<int>(h->K);
+  p.num_m = static_cast<int>(cdiv(M, 256));
+  p.num_n = static_cast<int>(cdiv(h->N, KG_BN));
+  p.gelu = (h->flags & SVDQ_EPI_GELU) ? 1 : 0;
+  p.err = h->err;
+  p.debug_mask = h->debug_mask;
+  p.timeout_ns = h->timeout_ns;
+  const int tiles = p.num_m * p.num_n;
+  const int n = tiles < clusters ? tiles : clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * n);
+  cfg.blockDim = dim3(KG_THREADS);
+  cfg.dynamicSmemBytes = S::TOTAL;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  SVDQ_TRY(cudaLaunchKernelEx(&cfg, kg_nvfp4_pair_kernel<R>, h->tm_a2, h->tm_b2, h->tm_blr2,
+                              h->tm_sfa2, h->tm_sfb2, p));
+  return SVDQ_OK;
+}
+
+// Per-call maps of the pair kernel over this call's codes and scales.
+svdq_status get_tm_pair(svdq_weights* h, const void* codes, const void* scales, int64_t M) {
+  if (h->tm_a2_ptr != codes || h->tm_a2_M != M) {
+    svdq_status s = make_tmap(&h->tm_a2, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h->K / 2, M, 128,
+                              128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != SVDQ_OK) return s;
+    h->tm_a2_ptr = codes;
+    h->tm_a2_M = M;
+  }
+  if (h->tm_sfa2_ptr != scales || h->tm_sfa2_M != M) {
+    svdq_status s = make_tmap(&h->tm_sfa2, scales, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128,
+                              cdiv(M, 128) * (h->K / 64), 128, 4, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (s != SVDQ_OK) return s;
+    h->tm_sfa2_ptr = scales;
+    h->tm_sfa2_M = M;
+  }
+  return SVDQ_OK;
+}
+
 template <int V>
-svdq_status launch_kg_v(svdq_weights* h, const CUtensorMap& tma, int64_t M, const uint8_t* sfa,
-                        const float* t, void* y, cudaStream_t st) {
+svdq_status launch_kg_v(svdq_weights* h, const CUtensorMap& tma, const uint8_t* codes, int64_t M,
+                        const uint8_t* sfa, const float* t, void* y, cudaStream_t st) {
+  if (V == 1 && M > 128 && (h->flags & SVDQ_GEMM_SM_PAIR)) {
+    int clusters = 0;
+    switch (h->r) {
+      case 0: clusters = pair_clusters<0>(h); break;
+      case 16: clusters = pair_clusters<16>(h); break;
+      case 32: clusters = pair_clusters<32>(h); break;
+      case 64: clusters = pair_clusters<64>(h); break;
+      case 128: clusters = pair_clusters<128>(h); break;
+      default: return SVDQ_ERR_SHAPE;
+    }
+    if (clusters > 0) {
+      svdq_status s = get_tm_pair(h, codes, sfa, M);
+      if (s != SVDQ_OK) return s;
+      switch (h->r) {
+        case 0: return launch_kg_pair_t<0>(h, M, sfa, t, y, clusters, st);
+        case 16: return launch_kg_pair_t<16>(h, M, sfa, t, y, clusters, st);
+        case 32: return launch_kg_pair_t<32>(h, M, sfa, t, y, clusters, st);
+        case 64: return launch_kg_pair_t<64>(h, M, sfa, t, y, clusters, st);
+        case 128: return launch_kg_pair_t<128>(h, M, sfa, t, y, clusters, st);
+      }
+    }
+  }
   switch (h->r) {
     case 0: return launch_kg_t<V, 0>(h, tma, M, sfa, t, y, st);
     case 16: return launch_kg_t<V, 16>(h, tma, M, sfa, t, y, st);
@@ -431,7 +545,7 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
   if (!d || !out) return SVDQ_ERR_INVALID_ARG;
   *out = nullptr;
   if (d->variant != SVDQ_INT4_G64_BF16 && d->variant != SVDQ_NVFP4_G16_E4M3) return SVDQ_ERR_INVALID_ARG;
-  if (d->flags & ~SVDQ_EPI_GELU) return SVDQ_ERR_INVALID_ARG;
+  if (d->flags & ~(SVDQ_EPI_GELU | SVDQ_GEMM_SM_PAIR)) return SVDQ_ERR_INVALID_ARG;
   const int64_t K = d->K, N = d->N, r = d->r;
   if (K < 128 || K % 128 != 0 || K > (1 << 20)) return SVDQ_ERR_SHAPE;
   if (N < 16 || N % 16 != 0 || N > (1 << 20)) return SVDQ_ERR_SHAPE;
@@ -572,6 +686,21 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
     h->tm_blr = h->tm_b;  // never read when r == 0
     h->tm_l1t = h->tm_b;
   }
+  if (d->variant == SVDQ_NVFP4_G16_E4M3) {
+    if ((s = make_tmap(&h->tm_b2, h->wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return fail(s);
+    if ((s = make_tmap(&h->tm_sfb2, h->wscales, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, 128,
+                       (h->npad / 128) * (K / 64), 128, 4, CU_TENSOR_MAP_SWIZZLE_NONE)) != SVDQ_OK)
+      return fail(s);
+    if (r > 0) {
+      if ((s = make_tmap(&h->tm_blr2, h->l2dup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->lr_cols, N,
+                         64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+        return fail(s);
+    } else {
+      h->tm_blr2 = h->tm_b2;  // never read when r == 0
+    }
+  }
   (void)G;
   *out = h;
   return SVDQ_OK;
@@ -617,8 +746,8 @@ svdq_status svdq_w4a4_gemm_lowrank_up(svdq_weights_t h, const uint8_t* act_codes
   if ((s = get_tm_a(h, act_codes, M)) != SVDQ_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const uint8_t* sfa = static_cast<const uint8_t*>(act_scales);
-  return h->variant == SVDQ_NVFP4_G16_E4M3 ? launch_kg_v<1>(h, h->tm_a, M, sfa, t, y, st)
-                                           : launch_kg_v<0>(h, h->tm_a, M, sfa, t, y, st);
+  return h->variant == SVDQ_NVFP4_G16_E4M3 ? launch_kg_v<1>(h, h->tm_a, act_codes, M, sfa, t, y, st)
+                                           : launch_kg_v<0>(h, h->tm_a, act_codes, M, sfa, t, y, st);
 }
 
 svdq_status svdq_linear_forward(svdq_weights_t h, const void* x, void* y, int64_t M, void* stream) {
