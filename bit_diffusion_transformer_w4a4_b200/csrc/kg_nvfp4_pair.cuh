@@ -21,8 +21,10 @@
 // Warp roles (640 threads per CTA):
 //   warp 0      TMA producer (both CTAs): transaction bytes of both CTAs are
 //               counted on the leader's full barrier
-//   warp 1      leader: scale-factor copies and MMAs for the pair; both CTAs:
-//               tensor-memory allocation (cta_group::2, same warp in both)
+//   warp 1      leader: MMAs for the pair; both CTAs: tensor-memory
+//               allocation (cta_group::2, same warp in both)
+//   warps 2, 3  leader: scale-factor copies for the pair (A's, B's), a stage
+//               ahead of the MMAs, from threads other than the MMA issuer
 //   warps 4-19  epilogue (both CTAs): drain this SM's accumulator half,
 //               prepare the next tile's low-rank operand rows, store
 // Cross-CTA signals: MMA completion is committed to the barrier at the same
@@ -84,6 +86,9 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   const uint32_t bar_drain = smem_u32(bars + 2 * NST + 3);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NST + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t bar_sfa = smem_u32(bars + 2 * NST + 5);        // leader: A's scales copied
+  const uint32_t bar_sfb = smem_u32(bars + 3 * NST + 5);        // leader: B's scales copied
+  const uint32_t bar_sf_drain = smem_u32(bars + 4 * NST + 5);   // two barriers
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -104,6 +109,12 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     mbar_init(bar_acc_empty, 2 * KG_EPI_WARPS);
     mbar_init(bar_lr_full, 2 * KG_EPI_WARPS);
     mbar_init(bar_drain, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_sfa + 8 * s, 1);
+      mbar_init(bar_sfb + 8 * s, 1);
+    }
+    mbar_init(bar_sf_drain, 1);
+    mbar_init(bar_sf_drain + 8, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -175,8 +186,6 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       constexpr uint32_t id_bf = idesc_bf16_f32(256, 256);
       const uint64_t dA0 = smem_desc(sbase, 16, S::SBO, SWZ_128B);
       const uint64_t dB0 = smem_desc(sbase + S::A_BYTES, 16, S::SBO, SWZ_128B);
-      const uint64_t dSFA0 = smem_desc(sbase + S::A_BYTES + S::B_BYTES, 0, 128, SWZ_NONE);
-      const uint64_t dSFB0 = smem_desc(sbase + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, 0, 128, SWZ_NONE);
       const uint64_t dLRA0 = smem_desc(sbase + S::ALR_OFF, 16, 1024, SWZ_128B);
       constexpr uint64_t kStage = S::STAGE >> 4;
       int s = 0;
@@ -186,19 +195,14 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         if (j > 0 && !(ok = wait_bounded_cl(bar_acc_empty, (j - 1) & 1, guard, 0x223))) break;
         tc_fence_after();
         for (int ks = 0; ks < nks; ++ks) {
-          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x224))) break;
+          if (!(ok = wait_bounded(bar_sfa + 8 * s, ph, guard, 0x224) &&
+                     wait_bounded(bar_sfb + 8 * s, ph, guard, 0x228)))
+            break;
           tc_fence_after();
           const uint64_t so = kStage * s;
           const int kv = min(KB, kblk - KB * ks);
           const uint32_t ca = tmem + S::SFA_COL + KB * 4 * s;
           const uint32_t cb = tmem + S::SFB_COL + KB * 8 * s;
-#pragma unroll
-          for (int kb = 0; kb < KB; ++kb) {
-            if (kb >= kv) break;
-            tmem_cp_32x128b_warpx4_pair(ca + 4 * kb, dSFA0 + so + 32 * kb);
-            tmem_cp_32x128b_warpx4_pair(cb + 8 * kb, dSFB0 + so + 32 * kb);
-            tmem_cp_32x128b_warpx4_pair(cb + 8 * kb + 4, dSFB0 + so + 32 * (KB + kb));
-          }
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) {
             if (kb >= kv) break;
@@ -213,7 +217,9 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           if (!(ok = wait_bounded_cl(bar_lr_full, j & 1, guard, 0x225))) break;
           tc_fence_after();
           for (int l = 0; l < S::LR_STAGES; ++l) {
-            if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x226))) break;
+            if (!(ok = wait_bounded(bar_sfa + 8 * s, ph, guard, 0x226) &&
+                       wait_bounded(bar_sfb + 8 * s, ph, guard, 0x229)))
+              break;
             tc_fence_after();
             const uint64_t so = kStage * s;
 #pragma unroll
@@ -233,6 +239,56 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       tc_commit_pair(bar_drain, 0x1);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < p.timeout_ns) {
+      }
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------ scale-factor copies (leader)
+    // Each copy lands in both CTAs' tensor memory, from each CTA's own stage;
+    // every stage completes the leader's ready barrier once, after the
+    // pair's data has landed (the leader's full barrier counts both CTAs).
+    if (lane == 0 && rank == 0) {
+      const bool is_a = warp == 2;
+      const uint32_t ready = is_a ? bar_sfa : bar_sfb;
+      const uint64_t d0 = is_a ? smem_desc(sbase + S::A_BYTES + S::B_BYTES, 0, 128, SWZ_NONE)
+                               : smem_desc(sbase + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, 0, 128, SWZ_NONE);
+      constexpr uint64_t kStage = S::STAGE >> 4;
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = cid; tile < num_tiles && ok; tile += nclu) {
+        for (int ks = 0; ks < nks; ++ks) {
+          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, is_a ? 0x22a : 0x22b))) break;
+          tc_fence_after();
+          const uint64_t d = d0 + kStage * s;
+          const int kv = min(KB, kblk - KB * ks);
+          if (is_a) {
+            const uint32_t ca = tmem + S::SFA_COL + KB * 4 * s;
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb)
+              if (kb < kv) tmem_cp_32x128b_warpx4_pair(ca + 4 * kb, d + 32 * kb);
+          } else {
+            const uint32_t cb = tmem + S::SFB_COL + KB * 8 * s;
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb)
+              if (kb < kv) {
+                tmem_cp_32x128b_warpx4_pair(cb + 8 * kb, d + 32 * kb);
+                tmem_cp_32x128b_warpx4_pair(cb + 8 * kb + 4, d + 32 * (KB + kb));
+              }
+          }
+          tc_commit_pair(ready + 8 * s, 0x1);
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+        for (int l = 0; l < S::LR_STAGES && ok; ++l) {
+          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x22c))) break;
+          tc_commit_pair(ready + 8 * s, 0x1);
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+      }
+      // this warp's copies have completed before tensor memory is freed
+      const uint32_t drain = bar_sf_drain + (is_a ? 0 : 8);
+      tc_commit_pair(drain, 0x1);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < p.timeout_ns) {
       }
     }
   } else if (warp >= 4) {

@@ -323,7 +323,7 @@ svdq_status get_tm_pair(svdq_weights* h, const void* codes, const void* scales, 
 template <int V>
 svdq_status launch_kg_v(svdq_weights* h, const CUtensorMap& tma, const uint8_t* codes, int64_t M,
                         const uint8_t* sfa, const float* t, void* y, cudaStream_t st) {
-  if (V == 1 && M > 128 && (h->flags & SVDQ_GEMM_SM_PAIR)) {
+  if (V == 1 && M > 128 && !(h->flags & SVDQ_GEMM_SINGLE_SM)) {
     int clusters = 0;
     switch (h->r) {
       case 0: clusters = pair_clusters<0>(h); break;
@@ -545,7 +545,7 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
   if (!d || !out) return SVDQ_ERR_INVALID_ARG;
   *out = nullptr;
   if (d->variant != SVDQ_INT4_G64_BF16 && d->variant != SVDQ_NVFP4_G16_E4M3) return SVDQ_ERR_INVALID_ARG;
-  if (d->flags & ~(SVDQ_EPI_GELU | SVDQ_GEMM_SM_PAIR)) return SVDQ_ERR_INVALID_ARG;
+  if (d->flags & ~(SVDQ_EPI_GELU | SVDQ_GEMM_SINGLE_SM)) return SVDQ_ERR_INVALID_ARG;
   const int64_t K = d->K, N = d->N, r = d->r;
   if (K < 128 || K % 128 != 0 || K > (1 << 20)) return SVDQ_ERR_SHAPE;
   if (N < 16 || N % 16 != 0 || N > (1 << 20)) return SVDQ_ERR_SHAPE;

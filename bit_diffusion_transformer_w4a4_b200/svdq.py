@@ -17,7 +17,7 @@ from . import build as _build
 INT4 = 0
 NVFP4 = 1
 EPI_GELU = 1
-GEMM_SM_PAIR = 2
+GEMM_SINGLE_SM = 2
 
 STATUS = {
     0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_SHAPE", 3: "SVDQ_ERR_ALIGNMENT",
@@ -122,10 +122,11 @@ def selftest_division(variant: int) -> tuple[int, int]:
 class SVDQWeights:
     """A loaded layer: owns a library handle (``svdq_weights_t``)."""
 
-    def __init__(self, pw, max_M: int, stream=None, sm_pair: bool = False):
+    def __init__(self, pw, max_M: int, stream=None, single_sm: bool = False):
         """``pw`` has fields variant, K, N, r, lam, L1, L2, codes, scales, bias, gelu
-        (host numpy arrays in the formats of ``svdq_weight_desc``).  ``sm_pair``
-        sets SVDQ_GEMM_SM_PAIR (NVFP4 GEMM on pairs of SMs when M > 128)."""
+        (host numpy arrays in the formats of ``svdq_weight_desc``).  ``single_sm``
+        sets SVDQ_GEMM_SINGLE_SM (NVFP4 GEMM on single SMs; by default it runs on
+        pairs of SMs when M > 128)."""
         self._keep = [np.ascontiguousarray(pw.lam, dtype=np.float32),
                       np.ascontiguousarray(pw.L1, dtype=np.uint16),
                       np.ascontiguousarray(pw.L2, dtype=np.uint16),
@@ -137,7 +138,7 @@ class SVDQWeights:
         self.max_M = int(max_M)
         self.gelu = bool(pw.gelu)
         d = WeightDesc(self.variant, self.K, self.N, self.r, self.max_M,
-                       (EPI_GELU if self.gelu else 0) | (GEMM_SM_PAIR if sm_pair else 0),
+                       (EPI_GELU if self.gelu else 0) | (GEMM_SINGLE_SM if single_sm else 0),
                        _ptr(lam), _ptr(L1) if self.r else 0, _ptr(L2) if self.r else 0,
                        _ptr(codes), _ptr(scales), _ptr(bias))
         h = ctypes.c_void_p(0)

@@ -68,12 +68,13 @@ typedef enum {
 
 /* svdq_weight_desc.flags */
 #define SVDQ_EPI_GELU 1u    /* apply GELU (tanh form) in the GEMM epilogue */
-/* NVFP4 only: when M > 128, run kernel 2 on pairs of SMs (a two-CTA cluster
- * per 256 x 256 tile, one M = 256 tensor-core MMA stream per pair) instead of
- * single SMs (128 x 256 tiles).  Both compute the same y up to fp32 summation
- * order; the single-SM kernel is the default because it measured faster on
- * B200 (fc1 4608 x 3072 x 12288: 127 vs 161 us). */
-#define SVDQ_GEMM_SM_PAIR 2u
+/* NVFP4 only: run kernel 2 on single SMs (128 x 256 tiles) for every M.  By
+ * default, when M > 128, it runs on pairs of SMs: a two-CTA cluster per
+ * 256 x 256 tile, one M = 256 tensor-core MMA stream per pair, which halves
+ * the B bytes each SM stages and so deepens the pipeline (B200, fc1
+ * 4608 x 3072 x 12288: 108.5 vs 118.8 us).  Both compute the same y up to
+ * fp32 summation order.  For comparison and tests. */
+#define SVDQ_GEMM_SINGLE_SM 2u
 
 typedef struct svdq_weights* svdq_weights_t;   /* opaque, library-owned */
 

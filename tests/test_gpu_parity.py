@@ -40,15 +40,15 @@ def test_activation_kernel(variant, r, M, K):
     PT.check_act(got, {"codes": codes, "scales": scales, "T": T}, r=r, label=f"v{variant} r{r} M{M} K{K}")
 
 
-# NVFP4 kernel 2 runs on single SMs, or on SM pairs for M > 128 when
-# SVDQ_GEMM_SM_PAIR is set: the NVFP4 cases run both kernels.
+# NVFP4 kernel 2 runs on SM pairs for M > 128, or on single SMs when
+# SVDQ_GEMM_SINGLE_SM is set: the NVFP4 cases run both kernels.
 KERNELS = [(INT4, False), (NVFP4, False), (NVFP4, True)]
-KIDS = ["int4", "nvfp4-1sm", "nvfp4-pair"]
+KIDS = ["int4", "nvfp4-pair", "nvfp4-1sm"]
 
 
-@pytest.mark.parametrize("variant,pair", KERNELS, ids=KIDS)
+@pytest.mark.parametrize("variant,single", KERNELS, ids=KIDS)
 @pytest.mark.parametrize("r", [0, 16, 32, 128])
-def test_gemm_isolated(variant, pair, r):
+def test_gemm_isolated(variant, single, r):
     """Kernel 2 alone, fed the oracle's activation codes / scales / T."""
     import torch
     M, K, N = 300, 512, 512
@@ -56,7 +56,7 @@ def test_gemm_isolated(variant, pair, r):
     inv = (np.float32(1) / pw.lam).astype(np.float32)
     codes, scales, T = O.quantize_act_lowrank_down(x, inv, pw.L1, variant)
     y_ref, Y_ref = O.gemm_lowrank_up(codes, scales, T, pw.codes, pw.scales, pw.L2, variant)
-    h = svdq.SVDQWeights(pw, M, sm_pair=pair)
+    h = svdq.SVDQWeights(pw, M, single_sm=single)
     sc = PT.tile_nvfp4_scales(scales, M, K) if variant == NVFP4 else scales.view(np.uint8).reshape(-1)
     tt = np.zeros((M, max(r, 1)), dtype=np.float32)
     tt[:, :r] = T
@@ -68,14 +68,14 @@ def test_gemm_isolated(variant, pair, r):
     PT.check_y(Yg, y_ref, Y_ref, label=f"gemm v{variant} r{r}")
 
 
-@pytest.mark.parametrize("variant,pair", KERNELS, ids=KIDS)
+@pytest.mark.parametrize("variant,single", KERNELS, ids=KIDS)
 @pytest.mark.parametrize("gelu,with_bias", [(False, False), (True, True), (False, True)])
 @pytest.mark.parametrize("M,K,N,r", [(300, 512, 448, 32), (129, 1024, 272, 16), (513, 384, 768, 64),
                                      (640, 768, 528, 128)])
-def test_forward_small(variant, pair, gelu, with_bias, M, K, N, r):
+def test_forward_small(variant, single, gelu, with_bias, M, K, N, r):
     """Ragged M and N (partial tiles), several K tiles, bias and GELU."""
     lay, x, pw = _prepped(M, K, N, r, variant, gelu=gelu, with_bias=with_bias)
-    h = svdq.SVDQWeights(pw, M, sm_pair=pair)
+    h = svdq.SVDQWeights(pw, M, single_sm=single)
     got = PT.gpu_forward(h, x, M)
     ref = O.linear_forward(x, pw)
     PT.check_act(got, ref, r=r, label="fwd")
@@ -122,16 +122,16 @@ def test_host_entry_point_matches_device(variant):
     assert np.array_equal(yh.numpy().view(np.uint16), dev["Y"])
 
 
-@pytest.mark.parametrize("variant,pair", KERNELS, ids=KIDS)
+@pytest.mark.parametrize("variant,single", KERNELS, ids=KIDS)
 @pytest.mark.parametrize("mask", [1, 2])
-def test_bounded_wait_reports_timeout(variant, pair, mask):
+def test_bounded_wait_reports_timeout(variant, single, mask):
     """A pipeline stage that is never filled: the kernel's bounded wait expires,
     the call reports SVDQ_ERR_DEVICE_TIMEOUT and the context stays usable."""
     M, K, N, r = 256, 1024, 512, 32
     lay = W.Layer("fault", M=M, K=K, N=N, r=r, variant=variant, config_id=62)
     pw = W.synthetic_packed(lay)
     x = W.activations(lay)
-    h = svdq.SVDQWeights(pw, M, sm_pair=pair)
+    h = svdq.SVDQWeights(pw, M, single_sm=single)
     ok = PT.gpu_forward(h, x, M)
     h.debug_set_fault(mask, 20000)                 # 20 ms limit
     import torch
@@ -152,8 +152,8 @@ def test_pair_and_single_sm_agree(M):
     lay = W.Layer("pair", M=M, K=K, N=N, r=r, variant=NVFP4, gelu=True, bias=True, config_id=63)
     pw = W.synthetic_packed(lay)
     x = W.activations(lay)
-    hp = svdq.SVDQWeights(pw, M, sm_pair=True)
-    hs = svdq.SVDQWeights(pw, M)
+    hp = svdq.SVDQWeights(pw, M)
+    hs = svdq.SVDQWeights(pw, M, single_sm=True)
     a = PT.gpu_forward(hp, x, M)
     b = PT.gpu_forward(hs, x, M)
     ref = O.linear_forward(x, pw)
