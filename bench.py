@@ -274,15 +274,19 @@ def run_ours(args, layer):
         raise RuntimeError("device status error in the end-to-end loop")
 
     pk, pk_src = peaks()
-    # dominant kernel: the 4-bit GEMM; FP4 dense peak = measured bf16 burst x 4 (9 / 2.25 PF nominal)
+    # dominant kernel: the 4-bit GEMM.  NVFP4 runs on the FP4 tensor path (dense
+    # peak = measured bf16 burst x 4, the 9 : 2.25 PF nominal ratio); INT4 on
+    # the int8 path (x 2, 4.5 : 2.25)
+    nvfp4 = layer.variant == W.NVFP4
     kg_flops = 2.0 * M * K * N + 2.0 * M * N * r
     achieved = kg_flops / (ms_kg * 1e-3) / 1e12
-    peak = pk["bf16_tflops"] * 4.0
+    ratio = 4.0 if nvfp4 else 2.0
+    peak = pk["bf16_tflops"] * ratio
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "nvfp4", "data": "synthetic",
+        "dtype": "nvfp4" if nvfp4 else "int4", "data": "synthetic",
         "config": {"workload": f"{layer.name} M{M} K{K} N{N} r{r}{' GELU' if layer.gelu else ''} "
                                f"{W.VARIANT_NAME[layer.variant]}",
                    "l2": "flushed before every step (256 MB write, outside the timed events)",
@@ -292,7 +296,9 @@ def run_ours(args, layer):
         "kernels_ms": {"quantize_act_lowrank_down": ms_kq, "w4a4_gemm_lowrank_up": ms_kg},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": recorded_traffic("w4a4_gemm_lowrank_up", args.workload),
-                     "peak_source": f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 4 (FP4:BF16 nominal 9:2.25)"},
+                     "peak_source": (f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 4 (FP4:BF16 nominal 9:2.25)"
+                                     if nvfp4 else
+                                     f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 2 (INT8:BF16 nominal 4.5:2.25)")},
         "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": 2 * args.steps,
