@@ -78,38 +78,9 @@ __device__ __forceinline__ void prep_lowrank_a(uint8_t* alr, const float* __rest
   }
 }
 
-// Store 64 fp32 accumulator columns of one row: + bias, GELU, bf16.
-__device__ __forceinline__ void store_row64(const KGParams& p, int gm, int n_base, const float* acc) {
-  if (gm >= p.M) return;
-  uint16_t* dst = p.y + static_cast<size_t>(gm) * p.N;
-#pragma unroll
-  for (int j8 = 0; j8 < 8; ++j8) {
-    const int n = n_base + 8 * j8;
-    if (n >= p.N) break;
-    float v[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = acc[8 * j8 + e];
-    if (p.bias != nullptr) {
-      const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
-      const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[2 * e] = __fadd_rn(v[2 * e], bf16lo(bw[e]));
-        v[2 * e + 1] = __fadd_rn(v[2 * e + 1], bf16hi(bw[e]));
-      }
-    }
-    if (p.gelu) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = gelu_tanh(v[e]);
-    }
-    *reinterpret_cast<uint4*>(dst + n) =
-        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                   pack_bf16x2(v[6], v[7]));
-  }
-}
-
-// Warp-cooperative form of store_row64 with full-line stores.  Lane l holds
-// 64 accumulator columns [n_base, n_base + 64) of row row0 + l.  After bias,
+// Epilogue store, warp-cooperative with full-line stores.  Lane l holds
+// 64 accumulator columns [n_base, n_base + 64) of row row0 + l: + bias,
+// GELU, bf16.  After bias,
 // GELU and bf16 packing each lane has eight 16-byte chunks of its row; an 8x8
 // transpose of those chunks inside each group of 8 lanes (three butterfly
 // stages of shfl.xor, stage b swapping bit b of the lane and chunk indices)
@@ -161,6 +132,61 @@ __device__ __forceinline__ void store_rows64_coalesced(const KGParams& p, int ro
   const int rg = row0 + (lane & ~7);
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
+    const int gm = rg + k;
+    if (gm < p.M)
+      *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(gm) * p.N + n) =
+          make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  }
+}
+
+// The same for 32 columns per lane: four 16-byte chunks, a 4 x 4 transpose
+// inside each group of 4 lanes (shfl.xor 1, 2), then each store writes, per
+// 4-lane group, a contiguous 64-byte row segment.  All 32 lanes must call it.
+__device__ __forceinline__ void store_rows32_coalesced(const KGParams& p, int row0, int n_base,
+                                                       const float* acc, int lane) {
+  uint32_t w[16];
+#pragma unroll
+  for (int j8 = 0; j8 < 4; ++j8) {
+    const int n = n_base + 8 * j8;
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = acc[8 * j8 + e];
+    if (p.bias != nullptr && n < p.N) {
+      const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
+      const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = __fadd_rn(v[2 * e], bf16lo(bw[e]));
+        v[2 * e + 1] = __fadd_rn(v[2 * e + 1], bf16hi(bw[e]));
+      }
+    }
+    if (p.gelu) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = gelu_tanh(v[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w[4 * j8 + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+  }
+#pragma unroll
+  for (int b = 1; b < 4; b <<= 1) {
+    const bool up = (lane & b) != 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c & b) continue;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t send = up ? w[4 * c + e] : w[4 * (c | b) + e];
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, b);
+        if (up) w[4 * c + e] = recv;
+        else w[4 * (c | b) + e] = recv;
+      }
+    }
+  }
+  const int n = n_base + 8 * (lane & 3);
+  if (n >= p.N) return;
+  const int rg = row0 + (lane & ~3);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
     const int gm = rg + k;
     if (gm < p.M)
       *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(gm) * p.N + n) =

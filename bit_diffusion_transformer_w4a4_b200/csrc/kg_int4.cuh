@@ -12,6 +12,13 @@
 // Mechanics of 4-Bit Efficiency and SVDQuant" (W4A4 residual + 16-bit
 // low-rank branch).
 //
+// Tile 128 x 128: tensor memory holds four 128-column s32 accumulators, so
+// the MMAs run up to three groups ahead of the epilogue's rescale, and each
+// epilogue thread keeps 32 fp32 sums (one 32-column tensor-memory load and
+// paired fp32 arithmetic per group).  The rescale -- a convert, a multiply
+// and an add per output and group, M N K/64 of them -- is the bound of this
+// variant; the int8 MMAs take a fraction of it.
+//
 // Warp roles (640 threads):
 //   warp 0      TMA producer: packed activation codes (32B swizzle) and int8
 //               weight codes (64B swizzle) for one 64-group per stage
@@ -25,18 +32,42 @@
 
 namespace svdq {
 
+constexpr int KGI4_BN = 128;   // tile columns (output features)
+constexpr int KGI4_BUFS = 4;   // s32 accumulators of 128 columns in tensor memory
+
 template <int R>
 struct KGI4Smem {
-  static constexpr int STAGES = R >= 128 ? 5 : 6;
-  static constexpr int APK_BYTES = KG_BM * 32;   // 128 rows x 32 B packed (64 codes)
-  static constexpr int A8_BYTES = KG_BM * 64;    // 128 rows x 64 int8
-  static constexpr int B_BYTES = KG_BN * 64;     // 256 rows x 64 int8
+  static constexpr int STAGES = R >= 128 ? 8 : (R >= 64 ? 9 : 10);
+  static constexpr int APK_BYTES = KG_BM * 32;    // 128 rows x 32 B packed (64 codes)
+  static constexpr int A8_BYTES = KG_BM * 64;     // 128 rows x 64 int8
+  static constexpr int B_BYTES = KGI4_BN * 64;    // 128 rows x 64 int8
   static constexpr int STAGE = APK_BYTES + A8_BYTES + B_BYTES;
   static constexpr int LR_CHUNKS = R > 0 ? (2 * R + 63) / 64 : 0;
   static constexpr int ALR_OFF = STAGES * STAGE;
   static constexpr int BAR_OFF = ALR_OFF + LR_CHUNKS * 16384;
   static constexpr int TOTAL = BAR_OFF + 512 + 1024;
+  static_assert(STAGE % 1024 == 0, "stages keep the swizzle alignment");
+  static_assert(TOTAL <= 232448, "shared memory per CTA");
 };
+
+// Paired fp32 arithmetic (one instruction per two lanes of data).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ float f2_lo(uint64_t a) { return __uint_as_float(static_cast<uint32_t>(a)); }
+__device__ __forceinline__ float f2_hi(uint64_t a) { return __uint_as_float(static_cast<uint32_t>(a >> 32)); }
 
 // 8 two's-complement nibbles (element 0 in the low nibble) -> 8 int8 bytes.
 __device__ __forceinline__ uint2 unpack_s4x8(uint32_t w) {
@@ -65,11 +96,11 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   const uint32_t bar_full = smem_u32(bars);
   const uint32_t bar_ready = smem_u32(bars + NST);
   const uint32_t bar_empty = smem_u32(bars + 2 * NST);
-  const uint32_t bar_gfull = smem_u32(bars + 3 * NST);       // [2]
-  const uint32_t bar_gempty = smem_u32(bars + 3 * NST + 2);  // [2]
-  const uint32_t bar_lr_full = smem_u32(bars + 3 * NST + 4);
-  const uint32_t bar_drain = smem_u32(bars + 3 * NST + 5);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NST + 6);
+  const uint32_t bar_gfull = smem_u32(bars + 3 * NST);                  // [KGI4_BUFS]
+  const uint32_t bar_gempty = smem_u32(bars + 3 * NST + KGI4_BUFS);     // [KGI4_BUFS]
+  const uint32_t bar_lr_full = smem_u32(bars + 3 * NST + 2 * KGI4_BUFS);
+  const uint32_t bar_drain = smem_u32(bars + 3 * NST + 2 * KGI4_BUFS + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NST + 2 * KGI4_BUFS + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -84,7 +115,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       mbar_init(bar_ready + 8 * s, 64);   // the 64 transform threads
       mbar_init(bar_empty + 8 * s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < KGI4_BUFS; ++b) {
       mbar_init(bar_gfull + 8 * b, 1);
       mbar_init(bar_gempty + 8 * b, KG_EPI_WARPS);
     }
@@ -121,7 +152,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
             const uint32_t fb = bar_full + 8 * s;
             mbar_expect_tx(fb, S::APK_BYTES + S::B_BYTES);
             tma_load_2d(st, &tm_a, fb, g * 32, mb * KG_BM);
-            tma_load_2d(st + S::APK_BYTES + S::A8_BYTES, &tm_b, fb, g * 64, nb * KG_BN);
+            tma_load_2d(st + S::APK_BYTES + S::A8_BYTES, &tm_b, fb, g * 64, nb * KGI4_BN);
             issued |= 1u << s;
             issued_par = (issued_par & ~(1u << s)) | (ph << s);
           }
@@ -131,9 +162,9 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           if (!(ok = wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x302))) break;
           issued &= ~(1u << s);
           const uint32_t fb = bar_full + 8 * s;
-          mbar_expect_tx(fb, KG_BN * 64);
+          mbar_expect_tx(fb, KGI4_BN * 64);
           tma_load_2d(sbase + s * S::STAGE + S::APK_BYTES + S::A8_BYTES, &tm_blr, fb, l * 32,
-                      nb * KG_BN);
+                      nb * KGI4_BN);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == NST) { s = 0; ph ^= 1; }
@@ -144,15 +175,15 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      constexpr uint32_t id_s8 = idesc_s8_s32(KG_BM, KG_BN);
-      constexpr uint32_t id_bf = idesc_bf16_f32(KG_BM, KG_BN);
+      constexpr uint32_t id_s8 = idesc_s8_s32(KG_BM, KGI4_BN);
+      constexpr uint32_t id_bf = idesc_bf16_f32(KG_BM, KGI4_BN);
       const uint32_t alr = sbase + S::ALR_OFF;
       int s = 0;
       uint32_t ph = 0, gc = 0;
       bool ok = true;
       for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
         for (int g = 0; g < ng; ++g, ++gc) {
-          const uint32_t b = gc & 1, use = gc >> 1;
+          const uint32_t b = gc % KGI4_BUFS, use = gc / KGI4_BUFS;
           if (!(ok = wait_bounded(bar_gempty + 8 * b, (use & 1) ^ 1, guard, 0x303))) break;
           if (!(ok = wait_bounded(bar_ready + 8 * s, ph, guard, 0x304))) break;
           if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x305))) break;
@@ -162,7 +193,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           for (int kk = 0; kk < 2; ++kk) {
             const uint64_t a = smem_desc(st + S::APK_BYTES + kk * 32, 16, 512, SWZ_64B);
             const uint64_t bd = smem_desc(st + S::APK_BYTES + S::A8_BYTES + kk * 32, 16, 512, SWZ_64B);
-            mma_s8(tmem + b * 256, a, bd, id_s8, kk);
+            mma_s8(tmem + b * KGI4_BN, a, bd, id_s8, kk);
           }
           tc_commit(bar_empty + 8 * s);
           tc_commit(bar_gfull + 8 * b);
@@ -170,7 +201,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         }
         if (!ok) break;
         if (R > 0) {
-          const uint32_t b = gc & 1, use = gc >> 1;
+          const uint32_t b = gc % KGI4_BUFS, use = gc / KGI4_BUFS;
           if (!(ok = wait_bounded(bar_gempty + 8 * b, (use & 1) ^ 1, guard, 0x306))) break;
           if (!(ok = wait_bounded(bar_lr_full, j & 1, guard, 0x307))) break;
           tc_fence_after();
@@ -184,7 +215,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
               const int kk = 2 * l + k2;
               const uint64_t a = smem_desc(alr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, SWZ_128B);
               const uint64_t bd = smem_desc(bst + k2 * 32, 16, 512, SWZ_64B);
-              mma_bf16(tmem + b * 256, a, bd, id_bf, kk != 0);
+              mma_bf16(tmem + b * KGI4_BN, a, bd, id_bf, kk != 0);
             }
             tc_commit(bar_empty + 8 * s);
             if (++s == NST) { s = 0; ph ^= 1; }
@@ -244,7 +275,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     uint8_t* alr = smem + S::ALR_OFF;
     const __nv_bfloat16* sx_all = reinterpret_cast<const __nv_bfloat16*>(p.sfa);
     const float* sw_all = reinterpret_cast<const float*>(p.sfb);
-    const int npad = p.num_n * KG_BN;
+    const int npad = (p.N + 255) / 256 * 256;  // row stride of the weight-scale table
     if constexpr (R > 0) {
       if (static_cast<int>(blockIdx.x) < num_tiles) {
         prep_lowrank_a<R>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid);
@@ -257,56 +288,55 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
       const int mb = tile % p.num_m, nb = tile / p.num_m;
       const int gm = mb * KG_BM + row;
-      const int n_base = nb * KG_BN + cs * 64;
+      const int n_base = nb * KGI4_BN + cs * 32;
       const __nv_bfloat16* sxr = sx_all + static_cast<size_t>(gm < p.M ? gm : 0) * ng;
-      float acc[64];
+      uint64_t acc[16];  // 32 fp32 sums, in pairs
 #pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+      for (int i = 0; i < 16; ++i) acc[i] = 0ull;
       float sx_next = gm < p.M ? __bfloat162float(sxr[0]) : 0.0f;
       for (int g = 0; g < ng; ++g, ++gc) {
-        const uint32_t b = gc & 1, use = gc >> 1;
+        const uint32_t b = gc % KGI4_BUFS, use = gc / KGI4_BUFS;
         const float sx = sx_next;
         if (g + 1 < ng) sx_next = gm < p.M ? __bfloat162float(sxr[g + 1]) : 0.0f;
+        const uint64_t sx2 = f2_pack(sx, sx);
+        const float4* swr = reinterpret_cast<const float4*>(sw_all + static_cast<size_t>(g) * npad + n_base);
         if (!(ok = __all_sync(0xffffffffu, wait_bounded(bar_gfull + 8 * b, use & 1, guard, 0x30a)))) break;
         tc_fence_after();
-        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * 256 + cs * 64;
-        const float4* swr = reinterpret_cast<const float4*>(sw_all + static_cast<size_t>(g) * npad + n_base);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          uint32_t v[16];
-          tmem_ld_x16(ta + 16 * h, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i4 = 0; i4 < 4; ++i4) {
-            const float4 w = __ldg(swr + 4 * h + i4);
-            const int i = 16 * h + 4 * i4;
-            acc[i] = __fmaf_rn(__int2float_rn(static_cast<int>(v[4 * i4])), sx * w.x, acc[i]);
-            acc[i + 1] = __fmaf_rn(__int2float_rn(static_cast<int>(v[4 * i4 + 1])), sx * w.y, acc[i + 1]);
-            acc[i + 2] = __fmaf_rn(__int2float_rn(static_cast<int>(v[4 * i4 + 2])), sx * w.z, acc[i + 2]);
-            acc[i + 3] = __fmaf_rn(__int2float_rn(static_cast<int>(v[4 * i4 + 3])), sx * w.w, acc[i + 3]);
-          }
-        }
+        uint32_t v[32];
+        tmem_ld_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * KGI4_BN + cs * 32, v);
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_gempty + 8 * b);
+        // acc += (s_x * s_w[n]) * float(P[n]), two columns per instruction
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 w = __ldg(swr + i4);
+          const uint64_t s01 = f2_mul(sx2, f2_pack(w.x, w.y));
+          const uint64_t s23 = f2_mul(sx2, f2_pack(w.z, w.w));
+          const uint64_t p01 = f2_pack(__int2float_rn(static_cast<int>(v[4 * i4])),
+                                       __int2float_rn(static_cast<int>(v[4 * i4 + 1])));
+          const uint64_t p23 = f2_pack(__int2float_rn(static_cast<int>(v[4 * i4 + 2])),
+                                       __int2float_rn(static_cast<int>(v[4 * i4 + 3])));
+          acc[2 * i4] = f2_fma(p01, s01, acc[2 * i4]);
+          acc[2 * i4 + 1] = f2_fma(p23, s23, acc[2 * i4 + 1]);
+        }
       }
       if (!ok) break;
       if constexpr (R > 0) {
-        const uint32_t b = gc & 1, use = gc >> 1;
+        const uint32_t b = gc % KGI4_BUFS, use = gc / KGI4_BUFS;
         if (!(ok = __all_sync(0xffffffffu, wait_bounded(bar_gfull + 8 * b, use & 1, guard, 0x30b)))) break;
         tc_fence_after();
-        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * 256 + cs * 64;
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          uint32_t v[16];
-          tmem_ld_x16(ta + 16 * h, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) acc[16 * h + i] = __fadd_rn(acc[16 * h + i], __uint_as_float(v[i]));
-        }
+        uint32_t v[32];
+        tmem_ld_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * KGI4_BN + cs * 32, v);
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_gempty + 8 * b);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          acc[i] = f2_pack(__fadd_rn(f2_lo(acc[i]), __uint_as_float(v[2 * i])),
+                           __fadd_rn(f2_hi(acc[i]), __uint_as_float(v[2 * i + 1])));
         ++gc;
         const int next = tile + gridDim.x;
         if (next < num_tiles) {
@@ -316,7 +346,13 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           mbar_arrive(bar_lr_full);
         }
       }
-      store_rows64_coalesced(p, mb * KG_BM + q * 32, n_base, acc, lane);
+      float out[32];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        out[2 * i] = f2_lo(acc[i]);
+        out[2 * i + 1] = f2_hi(acc[i]);
+      }
+      store_rows32_coalesced(p, mb * KG_BM + q * 32, n_base, out, lane);
     }
   }
 

@@ -222,7 +222,7 @@ svdq_status launch_kg_t(svdq_weights* h, const CUtensorMap& tma, int64_t M, cons
   p.N = static_cast<int>(h->N);
   p.K = static_cast<int>(h->K);
   p.num_m = static_cast<int>(cdiv(M, KG_BM));
-  p.num_n = static_cast<int>(cdiv(h->N, KG_BN));
+  p.num_n = static_cast<int>(cdiv(h->N, V == 1 ? KG_BN : KGI4_BN));
   p.gelu = (h->flags & SVDQ_EPI_GELU) ? 1 : 0;
   p.err = h->err;
   p.debug_mask = h->debug_mask;
@@ -669,15 +669,17 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
   const uint32_t rowb = wide ? 128 : 64;
   const CUtensorMapSwizzle swz = wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   h->stage_row_bytes = rowb;
+  // B tiles: 256 rows for the NVFP4 single-SM kernel, 128 for the INT4 kernel
+  const uint32_t brows = d->variant == SVDQ_NVFP4_G16_E4M3 ? 256 : KGI4_BN;
   svdq_status s = d->variant == SVDQ_NVFP4_G16_E4M3
                       ? make_tmap(&h->tm_b, h->wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N,
-                                  rowb, 256, swz)
+                                  rowb, brows, swz)
                       : make_tmap(&h->tm_b, h->wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, 64,
-                                  256, CU_TENSOR_MAP_SWIZZLE_64B);
+                                  brows, CU_TENSOR_MAP_SWIZZLE_64B);
   if (s != SVDQ_OK) return fail(s);
   if (r > 0) {
     if ((s = make_tmap(&h->tm_blr, h->l2dup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->lr_cols, N,
-                       rowb / 2, 256, swz)) != SVDQ_OK)
+                       rowb / 2, brows, swz)) != SVDQ_OK)
       return fail(s);
     if ((s = make_tmap(&h->tm_l1t, h->l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, r, 64,
                        static_cast<uint32_t>(r), CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
