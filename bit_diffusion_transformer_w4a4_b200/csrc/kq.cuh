@@ -83,6 +83,23 @@ __device__ __forceinline__ uint32_t e2m1x8(const float* v) {
       : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
   return out;
 }
+// Largest magnitude of the 2n bf16 values held in n packed words, as fp32:
+// pairwise magnitude maxima on bf16x2 (max.xorsign.abs keeps the larger
+// |value|; its sign is not used), then the larger of the two halves.  Exact:
+// only comparisons.
+template <int NW>
+__device__ __forceinline__ float bf16_amax(const uint32_t* w) {
+  uint32_t m[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) m[i] = w[i];
+#pragma unroll
+  for (int step = 1; step < NW; step *= 2)
+#pragma unroll
+    for (int i = 0; i + step < NW; i += 2 * step)
+      asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[i]) : "r"(m[i]), "r"(m[i + step]));
+  return fmaxf(fabsf(bf16lo(m[0])), fabsf(bf16hi(m[0])));
+}
+
 // Round half to even to an integer in [-8, 7], two's complement nibble.
 __device__ __forceinline__ uint32_t int4_rn(float v) {
   v = fminf(fmaxf(v, -8.0f), 7.0f);
@@ -273,10 +290,7 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
         uint32_t sc = 0;
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-          float a = 0.0f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            a = fmaxf(a, fmaxf(fabsf(bf16lo(w[8 * g + e])), fabsf(bf16hi(w[8 * g + e]))));
+          const float a = bf16_amax<8>(w + 8 * g);
           const uint32_t code = e4m3_rn(div_by_scale(a, 6.0f, kRcp6));
           const float s_ = e4m3_value(code);
           sc |= code << (8 * g);
@@ -306,9 +320,8 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
           *reinterpret_cast<uint32_t*>(sp) = sc;
         }
       } else {
-        float a = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) a = fmaxf(a, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+        const float a = fmaxf(fmaxf(bf16_amax<8>(w), bf16_amax<8>(w + 8)),
+                              fmaxf(bf16_amax<8>(w + 16), bf16_amax<8>(w + 24)));
         const __nv_bfloat16 sb = __float2bfloat16_rn(div_by_scale(a, 7.0f, kRcp7));
         const float s_ = __bfloat162float(sb);
         if (s_ >= kMinFastScale && s_ < kMaxFastScale) {
@@ -325,9 +338,10 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
             packed[j] = pk;
           }
         } else if (s_ > 0.0f) {  // scale outside the fast path's range: exact division
-#pragma unroll 1
+#pragma unroll
           for (int j = 0; j < 8; ++j) {
             uint32_t pk = 0;
+#pragma unroll
             for (int e = 0; e < 4; ++e) {
               const uint32_t ww = w[4 * j + e];
               pk |= int4_rn(__fdiv_rn(bf16lo(ww), s_)) << (8 * e);
