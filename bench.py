@@ -167,12 +167,30 @@ def run_reference(args, layer):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": f"{layer.name} M{layer.M} K{layer.K} N{layer.N} r{layer.r}"
-                                   f"{' GELU' if layer.gelu else ''} NVFP4",
+                                   f"{' GELU' if layer.gelu else ''} {W.VARIANT_NAME[layer.variant]}",
                        "step_sample_rows": nrows},
             "cpu_baseline": {k: times[-1][k] for k in ("unit", "cores", "kind", "sample")}
             | {"value": tflops},
             "e2e": {"value": tflops, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank values across the process group (the
+    slowest rank defines a multi-GPU step); identity on one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, flops_per_rank: float, ms_step: float) -> float:
+    """Whole-job TFLOPS: every rank processes its own batch (weak scaling),
+    timed by the slowest rank."""
+    return world * flops_per_rank / (ms_step * 1e-3) / 1e12
 
 
 def run_ours(args, layer):
@@ -243,13 +261,10 @@ def run_ours(args, layer):
     ms_step = statistics.mean(a + b for a, b in zip(t_kq, t_kg))
     ms_kg = statistics.mean(t_kg)
     ms_kq = statistics.mean(t_kq)
-    if world > 1:
-        tt = torch.tensor([ms_step, ms_kg, ms_kq], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step, ms_kg, ms_kq = tt.tolist()
+    ms_step, ms_kg, ms_kq = max_over_ranks([ms_step, ms_kg, ms_kq], "cuda")
 
     flops = layer.flops()
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = job_throughput(world, flops, ms_step)
 
     # end to end through the host entry point (pinned buffers, copies timed)
     xh = torch.from_numpy(x_bits.view(np.int16)).pin_memory()
@@ -266,10 +281,7 @@ def run_ours(args, layer):
     e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([ms_e2e], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_e2e = tt.item()
+    (ms_e2e,) = max_over_ranks([ms_e2e], "cuda")
     if h.device_status() != 0:
         raise RuntimeError("device status error in the end-to-end loop")
 
@@ -299,7 +311,7 @@ def run_ours(args, layer):
                      "peak_source": (f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 4 (FP4:BF16 nominal 9:2.25)"
                                      if nvfp4 else
                                      f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 2 (INT8:BF16 nominal 4.5:2.25)")},
-        "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS",
+        "e2e": {"value": job_throughput(world, flops, ms_e2e), "unit": "TFLOPS",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
