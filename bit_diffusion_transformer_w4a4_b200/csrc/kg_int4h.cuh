@@ -1,0 +1,320 @@
+// Kernel 2, INT4 variant on 16-bit tensor cores (opt-in: SVDQ_INT4_F16):
+// the same product as kg_int4_kernel,
+//   acc[m,n] = sum_g s_x[m,g] s_w[n,g] sum_{k in g} q_x[m,k] q_w[n,k],
+// computed as one fp16 GEMM of the dequantised operands
+//   A[m,k] = s_x[m,g(k)] q_x[m,k],   B[n,k] = s_w[n,g(k)] q_w[n,k].
+// Both are exact in fp16 while the scales stay in fp16's range: a bf16 scale
+// has 8 significant bits and |q| <= 8 has at most 3, so the product has at
+// most 11 -- fp16's precision -- and every A*B product is exact in the fp32
+// accumulator.  Only the summation order differs from the per-group form.
+// The per-group rescale of the int8 kernel (M N K/64 conversions and
+// multiply-adds, latency-bound per group) disappears: one epilogue per tile.
+//
+// Method: "Nunchaku 1.3.0 for Python3.14.x & alpha" (note.com), section
+// "SVDQ-FP4 on Blackwell", part "1. INT4" (INT4 -8..+7, W ~ int4 * scale);
+// "Nunchaku Lite ... integrated into Diffusers" (axbrief.com), section "The
+// Mechanics of 4-Bit Efficiency and SVDQuant" (W4A4 residual + 16-bit
+// low-rank branch).
+//
+// Weights arrive dequantised (fp16 [N x K], prepared at load, exactness
+// checked there); activations are dequantised per stage in shared memory.
+// Persistent CTAs, one per SM, tile 128 x 256, one 64-group per stage.
+// Warp roles (640 threads):
+//   warp 0      TMA producer: packed activation codes (32B swizzle), fp16
+//               weight tile (128B swizzle)
+//   warp 1      MMA issuer (kind::f16, fp16 x fp16, four k-steps of 16 per
+//               stage; low-rank bf16 k-steps), tensor-memory owner
+//   warps 2-3   dequantise the activation codes: q (from the nibble) times
+//               s_x, written as fp16 in the MMA's 128B-swizzled layout
+//   warps 4-19  epilogue: drain the accumulator, next tile's low-rank
+//               operand, bias + GELU + bf16 stores
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "kg_common.cuh"
+
+namespace svdq {
+
+// Largest activation scale whose products with |q| <= 7 stay finite in fp16
+// (7 * s <= 65504).  Larger scales are reported as a device error.
+constexpr float kInt4F16MaxScale = 9357.0f;
+
+template <int R>
+struct KGI4HSmem {
+  static constexpr int STAGES = R >= 64 ? 3 : 4;
+  static constexpr int APK_BYTES = KG_BM * 32;   // 128 rows x 32 B packed (64 codes)
+  static constexpr int AH_BYTES = KG_BM * 128;   // 128 rows x 64 fp16
+  static constexpr int B_BYTES = KG_BN * 128;    // 256 rows x 64 fp16
+  static constexpr int STAGE = APK_BYTES + AH_BYTES + B_BYTES;
+  static constexpr int LR_CHUNKS = R > 0 ? (2 * R + 63) / 64 : 0;
+  static constexpr int LR_STEPS = R / 8;                      // bf16 k-steps of 16 over [T_hi | T_lo]
+  static constexpr int LR_STAGES = (LR_STEPS + 3) / 4;        // a 128-byte B row holds 4 k-steps
+  static constexpr int ALR_OFF = STAGES * STAGE;
+  static constexpr int BAR_OFF = ALR_OFF + LR_CHUNKS * 16384;
+  static constexpr int TOTAL = BAR_OFF + 256 + 1024;
+  static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static_assert(TOTAL <= 232448, "shared memory per CTA");
+};
+
+// kind::f16 with fp16 A and B, fp32 accumulate, K-major both.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Eight INT4 codes (two's complement nibbles, element 0 low) times the scale
+// pair s2 -> four fp16x2 words.  q + 8 = q xor 8 for a 4-bit code; the fp16
+// with bits 0x6400 | u is 1024 + u, so subtracting 1032 gives q exactly.
+__device__ __forceinline__ void dequant8_f16(uint32_t w, uint32_t s2, uint32_t* out) {
+  const uint32_t u = w ^ 0x88888888u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t b = (u >> (8 * j)) & 0xFFu;
+    const uint32_t h = ((b & 0x0Fu) | ((b & 0xF0u) << 12)) | 0x64006400u;
+    uint32_t q2, r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q2) : "r"(h), "r"(0x64086408u));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(q2), "r"(s2));
+    out[j] = r;
+  }
+}
+
+template <int R>
+__global__ void __launch_bounds__(KG_THREADS, 1)
+    kg_int4h_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                    const __grid_constant__ CUtensorMap tm_blr, KGParams p) {
+  using S = KGI4HSmem<R>;
+  constexpr int NST = S::STAGES;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+  const uint32_t bar_full = smem_u32(bars);
+  const uint32_t bar_ready = smem_u32(bars + NST);       // dequantised A written
+  const uint32_t bar_empty = smem_u32(bars + 2 * NST);
+  const uint32_t bar_acc_full = smem_u32(bars + 3 * NST);
+  const uint32_t bar_acc_empty = smem_u32(bars + 3 * NST + 1);
+  const uint32_t bar_lr_full = smem_u32(bars + 3 * NST + 2);
+  const uint32_t bar_drain = smem_u32(bars + 3 * NST + 3);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NST + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Guard guard{p.err, abort_flag, p.timeout_ns};
+  const int num_tiles = p.num_m * p.num_n;
+  const int ng = p.K / 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_ready + 8 * s, 64);  // the 64 dequantising threads
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_acc_full, 1);
+    mbar_init(bar_acc_empty, KG_EPI_WARPS);
+    mbar_init(bar_lr_full, KG_EPI_WARPS * 32);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_b);
+      if (R > 0) tma_prefetch_desc(&tm_blr);
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
+        const int mb = tile % p.num_m, nb = tile / p.num_m;
+        for (int g = 0; g < ng; ++g) {
+          if (!(ok = wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x341))) break;
+          issued &= ~(1u << s);
+          if (!((p.debug_mask & 1u) && j == 0 && g == 1)) {  // test hook: leave one stage empty
+            const uint32_t st = sbase + s * S::STAGE;
+            const uint32_t fb = bar_full + 8 * s;
+            mbar_expect_tx(fb, S::APK_BYTES + S::B_BYTES);
+            tma_load_2d(st, &tm_a, fb, g * 32, mb * KG_BM);
+            tma_load_2d(st + S::APK_BYTES + S::AH_BYTES, &tm_b, fb, g * 64, nb * KG_BN);
+            issued |= 1u << s;
+            issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          }
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+        for (int l = 0; l < S::LR_STAGES && ok; ++l) {
+          if (!(ok = wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x342))) break;
+          issued &= ~(1u << s);
+          const uint32_t fb = bar_full + 8 * s;
+          mbar_expect_tx(fb, S::B_BYTES);
+          tma_load_2d(sbase + s * S::STAGE + S::APK_BYTES + S::AH_BYTES, &tm_blr, fb, l * 64, nb * KG_BN);
+          issued |= 1u << s;
+          issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+      }
+      if (*abort_flag) drain_loads(bar_full, issued, issued_par, NST, p.timeout_ns);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t id_h = idesc_f16_f32(KG_BM, KG_BN);
+      constexpr uint32_t id_bf = idesc_bf16_f32(KG_BM, KG_BN);
+      const uint64_t dA0 = smem_desc(sbase + S::APK_BYTES, 16, 1024, SWZ_128B);
+      const uint64_t dB0 = smem_desc(sbase + S::APK_BYTES + S::AH_BYTES, 16, 1024, SWZ_128B);
+      const uint64_t dLRA0 = smem_desc(sbase + S::ALR_OFF, 16, 1024, SWZ_128B);
+      constexpr uint64_t kStage = S::STAGE >> 4;
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
+        if (j > 0 && !(ok = wait_bounded(bar_acc_empty, (j - 1) & 1, guard, 0x343))) break;
+        tc_fence_after();
+        for (int g = 0; g < ng; ++g) {
+          if (!(ok = wait_bounded(bar_ready + 8 * s, ph, guard, 0x344))) break;
+          tc_fence_after();
+          const uint64_t so = kStage * s;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem, dA0 + so + 2 * kk, dB0 + so + 2 * kk, id_h, (g | kk) != 0);
+          tc_commit(bar_empty + 8 * s);
+          if (++s == NST) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        if (R > 0) {
+          if (!(ok = wait_bounded(bar_lr_full, j & 1, guard, 0x345))) break;
+          tc_fence_after();
+          for (int l = 0; l < S::LR_STAGES; ++l) {
+            if (!(ok = wait_bounded(bar_ready + 8 * s, ph, guard, 0x346))) break;
+            tc_fence_after();
+            const uint64_t so = kStage * s;
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) {
+              const int kk = 4 * l + k2;  // k-step over [T_hi | T_lo]
+              if (kk < S::LR_STEPS)
+                mma_bf16(tmem, dLRA0 + (kk / 4) * 1024 + (kk % 4) * 2, dB0 + so + 2 * k2, id_bf, 1);
+            }
+            tc_commit(bar_empty + 8 * s);
+            if (++s == NST) { s = 0; ph ^= 1; }
+          }
+          if (!ok) break;
+        }
+        tc_commit(bar_acc_full);
+      }
+      // drain: every MMA issued so far has completed before tensor memory is freed
+      tc_commit(bar_drain);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < p.timeout_ns) {
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------ dequantise activations
+    const int tt = threadIdx.x - 64;  // 0..63: rows tt and tt + 64
+    const __nv_bfloat16* sx_all = reinterpret_cast<const __nv_bfloat16*>(p.sfa);
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int mb = tile % p.num_m;
+      for (int g = 0; g < ng; ++g) {
+        // this group's scales of the two rows (rows past M read as 0)
+        float sx[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int gm = mb * KG_BM + tt + 64 * h;
+          sx[h] = gm < p.M ? __bfloat162float(sx_all[static_cast<size_t>(gm) * ng + g]) : 0.0f;
+        }
+        if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x349))) break;
+        const uint8_t* apk = smem + s * S::STAGE;
+        uint8_t* ah = smem + s * S::STAGE + S::APK_BYTES;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int row = tt + 64 * h;
+          if (sx[h] > kInt4F16MaxScale) atomicCAS(p.err, 0, 0x34f);  // fp16 would overflow
+          const __half2 s2h = __float2half2_rn(sx[h]);
+          const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&s2h);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(apk + swz_off(row, c, 32));
+            uint32_t o[16];
+            dequant8_f16(v.x, s2, o);
+            dequant8_f16(v.y, s2, o + 4);
+            dequant8_f16(v.z, s2, o + 8);
+            dequant8_f16(v.w, s2, o + 12);
+            // 32 codes = 4 chunks of 8 fp16 (16 bytes) of the 128-byte row
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint4*>(ah + swz_off(row, 4 * c + q, 128)) =
+                  make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar_ready + 8 * s);
+        if (++s == NST) { s = 0; ph ^= 1; }
+      }
+      // low-rank stages carry only the B operand; still pass each one through
+      // the ready barrier so its phase stays in step with the stage ring
+      for (int l = 0; l < S::LR_STAGES && ok; ++l) {
+        if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x34c))) break;
+        mbar_arrive(bar_ready + 8 * s);
+        if (++s == NST) { s = 0; ph ^= 1; }
+      }
+    }
+  } else {
+    // ----------------------------------------------------------------- epilogue
+    const int e = warp - 4;
+    const int q = warp & 3;        // tensor-memory lane group of this warp
+    const int cs = e >> 2;         // 64-column slice
+    const int etid = threadIdx.x - 128;
+    uint8_t* alr = smem + S::ALR_OFF;
+    if constexpr (R > 0) {
+      if (static_cast<int>(blockIdx.x) < num_tiles) {
+        prep_lowrank_a<R>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid);
+        fence_proxy_async_smem();
+        mbar_arrive(bar_lr_full);
+      }
+    }
+    for (int tile = blockIdx.x, j = 0; tile < num_tiles; tile += gridDim.x, ++j) {
+      const int mb = tile % p.num_m, nb = tile / p.num_m;
+      if (!__all_sync(0xffffffffu, wait_bounded(bar_acc_full, j & 1, guard, 0x347, 128))) break;
+      tc_fence_after();
+      uint32_t v[64];
+      const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + cs * 64;
+      tmem_ld_x32(ta, v);
+      tmem_ld_x32(ta + 32, v + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acc_empty);
+      if constexpr (R > 0) {
+        const int next = tile + gridDim.x;
+        if (next < num_tiles) {
+          prep_lowrank_a<R>(alr, p.t, (next % p.num_m) * KG_BM, p.M, etid);
+          fence_proxy_async_smem();
+          mbar_arrive(bar_lr_full);
+        }
+      }
+      store_rows64_coalesced(p, mb * KG_BM + q * 32, nb * KG_BN + cs * 64,
+                             reinterpret_cast<const float*>(v), lane);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace svdq

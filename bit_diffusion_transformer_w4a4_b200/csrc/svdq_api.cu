@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -14,6 +15,7 @@
 
 #include "../../include/svdq.h"
 #include "kg_int4.cuh"
+#include "kg_int4h.cuh"
 #include "kg_nvfp4.cuh"
 #include "kg_nvfp4_pair.cuh"
 #include "kq.cuh"
@@ -33,6 +35,26 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// fp16 bits of v if v is exactly an fp16 value (finite, normal or subnormal).
+bool fp16_exact(float v, uint16_t* out) {
+  uint32_t b;
+  std::memcpy(&b, &v, 4);
+  const uint16_t sign = static_cast<uint16_t>((b >> 16) & 0x8000u);
+  const float a = std::fabs(v);
+  if (a == 0.0f) { *out = sign; return true; }
+  if (!(a <= 65504.0f)) return false;
+  if (a >= 6.103515625e-05f) {  // normal: 2^-14 .. 65504, 10 stored fraction bits
+    const uint32_t e = ((b >> 23) & 0xFFu) - 127u + 15u;
+    if (b & 0x1FFFu) return false;  // fraction bits below fp16's
+    *out = static_cast<uint16_t>(sign | (e << 10) | ((b >> 13) & 0x3FFu));
+    return true;
+  }
+  const float m = a * 16777216.0f;  // multiples of 2^-24
+  if (m != std::floor(m)) return false;
+  *out = static_cast<uint16_t>(sign | static_cast<uint16_t>(m));
+  return true;
+}
 
 svdq_status check_device(int* dev_out, int* sms_out) {
   int dev = 0, n = 0;
@@ -102,6 +124,7 @@ struct svdq_weights {
   uint16_t* l2dup = nullptr;   // [N x 2r]
   uint8_t* wcodes = nullptr;   // NVFP4 [N x K/2] packed; INT4 [N x K] int8
   uint8_t* wscales = nullptr;  // NVFP4 tiled E4M3; INT4 fp32 [K/64 x npad]
+  uint16_t* wh = nullptr;      // INT4 with SVDQ_INT4_F16: fp16 s_w q_w [N x K]
   uint16_t* bias = nullptr;
   // activation-kernel scratch: partial T tiles of split row blocks and their
   // arrival counters (zero between launches)
@@ -121,6 +144,8 @@ struct svdq_weights {
   // NVFP4 CTA-pair GEMM: 128-row boxes of codes and L2, scale atoms as rows
   // of 128 32-bit words
   CUtensorMap tm_b2, tm_blr2, tm_sfb2;
+  // INT4 fp16 GEMM: dequantised weights and L2, 128-byte rows, 256-row boxes
+  CUtensorMap tm_bh, tm_blrh;
   // per-call maps, cached by (pointer, M)
   CUtensorMap tm_x, tm_a, tm_a2, tm_sfa2;
   const void* tm_x_ptr = nullptr;
@@ -140,7 +165,7 @@ size_t act_scale_bytes(const svdq_weights* h, int64_t M) {
 }
 
 void free_all(svdq_weights* h) {
-  void* ptrs[] = {h->inv_lam, h->l1t, h->l2dup, h->wcodes, h->wscales, h->bias, h->ws_codes,
+  void* ptrs[] = {h->inv_lam, h->l1t, h->l2dup, h->wcodes, h->wscales, h->wh, h->bias, h->ws_codes,
                   h->ws_scales, h->ws_t, h->x_dev, h->y_dev, h->err, h->kq_tpart, h->kq_counters};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -201,9 +226,44 @@ svdq_status launch_kq_v(svdq_weights* h, const CUtensorMap& tmx, int64_t M, uint
   return SVDQ_ERR_SHAPE;
 }
 
+template <int R>
+svdq_status launch_kg_int4h_t(svdq_weights* h, const CUtensorMap& tma, int64_t M, const uint8_t* sfa,
+                              const float* t, void* y, cudaStream_t st) {
+  using S = KGI4HSmem<R>;
+  static bool attr = false;
+  if (!attr) {
+    svdq_status s = set_smem(kg_int4h_kernel<R>, S::TOTAL);
+    if (s != SVDQ_OK) return s;
+    attr = true;
+  }
+  KGParams p;
+  p.sfa = sfa;
+  p.sfb = h->wscales;
+  p.t = t;
+  p.bias = h->bias;
+  p.y = static_cast<uint16_t*>(y);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(h->N);
+  p.K = static_cast<int>(h->K);
+  p.num_m = static_cast<int>(cdiv(M, KG_BM));
+  p.num_n = static_cast<int>(cdiv(h->N, KG_BN));
+  p.gelu = (h->flags & SVDQ_EPI_GELU) ? 1 : 0;
+  p.err = h->err;
+  p.debug_mask = h->debug_mask;
+  p.timeout_ns = h->timeout_ns;
+  const int tiles = p.num_m * p.num_n;
+  const int grid = tiles < h->sms ? tiles : h->sms;
+  kg_int4h_kernel<R><<<grid, KG_THREADS, S::TOTAL, st>>>(tma, h->tm_bh, h->tm_blrh, p);
+  SVDQ_TRY(cudaGetLastError());
+  return SVDQ_OK;
+}
+
 template <int V, int R>
 svdq_status launch_kg_t(svdq_weights* h, const CUtensorMap& tma, int64_t M, const uint8_t* sfa,
                         const float* t, void* y, cudaStream_t st) {
+  if constexpr (V == 0) {
+    if (h->wh) return launch_kg_int4h_t<R>(h, tma, M, sfa, t, y, st);
+  }
   const int smem = V == 1 ? KGF4Smem<R>::TOTAL : KGI4Smem<R>::TOTAL;
   auto kern = V == 1 ? kg_nvfp4_kernel<R> : kg_int4_kernel<R>;
   static bool attr = false;
@@ -535,6 +595,7 @@ const char* svdq_status_string(svdq_status s) {
     case SVDQ_ERR_OOM: return "SVDQ_ERR_OOM";
     case SVDQ_ERR_CUDA: return "SVDQ_ERR_CUDA";
     case SVDQ_ERR_DEVICE_TIMEOUT: return "SVDQ_ERR_DEVICE_TIMEOUT";
+    case SVDQ_ERR_RANGE: return "SVDQ_ERR_RANGE";
   }
   return "SVDQ_ERR_UNKNOWN";
 }
@@ -545,7 +606,7 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
   if (!d || !out) return SVDQ_ERR_INVALID_ARG;
   *out = nullptr;
   if (d->variant != SVDQ_INT4_G64_BF16 && d->variant != SVDQ_NVFP4_G16_E4M3) return SVDQ_ERR_INVALID_ARG;
-  if (d->flags & ~(SVDQ_EPI_GELU | SVDQ_GEMM_SINGLE_SM)) return SVDQ_ERR_INVALID_ARG;
+  if (d->flags & ~(SVDQ_EPI_GELU | SVDQ_GEMM_SINGLE_SM | SVDQ_INT4_F16)) return SVDQ_ERR_INVALID_ARG;
   const int64_t K = d->K, N = d->N, r = d->r;
   if (K < 128 || K % 128 != 0 || K > (1 << 20)) return SVDQ_ERR_SHAPE;
   if (N < 16 || N % 16 != 0 || N > (1 << 20)) return SVDQ_ERR_SHAPE;
@@ -602,6 +663,7 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
       l2dup[n * h->lr_cols + r + j] = v;
     }
   std::vector<uint8_t> codes, scales;
+  std::vector<uint16_t> wh;
   if (d->variant == SVDQ_NVFP4_G16_E4M3) {
     codes.assign(d->w_codes, d->w_codes + static_cast<size_t>(N) * (K / 2));
     scales.assign(static_cast<size_t>(h->npad) * (K / 16), 0);
@@ -629,6 +691,15 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
         std::memcpy(&f, &bits, 4);
         sf[g * h->npad + n] = f;
       }
+    if (d->flags & SVDQ_INT4_F16) {
+      // s_w q_w as fp16, which must be exact (else SVDQ_ERR_RANGE)
+      wh.resize(static_cast<size_t>(N) * K);
+      for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+          const float v = sf[(k / 64) * h->npad + n] * static_cast<float>(static_cast<int8_t>(codes[n * K + k]));
+          if (!fp16_exact(v, &wh[n * K + k])) return fail(SVDQ_ERR_RANGE);
+        }
+    }
   }
 
   // ---- device allocations and copies
@@ -644,6 +715,7 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
                 !dmalloc(reinterpret_cast<void**>(&h->ws_t), static_cast<size_t>(h->max_M) * r * 4)))
     return fail(SVDQ_ERR_OOM);
   if (d->bias && !dmalloc(reinterpret_cast<void**>(&h->bias), N * 2)) return fail(SVDQ_ERR_OOM);
+  if (!wh.empty() && !dmalloc(reinterpret_cast<void**>(&h->wh), wh.size() * 2)) return fail(SVDQ_ERR_OOM);
   if (r > 0 && (!dmalloc(reinterpret_cast<void**>(&h->kq_tpart), static_cast<size_t>(sms) * 128 * r * 4) ||
                 !dmalloc(reinterpret_cast<void**>(&h->kq_counters), cdiv(h->max_M, 128) * 4)))
     return fail(SVDQ_ERR_OOM);
@@ -660,6 +732,8 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
                 cudaMemcpy(h->l2dup, l2dup.data(), l2dup.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess))
     return fail(SVDQ_ERR_CUDA);
   if (d->bias && cudaMemcpy(h->bias, d->bias, N * 2, cudaMemcpyHostToDevice) != cudaSuccess)
+    return fail(SVDQ_ERR_CUDA);
+  if (!wh.empty() && cudaMemcpy(h->wh, wh.data(), wh.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess)
     return fail(SVDQ_ERR_CUDA);
 
   // ---- weight-side tensor maps
@@ -687,6 +761,18 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
   } else {
     h->tm_blr = h->tm_b;  // never read when r == 0
     h->tm_l1t = h->tm_b;
+  }
+  if (h->wh) {
+    if ((s = make_tmap(&h->tm_bh, h->wh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, N, 64, 256,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return fail(s);
+    if (r > 0) {
+      if ((s = make_tmap(&h->tm_blrh, h->l2dup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->lr_cols, N, 64, 256,
+                         CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+        return fail(s);
+    } else {
+      h->tm_blrh = h->tm_bh;  // never read when r == 0
+    }
   }
   if (d->variant == SVDQ_NVFP4_G16_E4M3) {
     if ((s = make_tmap(&h->tm_b2, h->wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128,
@@ -791,7 +877,7 @@ svdq_status svdq_device_status(svdq_weights_t h, void* stream) {
     cudaMemset(h->err, 0, sizeof(int));
     // an aborted launch may leave split arrival counters mid-count
     if (h->kq_counters) cudaMemset(h->kq_counters, 0, cdiv(h->max_M, 128) * 4);
-    return SVDQ_ERR_DEVICE_TIMEOUT;
+    return e == 0x34f ? SVDQ_ERR_RANGE : SVDQ_ERR_DEVICE_TIMEOUT;
   }
   return SVDQ_OK;
 }

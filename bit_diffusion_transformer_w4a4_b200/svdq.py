@@ -18,11 +18,12 @@ INT4 = 0
 NVFP4 = 1
 EPI_GELU = 1
 GEMM_SINGLE_SM = 2
+INT4_F16 = 4
 
 STATUS = {
     0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_SHAPE", 3: "SVDQ_ERR_ALIGNMENT",
     4: "SVDQ_ERR_UNSUPPORTED_DEVICE", 5: "SVDQ_ERR_OOM", 6: "SVDQ_ERR_CUDA",
-    7: "SVDQ_ERR_DEVICE_TIMEOUT",
+    7: "SVDQ_ERR_DEVICE_TIMEOUT", 8: "SVDQ_ERR_RANGE",
 }
 
 EXPORTED = [
@@ -122,11 +123,13 @@ def selftest_division(variant: int) -> tuple[int, int]:
 class SVDQWeights:
     """A loaded layer: owns a library handle (``svdq_weights_t``)."""
 
-    def __init__(self, pw, max_M: int, stream=None, single_sm: bool = False):
+    def __init__(self, pw, max_M: int, stream=None, single_sm: bool = False,
+                 int4_f16: bool = False):
         """``pw`` has fields variant, K, N, r, lam, L1, L2, codes, scales, bias, gelu
         (host numpy arrays in the formats of ``svdq_weight_desc``).  ``single_sm``
         sets SVDQ_GEMM_SINGLE_SM (NVFP4 GEMM on single SMs; by default it runs on
-        pairs of SMs when M > 128)."""
+        pairs of SMs when M > 128).  ``int4_f16`` sets SVDQ_INT4_F16 (INT4 GEMM as
+        one fp16 GEMM of the exactly dequantised operands)."""
         self._keep = [np.ascontiguousarray(pw.lam, dtype=np.float32),
                       np.ascontiguousarray(pw.L1, dtype=np.uint16),
                       np.ascontiguousarray(pw.L2, dtype=np.uint16),
@@ -138,7 +141,8 @@ class SVDQWeights:
         self.max_M = int(max_M)
         self.gelu = bool(pw.gelu)
         d = WeightDesc(self.variant, self.K, self.N, self.r, self.max_M,
-                       (EPI_GELU if self.gelu else 0) | (GEMM_SINGLE_SM if single_sm else 0),
+                       (EPI_GELU if self.gelu else 0) | (GEMM_SINGLE_SM if single_sm else 0)
+                       | (INT4_F16 if int4_f16 else 0),
                        _ptr(lam), _ptr(L1) if self.r else 0, _ptr(L2) if self.r else 0,
                        _ptr(codes), _ptr(scales), _ptr(bias))
         h = ctypes.c_void_p(0)

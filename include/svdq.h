@@ -58,7 +58,9 @@ typedef enum {
   SVDQ_ERR_UNSUPPORTED_DEVICE = 4, /* no CUDA device, or not compute capability 10.x */
   SVDQ_ERR_OOM = 5,                /* device allocation failed */
   SVDQ_ERR_CUDA = 6,               /* any other CUDA runtime / driver error */
-  SVDQ_ERR_DEVICE_TIMEOUT = 7      /* a kernel's bounded wait expired */
+  SVDQ_ERR_DEVICE_TIMEOUT = 7,     /* a kernel's bounded wait expired */
+  SVDQ_ERR_RANGE = 8               /* a value outside the range the selected path
+                                      computes exactly (see SVDQ_INT4_F16) */
 } svdq_status;
 
 typedef enum {
@@ -75,6 +77,17 @@ typedef enum {
  * 4608 x 3072 x 12288: 108.5 vs 118.8 us).  Both compute the same y up to
  * fp32 summation order.  For comparison and tests. */
 #define SVDQ_GEMM_SINGLE_SM 2u
+/* INT4 only: run kernel 2 as one fp16 GEMM of the dequantised operands
+ * (s_x q_x) and (s_w q_w) on the 16-bit tensor cores (kind::f16) instead of
+ * per-group int8 MMAs with an fp32 rescale of every group.  Both operands are
+ * exact in fp16 -- a bf16 scale has 8 significant bits, |q| <= 8 at most 3 --
+ * while the scales stay in fp16's range, and every product is exact in the
+ * fp32 accumulator, so y equals the int8 path's up to fp32 summation order.
+ * svdq_weights_load returns SVDQ_ERR_RANGE if a dequantised weight is not an
+ * fp16 value; svdq_device_status returns SVDQ_ERR_RANGE after a call in
+ * which an activation scale exceeded 9357 (7 s > 65504).  Activation scales
+ * below 2^-17 lose low bits of s q (absolute error below 2^-25 s). */
+#define SVDQ_INT4_F16 4u
 
 typedef struct svdq_weights* svdq_weights_t;   /* opaque, library-owned */
 
@@ -107,8 +120,9 @@ typedef struct {
  * current device and size the forward workspace for max_M tokens.
  * The weight scales of the NVFP4 variant are re-tiled into the tensor-core
  * scale-factor layout; the INT4 residual codes are additionally kept as int8
- * for the int8 tensor-core path.  On error *out is left NULL and nothing is
- * allocated.
+ * for the int8 tensor-core path (with SVDQ_INT4_F16: as fp16 s_w q_w
+ * [N x K] instead, SVDQ_ERR_RANGE if a value is not exact in fp16).  On error
+ * *out is left NULL and nothing is allocated.
  */
 svdq_status svdq_weights_load(const svdq_weight_desc* desc, svdq_weights_t* out, void* stream);
 

@@ -45,16 +45,36 @@ def test_workload_full_size(name, li):
     h.close()
 
 
-@pytest.mark.parametrize("name", ["qkv_int4", "fc1_nvfp4"])
-def test_workload_with_svd_prep(name):
+@pytest.mark.parametrize("name,opts", [("qkv_int4", {}), ("qkv_int4", {"int4_f16": True}),
+                                       ("fc1_nvfp4", {})], ids=["qkv_int4", "qkv_int4-f16", "fc1_nvfp4"])
+def test_workload_with_svd_prep(name, opts):
     """Full-size layer whose weights come from the oracle's calibration, SVD
-    and residual quantisation (the method's own weight distribution)."""
+    and residual quantisation (the method's own weight distribution); the INT4
+    layer also through the fp16-operand GEMM."""
     layer = WL[name][0]
     x = W.activations(layer)
     pw = P.prepare(x, W.weight(layer), layer.r, layer.variant, gelu=layer.gelu)
-    h = svdq.SVDQWeights(pw, layer.M)
+    h = svdq.SVDQWeights(pw, layer.M, **opts)
     got = PT.gpu_forward(h, x, layer.M, two_calls=False)
     rows = _rows(layer.M, 64, seed=1)
     ref = O.linear_forward(x, pw, rows=rows)
     PT.check_y(got["Y"][rows], ref["y"], ref["Y"], label=f"{name} prepped")
+    h.close()
+
+
+INT4_CASES = [(n, i) for n, i in CASES if WL[n][i].variant == W.INT4]
+
+
+@pytest.mark.parametrize("name,li", INT4_CASES, ids=[f"{n}-{i}" for n, i in INT4_CASES])
+def test_workload_full_size_int4_f16(name, li):
+    """Every INT4 workload layer at full size through the fp16-operand GEMM
+    (SVDQ_INT4_F16), sampled rows against the oracle."""
+    layer = WL[name][li]
+    x = W.activations(layer)
+    pw = W.synthetic_packed(layer)
+    h = svdq.SVDQWeights(pw, layer.M, int4_f16=True)
+    got = PT.gpu_forward(h, x, layer.M)
+    rows = _rows(layer.M, seed=2)
+    ref = O.linear_forward(x, pw, rows=rows)
+    PT.check_y(got["Y"][rows], ref["y"], ref["Y"], label=f"{name}[{li}] f16")
     h.close()

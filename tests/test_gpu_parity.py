@@ -1,5 +1,7 @@
 """GPU parity: the CUDA path, called through the C ABI, against the CPU oracle
 on the same seeded inputs.  Needs an sm_100 GPU (marked gpu)."""
+import copy
+
 import numpy as np
 import pytest
 
@@ -40,15 +42,16 @@ def test_activation_kernel(variant, r, M, K):
     PT.check_act(got, {"codes": codes, "scales": scales, "T": T}, r=r, label=f"v{variant} r{r} M{M} K{K}")
 
 
-# NVFP4 kernel 2 runs on SM pairs for M > 128, or on single SMs when
-# SVDQ_GEMM_SINGLE_SM is set: the NVFP4 cases run both kernels.
-KERNELS = [(INT4, False), (NVFP4, False), (NVFP4, True)]
-KIDS = ["int4", "nvfp4-pair", "nvfp4-1sm"]
+# Every kernel-2 implementation: INT4 as per-group int8 MMAs (default) or as
+# one fp16 GEMM of the dequantised operands (SVDQ_INT4_F16); NVFP4 on SM pairs
+# for M > 128 (default) or on single SMs (SVDQ_GEMM_SINGLE_SM).
+KERNELS = [(INT4, {}), (INT4, {"int4_f16": True}), (NVFP4, {}), (NVFP4, {"single_sm": True})]
+KIDS = ["int4", "int4-f16", "nvfp4-pair", "nvfp4-1sm"]
 
 
-@pytest.mark.parametrize("variant,single", KERNELS, ids=KIDS)
+@pytest.mark.parametrize("variant,opts", KERNELS, ids=KIDS)
 @pytest.mark.parametrize("r", [0, 16, 32, 128])
-def test_gemm_isolated(variant, single, r):
+def test_gemm_isolated(variant, opts, r):
     """Kernel 2 alone, fed the oracle's activation codes / scales / T."""
     import torch
     M, K, N = 300, 512, 512
@@ -56,7 +59,7 @@ def test_gemm_isolated(variant, single, r):
     inv = (np.float32(1) / pw.lam).astype(np.float32)
     codes, scales, T = O.quantize_act_lowrank_down(x, inv, pw.L1, variant)
     y_ref, Y_ref = O.gemm_lowrank_up(codes, scales, T, pw.codes, pw.scales, pw.L2, variant)
-    h = svdq.SVDQWeights(pw, M, single_sm=single)
+    h = svdq.SVDQWeights(pw, M, **opts)
     sc = PT.tile_nvfp4_scales(scales, M, K) if variant == NVFP4 else scales.view(np.uint8).reshape(-1)
     tt = np.zeros((M, max(r, 1)), dtype=np.float32)
     tt[:, :r] = T
@@ -68,14 +71,14 @@ def test_gemm_isolated(variant, single, r):
     PT.check_y(Yg, y_ref, Y_ref, label=f"gemm v{variant} r{r}")
 
 
-@pytest.mark.parametrize("variant,single", KERNELS, ids=KIDS)
+@pytest.mark.parametrize("variant,opts", KERNELS, ids=KIDS)
 @pytest.mark.parametrize("gelu,with_bias", [(False, False), (True, True), (False, True)])
 @pytest.mark.parametrize("M,K,N,r", [(300, 512, 448, 32), (129, 1024, 272, 16), (513, 384, 768, 64),
                                      (640, 768, 528, 128)])
-def test_forward_small(variant, single, gelu, with_bias, M, K, N, r):
+def test_forward_small(variant, opts, gelu, with_bias, M, K, N, r):
     """Ragged M and N (partial tiles), several K tiles, bias and GELU."""
     lay, x, pw = _prepped(M, K, N, r, variant, gelu=gelu, with_bias=with_bias)
-    h = svdq.SVDQWeights(pw, M, single_sm=single)
+    h = svdq.SVDQWeights(pw, M, **opts)
     got = PT.gpu_forward(h, x, M)
     ref = O.linear_forward(x, pw)
     PT.check_act(got, ref, r=r, label="fwd")
@@ -122,16 +125,16 @@ def test_host_entry_point_matches_device(variant):
     assert np.array_equal(yh.numpy().view(np.uint16), dev["Y"])
 
 
-@pytest.mark.parametrize("variant,single", KERNELS, ids=KIDS)
+@pytest.mark.parametrize("variant,opts", KERNELS, ids=KIDS)
 @pytest.mark.parametrize("mask", [1, 2])
-def test_bounded_wait_reports_timeout(variant, single, mask):
+def test_bounded_wait_reports_timeout(variant, opts, mask):
     """A pipeline stage that is never filled: the kernel's bounded wait expires,
     the call reports SVDQ_ERR_DEVICE_TIMEOUT and the context stays usable."""
     M, K, N, r = 256, 1024, 512, 32
     lay = W.Layer("fault", M=M, K=K, N=N, r=r, variant=variant, config_id=62)
     pw = W.synthetic_packed(lay)
     x = W.activations(lay)
-    h = svdq.SVDQWeights(pw, M, single_sm=single)
+    h = svdq.SVDQWeights(pw, M, **opts)
     ok = PT.gpu_forward(h, x, M)
     h.debug_set_fault(mask, 20000)                 # 20 ms limit
     import torch
@@ -162,3 +165,46 @@ def test_pair_and_single_sm_agree(M):
     ya = W.bf16_bits_to_f32(a["Y"]).astype(np.float64)
     yb = W.bf16_bits_to_f32(b["Y"]).astype(np.float64)
     assert np.linalg.norm(ya - yb) <= 1e-3 * np.linalg.norm(yb)
+
+
+@pytest.mark.parametrize("M,K,N,r", [(300, 512, 448, 32), (1000, 1024, 768, 64)])
+def test_int4_f16_and_int8_agree(M, K, N, r):
+    """The two INT4 GEMMs compute the same sum of exact products: equal up to
+    fp32 summation order."""
+    lay = W.Layer("i4h", M=M, K=K, N=N, r=r, variant=INT4, gelu=True, bias=True, config_id=64)
+    pw = W.synthetic_packed(lay)
+    x = W.activations(lay)
+    a = PT.gpu_forward(svdq.SVDQWeights(pw, M), x, M)
+    b = PT.gpu_forward(svdq.SVDQWeights(pw, M, int4_f16=True), x, M)
+    assert np.array_equal(a["codes"], b["codes"])
+    ya = W.bf16_bits_to_f32(a["Y"]).astype(np.float64)
+    yb = W.bf16_bits_to_f32(b["Y"]).astype(np.float64)
+    assert np.linalg.norm(ya - yb) <= 1e-3 * np.linalg.norm(ya)
+
+
+def test_int4_f16_range_errors():
+    """Weights whose dequantised values are not fp16 values are refused at
+    load; an activation scale above the fp16 bound is reported after the call."""
+    import torch
+    M, K, N, r = 256, 512, 256, 16
+    lay = W.Layer("i4r", M=M, K=K, N=N, r=r, variant=INT4, config_id=65)
+    pw = W.synthetic_packed(lay)
+    big = copy.deepcopy(pw)
+    big.scales = big.scales.copy()
+    big.scales.reshape(-1)[5] = 0x4900          # bf16 2^19: 7 * 2^19 > 65504
+    with pytest.raises(svdq.SvdqError) as e:
+        svdq.SVDQWeights(big, M, int4_f16=True)
+    assert "SVDQ_ERR_RANGE" in str(e.value)
+    svdq.SVDQWeights(big, M).close()            # the int8 path takes any scale
+    h = svdq.SVDQWeights(pw, M, int4_f16=True)
+    x = W.bf16_bits_to_f32(W.activations(lay)).copy()
+    x[7, :64] = 1.0e7                            # smoothed scale ~1e7 / (7 lambda) > 9357
+    xd = PT.to_dev(W.to_bf16_bits(x).view(np.int16)).view(torch.bfloat16)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    h.linear_forward(xd, y, M)
+    torch.cuda.synchronize()
+    assert h.device_status() == 8                # SVDQ_ERR_RANGE
+    ok = PT.gpu_forward(h, W.activations(lay), M)
+    assert h.device_status() == 0
+    ref = O.linear_forward(W.activations(lay), pw)
+    PT.check_y(ok["Y"], ref["y"], ref["Y"], label="after range error")
