@@ -44,12 +44,12 @@ __device__ __forceinline__ float gelu_tanh(float x) {
 
 // Write [T_hi | T_lo] of rows m0..m0+127 into the A operand buffer of the
 // low-rank k-steps: 128 rows x (64 bf16 = 128 B) chunks, 128B swizzle.
-// Called by the 512 epilogue threads (etid = 0..511).
-template <int R>
+// Called by NT epilogue threads (etid = 0..NT-1).
+template <int R, int NT = KG_EPI_WARPS * 32>
 __device__ __forceinline__ void prep_lowrank_a(uint8_t* alr, const float* __restrict__ t, int m0,
                                                int M, int etid) {
   constexpr int SEG = R / 8;  // 8 values of T per item
-  for (int it = etid; it < 128 * SEG; it += KG_EPI_WARPS * 32) {
+  for (int it = etid; it < 128 * SEG; it += NT) {
     const int row = it / SEG;
     const int seg = it % SEG;
     const int gm = m0 + row;

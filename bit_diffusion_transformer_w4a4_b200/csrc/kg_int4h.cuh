@@ -18,15 +18,22 @@
 //
 // Weights arrive dequantised (fp16 [N x K], prepared at load, exactness
 // checked there); activations are dequantised per stage in shared memory.
-// Persistent CTAs, one per SM, tile 128 x 256, one 64-group per stage.
-// Warp roles (640 threads):
+// Both operands hold K in the same order, permuted inside every block of 8
+// as (0,4,1,5,2,6,3,7): the order in which four lop3 operations lay out the
+// eight nibbles of a 32-bit word as fp16 pairs.  A dot product does not
+// depend on the order of its terms.
+// Persistent CTAs, one per SM, tile 128 x 256, one 64-group per stage, two
+// 128 x 256 fp32 accumulators in tensor memory (all 512 columns: no scale
+// factors live there), so the MMAs of tile j+1 run while tile j drains.
+// Warp roles (576 threads):
 //   warp 0      TMA producer: packed activation codes (32B swizzle), fp16
 //               weight tile (128B swizzle)
 //   warp 1      MMA issuer (kind::f16, fp16 x fp16, four k-steps of 16 per
 //               stage; low-rank bf16 k-steps), tensor-memory owner
-//   warps 2-3   dequantise the activation codes: q (from the nibble) times
-//               s_x, written as fp16 in the MMA's 128B-swizzled layout
-//   warps 4-19  epilogue: drain the accumulator, next tile's low-rank
+//   warps 2-9   dequantise the activation codes: q (from the nibble) times
+//               s_x, written as fp16 in the MMA's 128B-swizzled layout; two
+//               warps per SM sub-partition, one half row per thread
+//   warps 10-17 epilogue: drain an accumulator, next tile's low-rank
 //               operand, bias + GELU + bf16 stores
 #pragma once
 
@@ -40,6 +47,14 @@ namespace svdq {
 // (7 * s <= 65504).  Larger scales are reported as a device error.
 constexpr float kInt4F16MaxScale = 9357.0f;
 
+constexpr int KGI4H_DQ_WARPS = 8;
+constexpr int KGI4H_EPI_WARPS = 8;
+constexpr int KGI4H_THREADS = (2 + KGI4H_DQ_WARPS + KGI4H_EPI_WARPS) * 32;
+
+// K order inside each block of 8 (both operands): position p holds element
+// kInt4F16Perm[p] of the block.
+constexpr int kInt4F16Perm[8] = {0, 4, 1, 5, 2, 6, 3, 7};
+
 template <int R>
 struct KGI4HSmem {
   static constexpr int STAGES = R >= 64 ? 3 : 4;
@@ -52,7 +67,7 @@ struct KGI4HSmem {
   static constexpr int LR_STAGES = (LR_STEPS + 3) / 4;        // a 128-byte B row holds 4 k-steps
   static constexpr int ALR_OFF = STAGES * STAGE;
   static constexpr int BAR_OFF = ALR_OFF + LR_CHUNKS * 16384;
-  static constexpr int TOTAL = BAR_OFF + 256 + 1024;
+  static constexpr int TOTAL = BAR_OFF + 256 + 1024;  // barriers, tensor-memory slot, alignment
   static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
   static_assert(TOTAL <= 232448, "shared memory per CTA");
 };
@@ -62,28 +77,39 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Eight INT4 codes (two's complement nibbles, element 0 low) times the scale
-// pair s2 -> four fp16x2 words.  q + 8 = q xor 8 for a 4-bit code; the fp16
-// with bits 0x6400 | u is 1024 + u, so subtracting 1032 gives q exactly.
+// Eight INT4 codes (two's complement nibbles, element 0 lowest) times the
+// scale pair s2, as four fp16x2 words holding the elements (0,4) (1,5) (2,6)
+// (3,7).  lop3 with table 0x6A computes mask ? (w ^ c) : c: it keeps the
+// masked nibbles, flips their sign bit (q + 8 = q xor 8 for a 4-bit code) and
+// fills the rest with the fp16 exponent of 1024, so a nibble in bits 0-3 of a
+// half reads 1024 + (q + 8) and one in bits 4-7 reads 1024 + 16 (q + 8).
+// Subtracting 1032, or scaling by 1/16 and subtracting 72, gives q exactly;
+// the product with s (8 significant bits) is exact while it stays in range.
 __device__ __forceinline__ void dequant8_f16(uint32_t w, uint32_t s2, uint32_t* out) {
-  const uint32_t u = w ^ 0x88888888u;
+  const uint32_t w8 = w >> 8;
+  uint32_t t[4];
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t[0]) : "r"(w), "r"(0x000F000Fu), "r"(0x64086408u));
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t[1]) : "r"(w), "r"(0x00F000F0u), "r"(0x64806480u));
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t[2]) : "r"(w8), "r"(0x000F000Fu), "r"(0x64086408u));
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t[3]) : "r"(w8), "r"(0x00F000F0u), "r"(0x64806480u));
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t b = (u >> (8 * j)) & 0xFFu;
-    const uint32_t h = ((b & 0x0Fu) | ((b & 0xF0u) << 12)) | 0x64006400u;
-    uint32_t q2, r;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q2) : "r"(h), "r"(0x64086408u));
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(q2), "r"(s2));
-    out[j] = r;
+  for (int j = 0; j < 4; j += 2) {
+    uint32_t q0, q1;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q0) : "r"(t[j]), "r"(0x64086408u));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q1) : "r"(t[j + 1]), "r"(0x2C002C00u), "r"(0xD480D480u));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[j]) : "r"(q0), "r"(s2));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[j + 1]) : "r"(q1), "r"(s2));
   }
 }
 
 template <int R>
-__global__ void __launch_bounds__(KG_THREADS, 1)
+__global__ void __launch_bounds__(KGI4H_THREADS, 1)
     kg_int4h_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_blr, KGParams p) {
   using S = KGI4HSmem<R>;
   constexpr int NST = S::STAGES;
+  constexpr int NDQ = KGI4H_DQ_WARPS * 32;
+  constexpr int NEPI = KGI4H_EPI_WARPS * 32;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -92,11 +118,11 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   const uint32_t bar_full = smem_u32(bars);
   const uint32_t bar_ready = smem_u32(bars + NST);       // dequantised A written
   const uint32_t bar_empty = smem_u32(bars + 2 * NST);
-  const uint32_t bar_acc_full = smem_u32(bars + 3 * NST);
-  const uint32_t bar_acc_empty = smem_u32(bars + 3 * NST + 1);
-  const uint32_t bar_lr_full = smem_u32(bars + 3 * NST + 2);
-  const uint32_t bar_drain = smem_u32(bars + 3 * NST + 3);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NST + 4);
+  const uint32_t bar_acc_full = smem_u32(bars + 3 * NST);       // two, one per accumulator
+  const uint32_t bar_acc_empty = smem_u32(bars + 3 * NST + 2);  // two
+  const uint32_t bar_lr_full = smem_u32(bars + 3 * NST + 4);
+  const uint32_t bar_drain = smem_u32(bars + 3 * NST + 5);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NST + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -108,18 +134,20 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_ready + 8 * s, 64);  // the 64 dequantising threads
+      mbar_init(bar_ready + 8 * s, NDQ);  // every dequantising thread
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_acc_full, 1);
-    mbar_init(bar_acc_empty, KG_EPI_WARPS);
-    mbar_init(bar_lr_full, KG_EPI_WARPS * 32);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_acc_full + 8 * b, 1);
+      mbar_init(bar_acc_empty + 8 * b, KGI4H_EPI_WARPS);
+    }
+    mbar_init(bar_lr_full, NEPI);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -178,7 +206,9 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       uint32_t ph = 0;
       bool ok = true;
       for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
-        if (j > 0 && !(ok = wait_bounded(bar_acc_empty, (j - 1) & 1, guard, 0x343))) break;
+        const int b = j & 1;
+        const uint32_t acc = tmem + b * KG_BN;
+        if (j >= 2 && !(ok = wait_bounded(bar_acc_empty + 8 * b, ((j >> 1) - 1) & 1, guard, 0x343))) break;
         tc_fence_after();
         for (int g = 0; g < ng; ++g) {
           if (!(ok = wait_bounded(bar_ready + 8 * s, ph, guard, 0x344))) break;
@@ -186,7 +216,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           const uint64_t so = kStage * s;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem, dA0 + so + 2 * kk, dB0 + so + 2 * kk, id_h, (g | kk) != 0);
+            mma_bf16(acc, dA0 + so + 2 * kk, dB0 + so + 2 * kk, id_h, (g | kk) != 0);
           tc_commit(bar_empty + 8 * s);
           if (++s == NST) { s = 0; ph ^= 1; }
         }
@@ -202,14 +232,14 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
             for (int k2 = 0; k2 < 4; ++k2) {
               const int kk = 4 * l + k2;  // k-step over [T_hi | T_lo]
               if (kk < S::LR_STEPS)
-                mma_bf16(tmem, dLRA0 + (kk / 4) * 1024 + (kk % 4) * 2, dB0 + so + 2 * k2, id_bf, 1);
+                mma_bf16(acc, dLRA0 + (kk / 4) * 1024 + (kk % 4) * 2, dB0 + so + 2 * k2, id_bf, 1);
             }
             tc_commit(bar_empty + 8 * s);
             if (++s == NST) { s = 0; ph ^= 1; }
           }
           if (!ok) break;
         }
-        tc_commit(bar_acc_full);
+        tc_commit(bar_acc_full + 8 * b);
       }
       // drain: every MMA issued so far has completed before tensor memory is freed
       tc_commit(bar_drain);
@@ -217,47 +247,40 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < p.timeout_ns) {
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < 2 + KGI4H_DQ_WARPS) {
     // ------------------------------------------------ dequantise activations
-    const int tt = threadIdx.x - 64;  // 0..63: rows tt and tt + 64
+    const int dt = threadIdx.x - 64;    // 0..255
+    const int row = dt & (KG_BM - 1);   // one row of the tile
+    const int half = dt >> 7;           // codes [32 half, 32 half + 32) of the group
     const __nv_bfloat16* sx_all = reinterpret_cast<const __nv_bfloat16*>(p.sfa);
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int mb = tile % p.num_m;
+      const int gm = (tile % p.num_m) * KG_BM + row;
+      const __nv_bfloat16* sxr = sx_all + static_cast<size_t>(gm < p.M ? gm : 0) * ng;
+      // this row's scale of the next group, loaded one group ahead (rows past M: 0)
+      float sx_next = gm < p.M ? __bfloat162float(sxr[0]) : 0.0f;
       for (int g = 0; g < ng; ++g) {
-        // this group's scales of the two rows (rows past M read as 0)
-        float sx[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int gm = mb * KG_BM + tt + 64 * h;
-          sx[h] = gm < p.M ? __bfloat162float(sx_all[static_cast<size_t>(gm) * ng + g]) : 0.0f;
-        }
+        const float sx = sx_next;
+        if (g + 1 < ng && gm < p.M) sx_next = __bfloat162float(sxr[g + 1]);
         if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x349))) break;
+        if (sx > kInt4F16MaxScale) atomicCAS(p.err, 0, 0x34f);  // fp16 would overflow
+        const __half2 s2h = __float2half2_rn(sx);
+        const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&s2h);
         const uint8_t* apk = smem + s * S::STAGE;
         uint8_t* ah = smem + s * S::STAGE + S::APK_BYTES;
+        const uint4 v = *reinterpret_cast<const uint4*>(apk + swz_off(row, half, 32));
+        uint32_t o[16];
+        dequant8_f16(v.x, s2, o);
+        dequant8_f16(v.y, s2, o + 4);
+        dequant8_f16(v.z, s2, o + 8);
+        dequant8_f16(v.w, s2, o + 12);
+        // 32 codes = 4 chunks of 8 fp16 (16 bytes) of the 128-byte row
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int row = tt + 64 * h;
-          if (sx[h] > kInt4F16MaxScale) atomicCAS(p.err, 0, 0x34f);  // fp16 would overflow
-          const __half2 s2h = __float2half2_rn(sx[h]);
-          const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&s2h);
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(apk + swz_off(row, c, 32));
-            uint32_t o[16];
-            dequant8_f16(v.x, s2, o);
-            dequant8_f16(v.y, s2, o + 4);
-            dequant8_f16(v.z, s2, o + 8);
-            dequant8_f16(v.w, s2, o + 12);
-            // 32 codes = 4 chunks of 8 fp16 (16 bytes) of the 128-byte row
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              *reinterpret_cast<uint4*>(ah + swz_off(row, 4 * c + q, 128)) =
-                  make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-          }
-        }
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(ah + swz_off(row, 4 * half + q, 128)) =
+              make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
         fence_proxy_async_smem();
         mbar_arrive(bar_ready + 8 * s);
         if (++s == NST) { s = 0; ph ^= 1; }
@@ -272,40 +295,48 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     }
   } else {
     // ----------------------------------------------------------------- epilogue
-    const int e = warp - 4;
-    const int q = warp & 3;        // tensor-memory lane group of this warp
-    const int cs = e >> 2;         // 64-column slice
-    const int etid = threadIdx.x - 128;
+    const int e = warp - 2 - KGI4H_DQ_WARPS;  // 0..7
+    const int q = warp & 3;                   // tensor-memory lane group of this warp
+    const int cs = e >> 2;                    // 128-column half of the tile
+    const int etid = e * 32 + lane;
     uint8_t* alr = smem + S::ALR_OFF;
     if constexpr (R > 0) {
       if (static_cast<int>(blockIdx.x) < num_tiles) {
-        prep_lowrank_a<R>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid);
+        prep_lowrank_a<R, NEPI>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid);
         fence_proxy_async_smem();
         mbar_arrive(bar_lr_full);
       }
     }
     for (int tile = blockIdx.x, j = 0; tile < num_tiles; tile += gridDim.x, ++j) {
       const int mb = tile % p.num_m, nb = tile / p.num_m;
-      if (!__all_sync(0xffffffffu, wait_bounded(bar_acc_full, j & 1, guard, 0x347, 128))) break;
+      const int b = j & 1;
+      if (!__all_sync(0xffffffffu, wait_bounded(bar_acc_full + 8 * b, (j >> 1) & 1, guard, 0x347, 128))) break;
       tc_fence_after();
-      uint32_t v[64];
-      const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + cs * 64;
-      tmem_ld_x32(ta, v);
-      tmem_ld_x32(ta + 32, v + 32);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_acc_empty);
       if constexpr (R > 0) {
+        // the accumulator is complete, so the low-rank MMAs have read the
+        // operand buffer: prepare the next tile's
         const int next = tile + gridDim.x;
         if (next < num_tiles) {
-          prep_lowrank_a<R>(alr, p.t, (next % p.num_m) * KG_BM, p.M, etid);
+          prep_lowrank_a<R, NEPI>(alr, p.t, (next % p.num_m) * KG_BM, p.M, etid);
           fence_proxy_async_smem();
           mbar_arrive(bar_lr_full);
         }
       }
-      store_rows64_coalesced(p, mb * KG_BM + q * 32, nb * KG_BN + cs * 64,
-                             reinterpret_cast<const float*>(v), lane);
+      const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * KG_BN + cs * 128;
+      uint32_t v[64];
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        tmem_ld_x32(ta + 64 * h, v);
+        tmem_ld_x32(ta + 64 * h + 32, v + 32);
+        tmem_ld_wait();
+        if (h == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_acc_empty + 8 * b);
+        }
+        store_rows64_coalesced(p, mb * KG_BM + q * 32, nb * KG_BN + cs * 128 + 64 * h,
+                               reinterpret_cast<const float*>(v), lane);
+      }
     }
   }
 
@@ -313,7 +344,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 

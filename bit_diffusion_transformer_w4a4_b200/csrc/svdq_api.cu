@@ -253,7 +253,7 @@ svdq_status launch_kg_int4h_t(svdq_weights* h, const CUtensorMap& tma, int64_t M
   p.timeout_ns = h->timeout_ns;
   const int tiles = p.num_m * p.num_n;
   const int grid = tiles < h->sms ? tiles : h->sms;
-  kg_int4h_kernel<R><<<grid, KG_THREADS, S::TOTAL, st>>>(tma, h->tm_bh, h->tm_blrh, p);
+  kg_int4h_kernel<R><<<grid, KGI4H_THREADS, S::TOTAL, st>>>(tma, h->tm_bh, h->tm_blrh, p);
   SVDQ_TRY(cudaGetLastError());
   return SVDQ_OK;
 }
@@ -692,11 +692,14 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
         sf[g * h->npad + n] = f;
       }
     if (d->flags & SVDQ_INT4_F16) {
-      // s_w q_w as fp16, which must be exact (else SVDQ_ERR_RANGE)
+      // s_w q_w as fp16, which must be exact (else SVDQ_ERR_RANGE), with K
+      // permuted inside each block of 8 in the order the kernel's activation
+      // dequantiser produces
       wh.resize(static_cast<size_t>(N) * K);
       for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k) {
-          const float v = sf[(k / 64) * h->npad + n] * static_cast<float>(static_cast<int8_t>(codes[n * K + k]));
+          const int64_t ks = (k & ~int64_t(7)) + kInt4F16Perm[k & 7];
+          const float v = sf[(ks / 64) * h->npad + n] * static_cast<float>(static_cast<int8_t>(codes[n * K + ks]));
           if (!fp16_exact(v, &wh[n * K + k])) return fail(SVDQ_ERR_RANGE);
         }
     }
