@@ -43,6 +43,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="fc1_nvfp4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--int4-f16", action="store_true",
+                    help="INT4 workloads: kernel 2 as one fp16 GEMM of the dequantised operands "
+                         "(SVDQ_INT4_F16) instead of int8 MMAs")
     return ap.parse_args()
 
 
@@ -216,7 +219,8 @@ def run_ours(args, layer):
     M, K, N, r = layer.M, layer.K, layer.N, layer.r
     pw = W.synthetic_packed(layer, seed=rank)
     x_bits = W.activations(layer, seed=rank)
-    h = svdq.SVDQWeights(pw, M)
+    f16 = bool(args.int4_f16) and layer.variant == W.INT4
+    h = svdq.SVDQWeights(pw, M, int4_f16=f16)
     x = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     codes, scales, t = h.alloc_act(M)
@@ -288,29 +292,35 @@ def run_ours(args, layer):
     pk, pk_src = peaks()
     # dominant kernel: the 4-bit GEMM.  NVFP4 runs on the FP4 tensor path (dense
     # peak = measured bf16 burst x 4, the 9 : 2.25 PF nominal ratio); INT4 on
-    # the int8 path (x 2, 4.5 : 2.25)
+    # the int8 path (x 2, 4.5 : 2.25), or with fp16 operands on the 16-bit
+    # path (the measured bf16 burst itself)
     nvfp4 = layer.variant == W.NVFP4
     kg_flops = 2.0 * M * K * N + 2.0 * M * N * r
     achieved = kg_flops / (ms_kg * 1e-3) / 1e12
-    ratio = 4.0 if nvfp4 else 2.0
+    ratio = 4.0 if nvfp4 else (1.0 if f16 else 2.0)
     peak = pk["bf16_tflops"] * ratio
+    if nvfp4:
+        peak_src = f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 4 (FP4:BF16 nominal 9:2.25)"
+    elif f16:
+        peak_src = f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s (fp16 = bf16 rate)"
+    else:
+        peak_src = f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 2 (INT8:BF16 nominal 4.5:2.25)"
+    traffic_key = args.workload + ("/int4_f16" if f16 else "")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "nvfp4" if nvfp4 else "int4", "data": "synthetic",
+        "dtype": "nvfp4" if nvfp4 else ("int4 (fp16 operands)" if f16 else "int4"), "data": "synthetic",
         "config": {"workload": f"{layer.name} M{M} K{K} N{N} r{r}{' GELU' if layer.gelu else ''} "
-                               f"{W.VARIANT_NAME[layer.variant]}",
+                               f"{W.VARIANT_NAME[layer.variant]}{' fp16-operand GEMM' if f16 else ''}",
                    "l2": "flushed before every step (256 MB write, outside the timed events)",
                    "parallelism": f"replicas x{world}", "tokens_per_step": M * world},
         "tokens_per_s": world * M / (ms_step * 1e-3),
         "frac_of_fp4_roofline": None,
         "kernels_ms": {"quantize_act_lowrank_down": ms_kq, "w4a4_gemm_lowrank_up": ms_kg},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic("w4a4_gemm_lowrank_up", args.workload),
-                     "peak_source": (f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 4 (FP4:BF16 nominal 9:2.25)"
-                                     if nvfp4 else
-                                     f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 2 (INT8:BF16 nominal 4.5:2.25)")},
+                     "frac": achieved / peak, "traffic": recorded_traffic("w4a4_gemm_lowrank_up", traffic_key),
+                     "peak_source": peak_src},
         "e2e": {"value": job_throughput(world, flops, ms_e2e), "unit": "TFLOPS",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": 2 * args.steps,

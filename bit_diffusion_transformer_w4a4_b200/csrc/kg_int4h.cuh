@@ -31,8 +31,8 @@
 //   warp 1      MMA issuer (kind::f16, fp16 x fp16, four k-steps of 16 per
 //               stage; low-rank bf16 k-steps), tensor-memory owner
 //   warps 2-9   dequantise the activation codes: q (from the nibble) times
-//               s_x, written as fp16 in the MMA's 128B-swizzled layout; two
-//               warps per SM sub-partition, one half row per thread
+//               s_x, written as fp16 in the MMA's 128B-swizzled layout; one
+//               group of two warps per ring slot, two rows per thread
 //   warps 10-17 epilogue: drain an accumulator, next tile's low-rank
 //               operand, bias + GELU + bf16 stores
 #pragma once
@@ -57,7 +57,7 @@ constexpr int kInt4F16Perm[8] = {0, 4, 1, 5, 2, 6, 3, 7};
 
 template <int R>
 struct KGI4HSmem {
-  static constexpr int STAGES = R >= 64 ? 3 : 4;
+  static constexpr int STAGES = R >= 64 ? 3 : 4;  // one dequantising group (2 warps) per slot
   static constexpr int APK_BYTES = KG_BM * 32;   // 128 rows x 32 B packed (64 codes)
   static constexpr int AH_BYTES = KG_BM * 128;   // 128 rows x 64 fp16
   static constexpr int B_BYTES = KG_BN * 128;    // 256 rows x 64 fp16
@@ -70,6 +70,7 @@ struct KGI4HSmem {
   static constexpr int TOTAL = BAR_OFF + 256 + 1024;  // barriers, tensor-memory slot, alignment
   static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
   static_assert(TOTAL <= 232448, "shared memory per CTA");
+  static_assert(2 * STAGES <= KGI4H_DQ_WARPS, "two dequantising warps per ring slot");
 };
 
 // kind::f16 with fp16 A and B, fp32 accumulate, K-major both.
@@ -108,7 +109,6 @@ __global__ void __launch_bounds__(KGI4H_THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_blr, KGParams p) {
   using S = KGI4HSmem<R>;
   constexpr int NST = S::STAGES;
-  constexpr int NDQ = KGI4H_DQ_WARPS * 32;
   constexpr int NEPI = KGI4H_EPI_WARPS * 32;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(KGI4H_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_ready + 8 * s, NDQ);  // every dequantising thread
+      mbar_init(bar_ready + 8 * s, 64);  // one group of dequantising threads
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -249,47 +249,70 @@ __global__ void __launch_bounds__(KGI4H_THREADS, 1)
     }
   } else if (warp < 2 + KGI4H_DQ_WARPS) {
     // ------------------------------------------------ dequantise activations
-    const int dt = threadIdx.x - 64;    // 0..255
-    const int row = dt & (KG_BM - 1);   // one row of the tile
-    const int half = dt >> 7;           // codes [32 half, 32 half + 32) of the group
+    // NST groups of two warps (one group per ring slot) take every NST-th
+    // stage use, two rows per thread, so each thread has NST MMA stages' time
+    // for its share and every slot is dequantised by one group.  A group's
+    // previous use of a slot is then always its own, so its parity wait on the
+    // slot is unambiguous.  With three slots, warps 8 and 9 stay idle.
+    const int grp = (warp - 2) >> 1;                 // takes the uses u with u % NST == grp
+    const int t = ((warp - 2) & 1) * 32 + lane;      // rows t and t + 64 of the tile
     const __nv_bfloat16* sx_all = reinterpret_cast<const __nv_bfloat16*>(p.sfa);
     int s = 0;
-    uint32_t ph = 0;
-    bool ok = true;
+    uint32_t ph = 0, u = 0;
+    bool ok = grp < NST;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int gm = (tile % p.num_m) * KG_BM + row;
-      const __nv_bfloat16* sxr = sx_all + static_cast<size_t>(gm < p.M ? gm : 0) * ng;
-      // this row's scale of the next group, loaded one group ahead (rows past M: 0)
-      float sx_next = gm < p.M ? __bfloat162float(sxr[0]) : 0.0f;
-      for (int g = 0; g < ng; ++g) {
-        const float sx = sx_next;
-        if (g + 1 < ng && gm < p.M) sx_next = __bfloat162float(sxr[g + 1]);
-        if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x349))) break;
-        if (sx > kInt4F16MaxScale) atomicCAS(p.err, 0, 0x34f);  // fp16 would overflow
-        const __half2 s2h = __float2half2_rn(sx);
-        const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&s2h);
-        const uint8_t* apk = smem + s * S::STAGE;
-        uint8_t* ah = smem + s * S::STAGE + S::APK_BYTES;
-        const uint4 v = *reinterpret_cast<const uint4*>(apk + swz_off(row, half, 32));
-        uint32_t o[16];
-        dequant8_f16(v.x, s2, o);
-        dequant8_f16(v.y, s2, o + 4);
-        dequant8_f16(v.z, s2, o + 8);
-        dequant8_f16(v.w, s2, o + 12);
-        // 32 codes = 4 chunks of 8 fp16 (16 bytes) of the 128-byte row
+      int gm[2];
+      const __nv_bfloat16* sxr[2];
+      float nx[2];
+      // this thread's first group in the tile; its rows' scales are loaded
+      // one use ahead (rows past M: 0)
+      const int g0 = (grp - static_cast<int>(u % NST) + NST) % NST;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(ah + swz_off(row, 4 * half + q, 128)) =
-              make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-        fence_proxy_async_smem();
-        mbar_arrive(bar_ready + 8 * s);
+      for (int h = 0; h < 2; ++h) {
+        gm[h] = (tile % p.num_m) * KG_BM + t + 64 * h;
+        sxr[h] = sx_all + static_cast<size_t>(gm[h] < p.M ? gm[h] : 0) * ng;
+        nx[h] = (gm[h] < p.M && g0 < ng) ? __bfloat162float(sxr[h][g0]) : 0.0f;
+      }
+      for (int g = 0; g < ng; ++g, ++u) {
+        if (static_cast<int>(u % NST) == grp) {
+          float sx[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            sx[h] = nx[h];
+            if (g + NST < ng && gm[h] < p.M) nx[h] = __bfloat162float(sxr[h][g + NST]);
+          }
+          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x349))) break;
+          const uint8_t* apk = smem + s * S::STAGE;
+          uint8_t* ah = smem + s * S::STAGE + S::APK_BYTES;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int row = t + 64 * h;
+            if (sx[h] > kInt4F16MaxScale) atomicCAS(p.err, 0, 0x34f);  // fp16 would overflow
+            const __half2 s2h = __float2half2_rn(sx[h]);
+            const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&s2h);
+            const uint4 v0 = *reinterpret_cast<const uint4*>(apk + swz_off(row, 0, 32));
+            const uint4 v1 = *reinterpret_cast<const uint4*>(apk + swz_off(row, 1, 32));
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            // 64 codes = 8 chunks of 8 fp16 (16 bytes) of the 128-byte row
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint32_t o[4];
+              dequant8_f16(w[c], s2, o);
+              *reinterpret_cast<uint4*>(ah + swz_off(row, c, 128)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(bar_ready + 8 * s);
+        }
         if (++s == NST) { s = 0; ph ^= 1; }
       }
       // low-rank stages carry only the B operand; still pass each one through
       // the ready barrier so its phase stays in step with the stage ring
-      for (int l = 0; l < S::LR_STAGES && ok; ++l) {
-        if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x34c))) break;
-        mbar_arrive(bar_ready + 8 * s);
+      for (int l = 0; l < S::LR_STAGES && ok; ++l, ++u) {
+        if (static_cast<int>(u % NST) == grp) {
+          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, 0x34c))) break;
+          mbar_arrive(bar_ready + 8 * s);
+        }
         if (++s == NST) { s = 0; ph ^= 1; }
       }
     }

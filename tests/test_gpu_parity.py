@@ -88,6 +88,20 @@ def test_forward_small(variant, opts, gelu, with_bias, M, K, N, r):
     assert np.array_equal(got2["Y"], got["Y"])
 
 
+@pytest.mark.parametrize("variant,opts", KERNELS, ids=KIDS)
+def test_several_tiles_per_cta(variant, opts):
+    """More tiles than CTAs (or SM pairs): every persistent CTA takes two or
+    three tiles, so stage-ring phases, both accumulators and the low-rank
+    operand carry across tiles.  Ragged M and N."""
+    M, K, N, r = 2000, 256, 4848, 32
+    lay, x, pw = _prepped(M, K, N, r, variant, gelu=True, with_bias=True, cid=66)
+    h = svdq.SVDQWeights(pw, M, **opts)
+    got = PT.gpu_forward(h, x, M)
+    rows = np.unique(np.concatenate([np.arange(0, M, 7), [M - 1]]))
+    ref = O.linear_forward(x, pw, rows=rows)
+    PT.check_y(got["Y"][rows], ref["y"], ref["Y"], label=f"multi-tile v{variant} {opts}")
+
+
 def test_quantizer_edge_values():
     """All-zero groups, tiny values whose sign survives rounding to zero, huge
     outliers that saturate E4M3 scales, and exact ties."""
