@@ -154,7 +154,7 @@ def run_reference(args, layer):
     pw = W.synthetic_packed(layer)
     x = W.activations(layer)
     nrows = 64
-    for _ in range(min(args.warmup, 1)):
+    for _ in range(min(args.warmup, 3)):
         cpu_baseline(layer, pw, x, nrows)
     times, t_start = [], time.perf_counter()
     for _ in range(args.steps):
@@ -166,7 +166,7 @@ def run_reference(args, layer):
     tflops = statistics.median(t["value"] for t in times)
     ms = flops / (tflops * 1e12) * 1e3
     line = {"metric": METRIC, "value": tflops, "unit": "TFLOPS", "n_gpus": args.gpus,
-            "steps": len(times), "warmup": min(args.warmup, 1), "ms_per_step": ms,
+            "steps": len(times), "warmup": min(args.warmup, 3), "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": f"{layer.name} M{layer.M} K{layer.K} N{layer.N} r{layer.r}"
