@@ -205,7 +205,8 @@ svdq_status svdq_linear_forward_host(svdq_weights_t h, const void* x_host, void*
  * Every call shares the one array: the counters are cleared on `stream`
  * before each launch, and calls that overlap on the GPU (two streams, two
  * threads) race on it and must be serialised by the caller.
- * The paper has no counterpart to this entry point.
+ * The method describes no counterpart to this entry point; it serves callers
+ * that must not allocate.
  */
 svdq_status svdq_quantize_act_lowrank_down_static(svdq_variant variant, int64_t K, int64_t r,
                                                   const float* inv_lambda, const uint16_t* l1t,

@@ -22,7 +22,7 @@ Sources (page title, section):
             W ~ int4 * scale; part "2. SVDQ-FP4" -- FP4 has a sign bit, a
             small exponent and the rest mantissa.
 
-Readings where the pages are silent (each listed in the design doc): alpha = 0.5
+Readings where the pages are silent: alpha = 0.5
 balanced migration; lambda calibrated on the runtime X; sqrt(Sigma) split of
 the SVD factors; groups along K for both operands; scale = amax/7 (INT4, bf16)
 and amax/6 (NVFP4, E4M3); round-half-to-even everywhere; X' rounded to bf16;

@@ -1,7 +1,7 @@
 """Helpers shared by the GPU parity tests: run the CUDA path through the C ABI
 and the CPU oracle on the same seeded inputs, and compare them.
 
-Bars (the layer's stated tolerances, see DESIGN.md "Parity"):
+Bars (the layer's stated tolerances):
   * activation codes and scales: bit-exact;
   * T = X' L1: ||dT||_F <= 4 sqrt(K) 2^-24 || |X'| |L1| ||_F, the fp32
     accumulation bound for a K-term dot product (t_bound); small-K cases
