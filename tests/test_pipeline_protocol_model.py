@@ -1,0 +1,216 @@
+"""Model check of the stage-ring protocol of the fp16-operand INT4 GEMM, on
+the CPU.  The kernel's roles are modelled as coroutines over mbarriers with
+the hardware's phase-parity semantics:
+  * a TMA producer that fills slot s for stage use u after the slot's
+    previous use is consumed (asynchronous completion, as a TMA load);
+  * dequantising groups that take the uses u with u % groups == g, wait on
+    the slot's full barrier and publish the dequantised operand;
+  * the MMA issuer that waits for each use's operand, "multiplies" it into one
+    of two accumulators (asynchronous completion, as tcgen05.commit), and
+    needs the low-rank operand for each tile;
+  * epilogue warps that drain an accumulator, hand it back and prepare the
+    next tile's low-rank operand.
+Random schedules check that no wait returns on the wrong phase (each consumer
+sees exactly the data of the use it waits for), that nothing deadlocks, and
+that every tile's accumulator holds exactly its own uses.  A planted
+mistake -- more dequantising groups than ring slots -- must be caught.
+"""
+import random
+
+import pytest
+
+
+class MBar:
+    """mbarrier: arrival count plus transaction bytes; completed phases counted."""
+
+    def __init__(self, count, errors):
+        self.count = count
+        self.pending = count
+        self.tx = 0
+        self.completed = 0
+        self.errors = errors
+
+    def _check(self):
+        if self.pending == 0 and self.tx == 0:
+            self.completed += 1
+            self.pending = self.count
+
+    def arrive(self, expect_tx=0):
+        self.tx += expect_tx
+        self.pending -= 1
+        if self.pending < 0:  # more arrivals than the phase expects: undefined on hardware
+            self.errors.append("barrier over-arrival")
+            self.pending = 0
+        self._check()
+
+    def complete_tx(self, n):
+        self.tx -= n
+        self._check()
+
+    def try_wait(self, parity):
+        # true once the phase with this parity has completed: the current
+        # (incomplete) phase has the other parity
+        return (self.completed & 1) != parity
+
+
+class Model:
+    def __init__(self, nst, groups, ng, lr_stages, tiles, rng):
+        self.nst, self.groups, self.ng, self.lr, self.tiles = nst, groups, ng, lr_stages, tiles
+        self.rng = rng
+        self.errors = []
+        e = self.errors
+        self.full = [MBar(1, e) for _ in range(nst)]
+        self.ready = [MBar(1, e) for _ in range(nst)]   # one arrival per group use
+        self.empty = [MBar(1, e) for _ in range(nst)]
+        self.acc_full = [MBar(1, e) for _ in range(2)]
+        self.acc_empty = [MBar(1, e) for _ in range(2)]
+        self.lr_full = MBar(1, e)
+        self.slot_codes = [None] * nst    # use id whose codes (or weight rows) are in the slot
+        self.slot_operand = [None] * nst  # use id whose dequantised operand is in the slot
+        self.acc = [[] for _ in range(2)]
+        self.lr_operand = None
+        self.tma_ops = []                 # pending TMA landings: complete in any order
+        self.mma_ops = []                 # pending MMA completions: in issue order
+
+    def uses(self):
+        """(tile, use id, is_low_rank) in ring order."""
+        u = 0
+        for j in range(self.tiles):
+            for _ in range(self.ng):
+                yield j, u, False
+                u += 1
+            for _ in range(self.lr):
+                yield j, u, True
+                u += 1
+
+    def producer(self):
+        for j, u, lr in self.uses():
+            s, ph = u % self.nst, (u // self.nst) & 1
+            yield ("wait", self.empty[s], ph ^ 1)
+
+            def land(s=s, u=u):
+                self.slot_codes[s] = u
+                self.full[s].complete_tx(1)
+            self.full[s].arrive(expect_tx=1)
+            self.tma_ops.append(land)
+
+    def dequant(self, g):
+        for j, u, lr in self.uses():
+            if u % self.groups != g:
+                continue
+            s, ph = u % self.nst, (u // self.nst) & 1
+            yield ("wait", self.full[s], ph)
+            if self.slot_codes[s] != u:
+                self.errors.append(f"group {g} read use {self.slot_codes[s]} for use {u}")
+            if not lr:
+                self.slot_operand[s] = u
+            self.ready[s].arrive()
+
+    def mma(self):
+        uses = list(self.uses())
+        for j in range(self.tiles):
+            b = j & 1
+            if j >= 2:
+                yield ("wait", self.acc_empty[b], ((j >> 1) - 1) & 1)
+            for jj, u, lr in uses:
+                if jj != j:
+                    continue
+                s, ph = u % self.nst, (u // self.nst) & 1
+                if lr and u == min(x[1] for x in uses if x[0] == j and x[2]):
+                    yield ("wait", self.lr_full, j & 1)
+                    if self.lr_operand != j:
+                        self.errors.append(f"tile {j} low-rank operand is tile {self.lr_operand}")
+                yield ("wait", self.ready[s], ph)
+                if not lr and self.slot_operand[s] != u:
+                    self.errors.append(f"MMA read operand of use {self.slot_operand[s]} for use {u}")
+                if self.slot_codes[s] != u:
+                    self.errors.append(f"MMA read weight rows of use {self.slot_codes[s]} for use {u}")
+
+                def done(s=s, u=u, b=b, lr=lr, j=j):
+                    # the tensor core reads its operands until the MMA completes
+                    if self.slot_codes[s] != u or (not lr and self.slot_operand[s] != u):
+                        self.errors.append(f"slot {s} overwritten before use {u} completed")
+                    if lr and self.lr_operand != j:
+                        self.errors.append(f"low-rank operand of tile {j} overwritten in flight")
+                    self.acc[b].append(u)
+                    self.empty[s].arrive()
+                self.mma_ops.append(done)
+
+            def tile_done(b=b):
+                self.acc_full[b].arrive()
+            self.mma_ops.append(tile_done)
+
+    def epilogue(self):
+        uses = list(self.uses())
+        if self.lr:
+            self.lr_operand = 0
+            self.lr_full.arrive()
+        for j in range(self.tiles):
+            b = j & 1
+            yield ("wait", self.acc_full[b], (j >> 1) & 1)
+            want = [u for jj, u, _ in uses if jj == j]
+            if sorted(self.acc[b]) != want:
+                self.errors.append(f"tile {j} accumulator holds {sorted(self.acc[b])}")
+            self.acc[b] = []
+            if self.lr and j + 1 < self.tiles:
+                self.lr_operand = j + 1
+                self.lr_full.arrive()
+            self.acc_empty[b].arrive()
+
+    def run(self):
+        agents = [self.producer(), self.mma(), self.epilogue()] + [self.dequant(g) for g in range(self.groups)]
+        blocked = {i: None for i in range(len(agents))}
+        live = set(range(len(agents)))
+        steps = 0
+        while live or self.tma_ops or self.mma_ops:
+            steps += 1
+            assert steps < 200000
+            runnable = [i for i in live if blocked[i] is None or blocked[i][0].try_wait(blocked[i][1])]
+            # asynchronous completions are scheduled like agents
+            choices = runnable + (["tma"] if self.tma_ops else []) + (["mma"] if self.mma_ops else [])
+            if not choices:
+                return "deadlock"
+            c = self.rng.choice(choices)
+            if c == "tma":
+                self.tma_ops.pop(self.rng.randrange(len(self.tma_ops)))()
+                continue
+            if c == "mma":
+                self.mma_ops.pop(0)()
+                continue
+            blocked[c] = None
+            try:
+                op = next(agents[c])
+                blocked[c] = (op[1], op[2])
+            except StopIteration:
+                live.discard(c)
+        return "ok"
+
+
+CONFIGS = [(nst, ng, lr, tiles) for nst in (3, 4) for ng in (1, 2, 5) for lr in (0, 1, 4) for tiles in (1, 3, 5)]
+
+
+@pytest.mark.parametrize("nst,ng,lr,tiles", CONFIGS)
+def test_one_group_per_slot_is_safe(nst, ng, lr, tiles):
+    """The kernel's rule: as many dequantising groups as ring slots."""
+    for seed in range(40):
+        m = Model(nst, nst, ng, lr, tiles, random.Random(seed))
+        assert m.run() == "ok"
+        assert not m.errors, m.errors[:3]
+
+
+@pytest.mark.parametrize("groups", [1, 2])
+def test_groups_dividing_the_ring_are_safe(groups):
+    for seed in range(60):
+        m = Model(4, groups, 3, 1, 3, random.Random(seed))
+        assert m.run() == "ok" and not m.errors, m.errors[:3]
+
+
+def test_more_groups_than_slots_is_caught():
+    """Planted mistake: four groups on a three-slot ring.  A group can start
+    its parity wait two phases early and read another use's data."""
+    bad = 0
+    for seed in range(400):
+        m = Model(3, 4, 5, 1, 3, random.Random(seed))
+        res = m.run()
+        bad += res != "ok" or bool(m.errors)
+    assert bad > 0
