@@ -214,3 +214,170 @@ def test_more_groups_than_slots_is_caught():
         res = m.run()
         bad += res != "ok" or bool(m.errors)
     assert bad > 0
+
+
+class PairModel:
+    """The SM-pair NVFP4 GEMM's protocol.  Two CTAs; the leader's full barrier
+    counts both CTAs' TMA bytes; two leader copy warps move each stage's scale
+    factors into tensor memory and commit to their ready barriers; the
+    leader's MMA warp waits for both, multiplies, and commits the stage's
+    empty barrier in both CTAs; one accumulator per SM, handed back by both
+    CTAs' epilogues on the leader's barrier, which also collects both CTAs'
+    low-rank operands.  ``copy_skips_lr`` plants a known mistake: copy warps
+    that do not pass the low-rank stages through their ready barriers."""
+
+    def __init__(self, nst, nks, lr_stages, tiles, rng, copy_skips_lr=False):
+        self.nst, self.nks, self.lr, self.tiles, self.rng = nst, nks, lr_stages, tiles, rng
+        self.copy_skips_lr = copy_skips_lr
+        self.errors = []
+        e = self.errors
+        self.full = [MBar(1, e) for _ in range(nst)]                       # leader's
+        self.empty = [[MBar(1, e) for _ in range(nst)] for _ in range(2)]  # per CTA
+        self.ready = {w: [MBar(1, e) for _ in range(nst)] for w in ("a", "b")}
+        self.acc_full = [MBar(1, e) for _ in range(2)]                     # per CTA
+        self.acc_empty = MBar(2, e)                                        # leader's: both epilogues
+        self.lr_full = MBar(2, e)                                          # leader's: both epilogues
+        self.slot = [[None] * nst for _ in range(2)]                       # per CTA: use id in the slot
+        self.sf = {w: [None] * nst for w in ("a", "b")}                    # tensor-memory scale slots
+        self.acc = [[], []]
+        self.lr_operand = [None, None]
+        self.tma_ops, self.tc_ops = [], {"a": [], "b": [], "mma": []}
+
+    def uses(self):
+        u = 0
+        for j in range(self.tiles):
+            for _ in range(self.nks):
+                yield j, u, False
+                u += 1
+            for _ in range(self.lr):
+                yield j, u, True
+                u += 1
+
+    def producer(self, rank):
+        for j, u, lr in self.uses():
+            s, ph = u % self.nst, (u // self.nst) & 1
+            yield ("wait", self.empty[rank][s], ph ^ 1)
+            if rank == 0:
+                self.full[s].arrive(expect_tx=2)
+
+            def land(s=s, u=u, rank=rank):
+                self.slot[rank][s] = u
+                self.full[s].complete_tx(1)
+            self.tma_ops.append(land)
+
+    def copier(self, w):
+        for j, u, lr in self.uses():
+            if lr and self.copy_skips_lr:
+                continue
+            s, ph = u % self.nst, (u // self.nst) & 1
+            yield ("wait", self.full[s], ph)
+            if self.slot[0][s] != u or self.slot[1][s] != u:
+                self.errors.append(f"copy warp {w} saw stage data {self.slot[0][s]}/{self.slot[1][s]} for use {u}")
+
+            def copied(s=s, u=u, w=w, lr=lr):
+                if not lr:
+                    self.sf[w][s] = u
+                self.ready[w][s].arrive()
+            self.tc_ops[w].append(copied)
+
+    def mma(self):
+        uses = list(self.uses())
+        for j in range(self.tiles):
+            if j > 0:
+                yield ("wait", self.acc_empty, (j - 1) & 1)
+            first_lr = True
+            for jj, u, lr in uses:
+                if jj != j:
+                    continue
+                s, ph = u % self.nst, (u // self.nst) & 1
+                if lr and first_lr:
+                    first_lr = False
+                    yield ("wait", self.lr_full, j & 1)
+                yield ("wait", self.ready["a"][s], ph)
+                yield ("wait", self.ready["b"][s], ph)
+
+                def done(s=s, u=u, lr=lr, j=j):
+                    if self.slot[0][s] != u or self.slot[1][s] != u:
+                        self.errors.append(f"MMA of use {u} read stage data {self.slot[0][s]}/{self.slot[1][s]}")
+                    if not lr and (self.sf["a"][s] != u or self.sf["b"][s] != u):
+                        self.errors.append(f"MMA of use {u} read scales {self.sf['a'][s]}/{self.sf['b'][s]}")
+                    if lr and self.lr_operand != [j, j]:
+                        self.errors.append(f"MMA of tile {j} read low-rank operands {self.lr_operand}")
+                    for r in (0, 1):
+                        self.acc[r].append(u)
+                        self.empty[r][s].arrive()
+                self.tc_ops["mma"].append(done)
+
+            def tile_done():
+                for r in (0, 1):
+                    self.acc_full[r].arrive()
+            self.tc_ops["mma"].append(tile_done)
+
+    def epilogue(self, rank):
+        uses = list(self.uses())
+        if self.lr:
+            self.lr_operand[rank] = 0
+            self.lr_full.arrive()
+        for j in range(self.tiles):
+            yield ("wait", self.acc_full[rank], j & 1)
+            want = [u for jj, u, _ in uses if jj == j]
+            if sorted(self.acc[rank]) != want:
+                self.errors.append(f"CTA {rank} tile {j} accumulator holds {sorted(self.acc[rank])}")
+            self.acc[rank] = []
+            self.acc_empty.arrive()
+            if self.lr and j + 1 < self.tiles:
+                self.lr_operand[rank] = j + 1
+                self.lr_full.arrive()
+
+    def run(self):
+        agents = ([self.producer(0), self.producer(1), self.copier("a"), self.copier("b"), self.mma(),
+                   self.epilogue(0), self.epilogue(1)])
+        blocked = {i: None for i in range(len(agents))}
+        live = set(range(len(agents)))
+        steps = 0
+        while live or self.tma_ops or any(self.tc_ops.values()):
+            steps += 1
+            if steps > 400000:
+                return "livelock"
+            runnable = [i for i in live if blocked[i] is None or blocked[i][0].try_wait(blocked[i][1])]
+            choices = (runnable + (["tma"] if self.tma_ops else [])
+                       + [k for k, q in self.tc_ops.items() if q])
+            if not choices:
+                return "deadlock"
+            c = self.rng.choice(choices)
+            if c == "tma":
+                self.tma_ops.pop(self.rng.randrange(len(self.tma_ops)))()
+                continue
+            if isinstance(c, str):
+                self.tc_ops[c].pop(0)()   # each warp's tensor-core operations complete in order
+                continue
+            blocked[c] = None
+            try:
+                op = next(agents[c])
+                blocked[c] = (op[1], op[2])
+            except StopIteration:
+                live.discard(c)
+        return "ok"
+
+
+PAIR_CONFIGS = [(nst, nks, lr, tiles) for nst in (4, 5) for nks in (1, 2, 5) for lr in (0, 1, 2)
+                for tiles in (1, 3, 5)]
+
+
+@pytest.mark.parametrize("nst,nks,lr,tiles", PAIR_CONFIGS)
+def test_pair_protocol_is_safe(nst, nks, lr, tiles):
+    for seed in range(30):
+        m = PairModel(nst, nks, lr, tiles, random.Random(seed))
+        assert m.run() == "ok"
+        assert not m.errors, m.errors[:3]
+
+
+def test_pair_copy_warps_skipping_low_rank_stages_is_caught():
+    """Planted mistake: copy warps whose ready barriers skip the low-rank
+    stages fall out of step with the ring once a tile has passed."""
+    bad = 0
+    for seed in range(100):
+        m = PairModel(4, 3, 1, 3, random.Random(seed), copy_skips_lr=True)
+        res = m.run()
+        bad += res != "ok" or bool(m.errors)
+    assert bad > 0
