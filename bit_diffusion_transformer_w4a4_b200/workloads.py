@@ -173,13 +173,15 @@ class PackedWeights:
     meta: dict = field(default_factory=dict)
 
 
-def synthetic_packed(layer: Layer, seed: int = 0) -> PackedWeights:
+def synthetic_packed(layer: Layer, seed: int = 0, int4_min: int = -7) -> PackedWeights:
     """Random pre-packed weights with realistic magnitudes, for timing runs.
 
     Codes are raw nibbles drawn from a discretised bell shape, scales are raw
     bf16 / E4M3 bit patterns drawn from a band of magnitudes, lambda is
     log-normal with the outlier channels larger.  No quantisation or SVD is
-    performed -- the bit patterns are sampled directly.
+    performed -- the bit patterns are sampled directly.  INT4 codes are drawn
+    in [int4_min, 7]; -8 is a valid code of the format that the amax/7 rule
+    never produces, so it only appears when int4_min = -8.
     """
     K, N, r, G = layer.K, layer.N, layer.r, layer.G
     g = _rng(seed, layer.config_id, 10 * layer.layer_id + 7)
@@ -188,7 +190,7 @@ def synthetic_packed(layer: Layer, seed: int = 0) -> PackedWeights:
     L1 = to_bf16_bits(g.standard_normal((K, r), dtype=np.float32) * np.float32(0.05))
     L2 = to_bf16_bits(g.standard_normal((r, N), dtype=np.float32) * np.float32(0.05))
     if layer.variant == INT4:
-        q = np.clip(np.rint(g.normal(0.0, 2.5, (N, K))), -7, 7).astype(np.int8)
+        q = np.clip(np.rint(g.normal(0.0, 2.5, (N, K))), int4_min, 7).astype(np.int8)
         nib = (q.astype(np.int16) & 0xF).astype(np.uint8)
         scales = to_bf16_bits(np.exp(g.normal(np.log(0.02), 0.3, (N, K // G))).astype(np.float32))
     else:

@@ -26,6 +26,14 @@ T_REL = 1e-5
 Y_REL = 1e-3
 Y_MAXABS_RMS = 2e-2
 
+# (label, quantity, measured, bar) of every bar checked in this process; the
+# terminal summary (tests/conftest.py) prints them with the margin left.
+MARGINS: list[tuple[str, str, float, float]] = []
+
+
+def record(label: str, what: str, value: float, bar: float) -> None:
+    MARGINS.append((label, what, float(value), float(bar)))
+
 
 def torch_mod():
     import torch
@@ -104,8 +112,10 @@ def check_act(got: dict, ref: dict, rows=None, r: int = 0, label: str = "", tb: 
         d = float(np.linalg.norm(got["T"][sel].astype(np.float64) - ref["T"]))
         if tb is None:
             e = rel_fro(got["T"][sel], ref["T"])
+            record(label, "T rel Frobenius", e, T_REL)
             assert e <= T_REL, f"{label}: T rel err {e:.3e}"
         else:
+            record(label, "||dT|| / fp32 bound", d / tb if tb > 0 else 0.0, 1.0)
             assert d <= tb, f"{label}: ||dT|| {d:.3e} > fp32 accumulation bound {tb:.3e}"
 
 
@@ -119,6 +129,8 @@ def check_y(Y_gpu_bits: np.ndarray, y_ref: np.ndarray, Y_ref_bits: np.ndarray, l
     # error beyond the bf16 output rounding itself (half a bf16 ulp of y)
     excess = np.maximum(np.abs(yg - y_ref) - bf16_half_ulp(y_ref), 0.0)
     mx = float(np.max(excess)) if yg.size else 0.0
+    record(label, "Y rel Frobenius", e, Y_REL)
+    record(label, "Y max excess / rms", mx / rms if rms > 0 else 0.0, Y_MAXABS_RMS)
     assert e <= Y_REL, f"{label}: Y rel Frobenius {e:.3e} > {Y_REL}"
     assert mx <= Y_MAXABS_RMS * rms, f"{label}: max|dY| beyond bf16 rounding {mx:.3e} > " \
         f"{Y_MAXABS_RMS} * rms {rms:.3e}"
@@ -133,3 +145,39 @@ def bf16_half_ulp(y: np.ndarray) -> np.ndarray:
 
 def oracle_rows(pw, x_bits: np.ndarray, rows: np.ndarray) -> dict:
     return O.linear_forward(x_bits, pw, rows=rows)
+
+
+def oracle_act_all(pw, x_bits: np.ndarray, chunk: int = 2048) -> dict:
+    """The oracle's activation side (codes, canonical scales, T) on every
+    token row, computed in row blocks to bound host memory."""
+    inv = (np.float32(1) / np.asarray(pw.lam, dtype=np.float32)).astype(np.float32)
+    parts = [O.quantize_act_lowrank_down(x_bits[i:i + chunk], inv, pw.L1, pw.variant)
+             for i in range(0, x_bits.shape[0], chunk)]
+    return {"codes": np.concatenate([p[0] for p in parts]),
+            "scales": np.concatenate([p[1] for p in parts]),
+            "T": np.concatenate([p[2] for p in parts])}
+
+
+def oracle_y_all(pw, act: dict, chunk: int = 2048):
+    """The oracle's weight side on every row (y fp64, Y bf16 bits), from the
+    oracle's own activation codes, scales and T, in row blocks."""
+    ys, Ys = [], []
+    for i in range(0, act["codes"].shape[0], chunk):
+        y, Y = O.gemm_lowrank_up(act["codes"][i:i + chunk], act["scales"][i:i + chunk],
+                                 act["T"][i:i + chunk], pw.codes, pw.scales, pw.L2, pw.variant,
+                                 pw.bias, pw.gelu)
+        ys.append(y)
+        Ys.append(Y)
+    return np.concatenate(ys), np.concatenate(Ys)
+
+
+def t_bound_all(pw, x_bits: np.ndarray, chunk: int = 2048) -> float:
+    """t_bound over every row, accumulated in row blocks."""
+    inv = (np.float32(1) / np.asarray(pw.lam, dtype=np.float32)).astype(np.float32)
+    L1 = np.abs(F.bf16_from_bits(pw.L1))
+    K = x_bits.shape[1]
+    acc = 0.0
+    for i in range(0, x_bits.shape[0], chunk):
+        xp = np.abs(O.smooth_activations(x_bits[i:i + chunk], inv).astype(np.float64))
+        acc += float(np.sum((xp @ L1) ** 2))
+    return 4.0 * np.sqrt(K) * 2.0 ** -24 * np.sqrt(acc)

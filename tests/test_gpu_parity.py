@@ -222,3 +222,22 @@ def test_int4_f16_range_errors():
     assert h.device_status() == 0
     ref = O.linear_forward(W.activations(lay), pw)
     PT.check_y(ok["Y"], ref["y"], ref["Y"], label="after range error")
+
+
+@pytest.mark.parametrize("opts", [{}, {"int4_f16": True}], ids=["int4", "int4-f16"])
+def test_int4_weight_code_minus8(opts):
+    """INT4 weight codes span the whole format, -8..7 (the amax/7 rule never
+    produces -8, but the format and the load call accept it): the int8 unpack
+    must sign-extend 0x8 to -8, and with fp16 operands -8 s must stay exact."""
+    M, K, N, r = 300, 512, 528, 32
+    lay = W.Layer("i4m8", M=M, K=K, N=N, r=r, variant=INT4, gelu=True, bias=True, config_id=67)
+    pw = W.synthetic_packed(lay, int4_min=-8)
+    nib = np.stack([pw.codes & 0xF, pw.codes >> 4], axis=-1)
+    assert (nib == 8).sum() >= 100                   # -8 occurs (about 0.14% of codes)
+    x = W.activations(lay)
+    h = svdq.SVDQWeights(pw, M, **opts)
+    got = PT.gpu_forward(h, x, M)
+    ref = O.linear_forward(x, pw)
+    PT.check_act(got, ref, r=r, label="int4 -8")
+    PT.check_y(got["Y"], ref["y"], ref["Y"], label=f"int4 -8 {opts}")
+    h.close()

@@ -175,8 +175,9 @@ def _e4m3(fr):  return _rne(fr, 4, -6, Fraction(448), True)
 def _e2m1(fr):  return _rne(fr, 2, 0, Fraction(6), True)
 
 
-def _brute_layer(x, inv_lam, L1, L2, wq, ws, variant, gelu):
-    """Pure-python exact restatement: lists of Fractions, explicit loops."""
+def _brute_layer(x, inv_lam, L1, L2, wq, ws, variant, gelu, bias=None):
+    """Pure-python exact restatement: lists of Fractions, explicit loops.
+    The bias (if any) is added to the accumulator before GELU."""
     G = O.GROUP[variant]
     M, K = len(x), len(x[0])
     N, r = len(wq), len(L2)
@@ -211,6 +212,8 @@ def _brute_layer(x, inv_lam, L1, L2, wq, ws, variant, gelu):
             for gi, g0 in enumerate(range(0, K, G)):
                 acc += sx[m][gi] * ws[n][gi] * sum(qx[m][k] * wq[n][k] for k in range(g0, g0 + G))
             acc += sum(T[m][j] * L2[j][n] for j in range(r))
+            if bias is not None:
+                acc += bias[n]
             a = float(acc)
             if gelu:
                 a = 0.5 * a * (1 + math.tanh(math.sqrt(2 / math.pi) * (a + 0.044715 * a ** 3)))
@@ -220,9 +223,10 @@ def _brute_layer(x, inv_lam, L1, L2, wq, ws, variant, gelu):
 
 
 @pytest.mark.parametrize("variant", [INT4, NVFP4])
-@pytest.mark.parametrize("gelu", [False, True])
-def test_brute_force_8x8(variant, gelu):
-    g = np.random.default_rng(10 + variant + 2 * gelu)
+@pytest.mark.parametrize("gelu,with_bias", [(False, False), (True, False), (False, True),
+                                            (True, True)])
+def test_brute_force_8x8(variant, gelu, with_bias):
+    g = np.random.default_rng(10 + variant + 2 * gelu + 4 * with_bias)
     G = O.GROUP[variant]
     M = N = 8
     K, r = G, 3
@@ -245,14 +249,17 @@ def test_brute_force_8x8(variant, gelu):
         ws = F.e4m3_encode(np.exp(g.normal(-3, 0.5, (N, K // G))))
         wsv = F.e4m3_decode(ws)
         wqv = F.e2m1_decode(wq_nib)
+    # a bias large enough to move GELU's operating point (bf16 values)
+    bias_bits = F.bf16_bits(g.standard_normal(N) * 2.0) if with_bias else None
     codes, scales, T = O.quantize_act_lowrank_down(x_bits, inv_lam, L1b, variant)
     y, Y = O.gemm_lowrank_up(codes, scales, T, F.pack_nibbles(wq_nib), ws, L2b, variant,
-                             gelu=gelu)
+                             bias_bits=bias_bits, gelu=gelu)
 
     fr = lambda a: [[Fraction(float(v)) for v in row] for row in a]
     qx, sx, Tb, yb = _brute_layer(
         fr(F.bf16_from_bits(x_bits)), [Fraction(float(v)) for v in inv_lam],
-        fr(F.bf16_from_bits(L1b)), fr(F.bf16_from_bits(L2b)), fr(wqv), fr(wsv), variant, gelu)
+        fr(F.bf16_from_bits(L1b)), fr(F.bf16_from_bits(L2b)), fr(wqv), fr(wsv), variant, gelu,
+        None if bias_bits is None else [Fraction(float(v)) for v in F.bf16_from_bits(bias_bits)])
 
     nib = F.unpack_nibbles(codes)
     dq = F.int4_decode(nib) if variant == INT4 else F.e2m1_decode(nib)
@@ -267,3 +274,104 @@ def test_brute_force_8x8(variant, gelu):
     if variant == NVFP4:
         # the all-zero row has scale 0 and +0 codes
         assert np.all(nib[1] == 0) and np.all(sv[1] == 0)
+
+
+# ------------------------------------------------------------ GELU (tanh form)
+def test_gelu_tanh_against_torch_and_identities():
+    """The oracle's GELU against an independent implementation (torch's
+    tanh-approximate GELU, fp64 on the CPU) over a dense grid and at large
+    magnitudes, and against what the formula fixes: GELU(0) = 0, the odd-part
+    identity GELU(x) - GELU(-x) = x (tanh is odd), GELU(x) -> x for large x
+    and -> -0 for very negative x."""
+    import torch
+    xs = np.concatenate([np.linspace(-12.0, 12.0, 48001),
+                         [-1e300, -1e150, -1e30, -1e6, -60.0, -30.0, 30.0, 60.0, 1e6, 1e30,
+                          1e150, 1e300]])
+    ref = torch.nn.functional.gelu(torch.from_numpy(xs), approximate="tanh").numpy()
+    got = O.gelu_tanh(xs)
+    fin = np.abs(xs) < 1e100
+    # 1 + tanh(u) cancels for negative x in both implementations: compare in
+    # absolute terms, a few fp64 ulps of max(1, |x|)
+    assert np.all(np.abs(got[fin] - ref[fin]) <= 4e-15 * np.maximum(1.0, np.abs(xs[fin])))
+    assert np.all(got[xs >= 30] == xs[xs >= 30])           # tanh(u) == 1 in fp64
+    assert np.all(got[xs <= -30] == 0.0)
+    g = np.linspace(-6.0, 6.0, 1201)
+    assert O.gelu_tanh(0.0) == 0.0
+    assert np.allclose(O.gelu_tanh(g) - O.gelu_tanh(-g), g, rtol=0, atol=1e-15)
+    # the slope at 0 is 1/2 (d/dx of 0.5 x (1 + tanh(c x + ...)) at 0)
+    h = 1e-7
+    assert abs((O.gelu_tanh(h) - O.gelu_tanh(-h)) / (2 * h) - 0.5) < 1e-8
+
+
+# ------------------------------------------------- smoothing factor edge rules
+def test_lambda_edge_rules():
+    """lambda = 1 where either calibration maximum is zero; lambda clamped to
+    [2^-20, 2^20]; otherwise max|X_k|^0.5 / max|W_k|^0.5 (alpha = 0.5)."""
+    x = np.ones((4, 6))
+    w = np.ones((6, 3))
+    x[:, 0] = 0.0                      # all-zero activation channel
+    w[1, :] = 0.0                      # all-zero weight row
+    x[:, 2] = 2.0 ** 50                # would give 2^25 / 2^-25 = 2^50: clamped
+    w[2, :] = 2.0 ** -50
+    x[:, 3] = 2.0 ** -50               # 2^-50: clamped at the bottom
+    w[3, :] = 2.0 ** 50
+    x[:, 4] = 16.0                     # plain case: sqrt(16) / sqrt(4) = 2
+    w[4, :] = -4.0
+    lam = P.calibrate_lambda(x, w)
+    assert lam.dtype == np.float32
+    assert lam[0] == 1.0 and lam[1] == 1.0
+    assert lam[2] == np.float32(2.0 ** 20) and lam[3] == np.float32(2.0 ** -20)
+    assert lam[4] == 2.0 and lam[5] == 1.0
+
+
+# ------------------------------------- the whole weight preparation at full rank
+@pytest.mark.parametrize("K,N,variant", [(128, 64, INT4), (64, 128, INT4), (48, 32, NVFP4),
+                                         (32, 80, NVFP4)])
+def test_prepare_full_rank_reconstructs_xw(K, N, variant):
+    """prepare() end to end with r = min(K, N) and K != N: calibration, row
+    smoothing, SVD, bf16 factors and the residual over the stored factors.
+    With the fp64 residual the exact-arithmetic layer reproduces X W to fp64
+    rounding (the residual then holds only the factor rounding), the residual
+    codes are grouped along K per output feature, and the quantised forward
+    stays within the bf16 rounding of X'."""
+    g = np.random.default_rng(11 + K + N)
+    M = 24
+    x = g.standard_normal((M, K))
+    x[:, 1] *= 20
+    w = F.bf16_round(g.standard_normal((K, N)) * 0.02)
+    w[1, :] *= 8
+    x_bits = F.bf16_bits(x)
+    r = min(K, N)
+    pw = P.prepare(x_bits, w, r=r, variant=variant)
+    xv = F.bf16_from_bits(x_bits)
+    L1 = F.bf16_from_bits(pw.L1)
+    L2 = F.bf16_from_bits(pw.L2)
+    assert L1.shape == (K, r) and L2.shape == (r, N)
+    # the factors are full rank, so the residual is only their bf16 rounding
+    assert np.linalg.norm(pw.R) <= 2.0 ** -7 * np.linalg.norm(pw.w_hat)
+    y = O.exact_forward(xv, pw.lam, L1, L2, pw.R)
+    ref = xv @ w
+    assert np.abs(y - ref).max() <= 1e-12 * np.abs(ref).max()
+    # residual codes: [N, K/2] bytes, groups of G along K for each output n
+    G = O.GROUP[variant]
+    assert pw.codes.shape == (N, K // 2) and pw.scales.shape == (N, K // G)
+    deq = O.dequantize(F.unpack_nibbles(pw.codes), pw.scales, variant)     # [N, K]
+    if variant == INT4:
+        s = np.repeat(F.bf16_from_bits(pw.scales), G, axis=1)
+        assert np.all(np.abs(pw.R.T - deq) <= s / 2 * (1 + 1e-12))
+    else:
+        # with no per-tensor scale the tiny residual's E4M3 group scales are
+        # mostly subnormal or zero: zero scales mean amax / 6 rounded to 0
+        # (amax <= 6 * 2^-10); elsewhere codes stay within +-6 s with R's sign,
+        # and normal scales bound the error by s (half the widest E2M1 gap)
+        s = np.repeat(F.e4m3_decode(pw.scales), G, axis=1)
+        Rt = pw.R.T
+        assert np.all(np.abs(Rt[s == 0]) <= 6 * 2.0 ** -10)
+        assert np.all(np.abs(deq) <= 6 * s)
+        assert np.all((deq == 0) | (np.sign(deq) == np.sign(Rt)))
+        nrm = s >= 2.0 ** -6
+        assert np.all(np.abs(Rt - deq)[nrm] <= s[nrm])
+    # quantised forward: the residual is tiny, the rest is X' in bf16 and T in fp32
+    out = O.linear_forward(x_bits, pw)
+    e = np.linalg.norm(out["y"] - ref) / np.linalg.norm(ref)
+    assert e < 1e-2, e

@@ -76,3 +76,29 @@ def test_static_scratch_refuses_oversize():
         W.NVFP4, 3072, 32, fake, fake, fake, 4096 * 128 + 1, fake, fake, fake, None, None) == 2
     assert L.svdq_quantize_act_lowrank_down_static(
         W.NVFP4, 3000, 32, fake, fake, fake, 128, fake, fake, fake, None, None) == 2
+
+
+def test_static_scratch_null_error_word():
+    """device_error may be NULL (timeouts are then not reported to anyone):
+    the outputs of a normal call are the same."""
+    import torch
+    M, K, r = 384, 512, 32
+    lay = W.Layer("noalloc0", M=M, K=K, N=256, r=r, variant=W.NVFP4, config_id=81)
+    pw = W.synthetic_packed(lay)
+    x = W.activations(lay)
+    h = svdq.SVDQWeights(pw, M)
+    ref = PT.gpu_forward(h, x, M)
+    L = svdq.lib()
+    inv_d = torch.from_numpy((np.float32(1) / pw.lam).astype(np.float32)).cuda()
+    l1t_d = torch.from_numpy(np.ascontiguousarray(pw.L1.T).view(np.int16)).cuda()
+    x_d = torch.from_numpy(x.view(np.int16)).cuda()
+    codes, scales, t = h.alloc_act(M)
+    st = torch.cuda.current_stream().cuda_stream
+    assert L.svdq_quantize_act_lowrank_down_static(
+        lay.variant, K, r, inv_d.data_ptr(), l1t_d.data_ptr(), x_d.data_ptr(), M, codes.data_ptr(),
+        scales.data_ptr(), t.data_ptr(), None, st) == 0
+    torch.cuda.synchronize()
+    assert np.array_equal(codes.cpu().numpy(), ref["codes"])
+    assert np.array_equal(svdq.untile_nvfp4_scales(scales.cpu().numpy(), M, K), ref["scales"])
+    assert PT.rel_fro(t.cpu().numpy()[:, :r], ref["T"]) <= PT.T_REL
+    h.close()
