@@ -7,9 +7,11 @@
 A step is one pass of the whole layer over one batch: the activation kernel
 (smooth + quantise + pack + down projection) and the 4-bit GEMM kernel (with
 the low-rank up projection, GELU and bf16 store), for the headline layer
-M=4608 tokens, K=3072, N=12288, r=32.  Inputs are seeded synthetic data
-already resident in HBM; L2 is flushed (a 256 MB write, outside the timed
-events) before every step.  Under torchrun each rank runs its own replica of
+M=4608 tokens, K=3072, N=12288, r=32 (``--workload`` picks another; the
+2048-px DiT block runs its four linears back to back, fc2 fed with fc1's
+output).  Inputs are seeded synthetic data already resident in HBM; L2 is
+flushed (a 256 MB write and a 256 MB read, outside the timed events) before
+every step.  Under torchrun each rank runs its own replica of
 the layer (the layer is token-parallel; no collective is on the data path),
 and the slowest rank's device time is reported.
 
@@ -127,55 +129,88 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_baseline(layer, pw, x_bits, nrows: int):
-    """The oracle, as it stands, on a row sample of the same workload."""
+def layer_bytes(layer) -> int:
+    """Algorithmic HBM bytes of one layer pass: X read; activation codes and
+    scales written and read back; the packed weight codes and scales, L1, L2
+    read; T written and read; Y written."""
+    from bit_diffusion_transformer_w4a4_b200 import workloads as W
+    M, K, N, r, G = layer.M, layer.K, layer.N, layer.r, layer.G
+    sb = 2 if layer.variant == W.INT4 else 1          # bf16 or E4M3 scale bytes
+    return (M * K * 2 + 2 * (M * K // 2) + 2 * (M * K // G) * sb + N * K // 2 + (N * K // G) * sb
+            + K * r * 2 + r * N * 2 + 2 * M * r * 4 + M * N * 2)
+
+
+def layer_desc(layer, f16: bool = False) -> str:
+    from bit_diffusion_transformer_w4a4_b200 import workloads as W
+    return (f"{layer.name} M{layer.M} K{layer.K} N{layer.N} r{layer.r}{' GELU' if layer.gelu else ''} "
+            f"{W.VARIANT_NAME[layer.variant]}{' fp16-operand GEMM' if f16 else ''}")
+
+
+def cpu_baseline(layer, pw, x_bits, nrows: int, one_core: bool = True):
+    """The oracle, as it stands, on a row sample of the same workload: on all
+    host threads its BLAS uses, and (``one_core``) again limited to one."""
     import numpy as np
     from oracle import forward as O
     rows = np.arange(nrows)
+    flops = 2.0 * nrows * layer.K * layer.N + 2.0 * nrows * layer.r * (layer.K + layer.N)
     t = time.perf_counter()
     O.linear_forward(x_bits, pw, rows=rows)
     dt = time.perf_counter() - t
-    flops = 2.0 * nrows * layer.K * layer.N + 2.0 * nrows * layer.r * (layer.K + layer.N)
+    out = {"value": flops / dt / 1e12, "unit": "TFLOPS", "kind": "oracle",
+           "sample": f"{nrows} of {layer.M} token rows of {layer.name} (numpy fp64), {dt:.2f} s"}
     try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        from threadpoolctl import threadpool_info, threadpool_limits
+        out["cores"] = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        if one_core:
+            n1 = max(8, nrows // 8)
+            with threadpool_limits(limits=1):
+                t = time.perf_counter()
+                O.linear_forward(x_bits, pw, rows=np.arange(n1))
+                d1 = time.perf_counter() - t
+            f1 = flops * n1 / nrows
+            out["value_1core"] = f1 / d1 / 1e12
+            out["sample_1core"] = f"{n1} rows on 1 thread, {d1:.2f} s"
     except Exception:
-        cores = os.cpu_count()
-    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-            "sample": f"{nrows} of {layer.M} token rows of {layer.name} (numpy fp64), "
-                      f"{dt:.2f} s"}
+        out["cores"] = os.cpu_count()
+    return out
 
 
-def run_reference(args, layer):
+def run_reference(args, layers):
     from bit_diffusion_transformer_w4a4_b200 import workloads as W
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    layer = layers[0]
     pw = W.synthetic_packed(layer)
     x = W.activations(layer)
     nrows = 64
     for _ in range(min(args.warmup, 3)):
-        cpu_baseline(layer, pw, x, nrows)
+        cpu_baseline(layer, pw, x, nrows, one_core=False)
     times, t_start = [], time.perf_counter()
     for _ in range(args.steps):
-        r = cpu_baseline(layer, pw, x, nrows)
+        r = cpu_baseline(layer, pw, x, nrows, one_core=False)
         times.append(r)
         if time.perf_counter() - t_start > 120.0:
             break
     flops = 2.0 * nrows * layer.K * layer.N + 2.0 * nrows * layer.r * (layer.K + layer.N)
     tflops = statistics.median(t["value"] for t in times)
     ms = flops / (tflops * 1e12) * 1e3
-    line = {"metric": METRIC, "value": tflops, "unit": "TFLOPS", "n_gpus": args.gpus,
-            "steps": len(times), "warmup": min(args.warmup, 3), "ms_per_step": ms,
+    line = {"metric": metric_name(args.workload, layers), "value": tflops, "unit": "TFLOPS",
+            "n_gpus": args.gpus, "steps": len(times), "warmup": min(args.warmup, 3), "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": f"{layer.name} M{layer.M} K{layer.K} N{layer.N} r{layer.r}"
-                                   f"{' GELU' if layer.gelu else ''} {W.VARIANT_NAME[layer.variant]}",
-                       "step_sample_rows": nrows},
+            "config": {"workload": layer_desc(layer), "step_sample_rows": nrows},
             "cpu_baseline": {k: times[-1][k] for k in ("unit", "cores", "kind", "sample")}
             | {"value": tflops},
             "e2e": {"value": tflops, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def metric_name(workload: str, layers) -> str:
+    if workload == "fc1_nvfp4":
+        return METRIC
+    flops = sum(l.flops() for l in layers)
+    return f"W4A4+low-rank linear effective TFLOPS, {workload} ({len(layers)} layer(s), {flops / 1e9:.0f} GFLOP per step)"
 
 
 def max_over_ranks(values, device):
@@ -196,7 +231,7 @@ def job_throughput(world: int, flops_per_rank: float, ms_step: float) -> float:
     return world * flops_per_rank / (ms_step * 1e-3) / 1e12
 
 
-def run_ours(args, layer):
+def run_ours(args, layers):
     import numpy as np
     import torch
     import torch.distributed as dist
@@ -216,85 +251,131 @@ def run_ours(args, layer):
         if world > 1:
             dist.barrier()
 
-    M, K, N, r = layer.M, layer.K, layer.N, layer.r
-    pw = W.synthetic_packed(layer, seed=rank)
-    x_bits = W.activations(layer, seed=rank)
-    f16 = bool(args.int4_f16) and layer.variant == W.INT4
-    h = svdq.SVDQWeights(pw, M, int4_f16=f16)
-    x = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
-    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    codes, scales, t = h.alloc_act(M)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    # one handle and one set of buffers per layer; in the DiT block fc2 reads
+    # fc1's output (the MLP pair chained), the other layers their own inputs
+    names = [l.name for l in layers]
+    L = []
+    for i, layer in enumerate(layers):
+        f16 = bool(args.int4_f16) and layer.variant == W.INT4
+        pw = W.synthetic_packed(layer, seed=rank)
+        x_bits = W.activations(layer, seed=rank)
+        h = svdq.SVDQWeights(pw, layer.M, int4_f16=f16)
+        chained = layer.name.endswith("fc2") and any(n.endswith("fc1") for n in names[:i])
+        if chained:
+            x = L[names.index(names[i - 1])]["y"]
+        else:
+            x = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+        y = torch.empty((layer.M, layer.N), dtype=torch.bfloat16, device="cuda")
+        codes, scales, t = h.alloc_act(layer.M)
+        L.append(dict(layer=layer, pw=pw, x_bits=x_bits, h=h, x=x, y=y, codes=codes, scales=scales,
+                      t=t, f16=f16, chained=chained))
+    # L2 flush before every step, outside the timed events: a 256 MB write,
+    # then a 256 MB read of another buffer, so that L2 holds neither the inputs
+    # nor dirty lines whose write-back would land inside the next step
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
-        flush.zero_()                      # L2 flush, outside the timed events
-        if ev is not None:
-            ev[0].record(stream)
-        h.quantize_act_lowrank_down(x, M, codes, scales, t)
-        if ev is not None:
-            ev[1].record(stream)
-        h.w4a4_gemm_lowrank_up(codes, scales, t, M, y)
-        if ev is not None:
-            ev[2].record(stream)
+    def flush():
+        flush_w.zero_()
+        flush_r.sum()
+
+    def run_layers(evs=None):
+        for i, d in enumerate(L):
+            d["h"].quantize_act_lowrank_down(d["x"], d["layer"].M, d["codes"], d["scales"], d["t"])
+            if evs is not None:
+                evs[2 * i + 1].record(stream)
+            d["h"].w4a4_gemm_lowrank_up(d["codes"], d["scales"], d["t"], d["layer"].M, d["y"])
+            if evs is not None:
+                evs[2 * i + 2].record(stream)
 
     for _ in range(args.warmup):
-        step()
+        flush()
+        run_layers()
     torch.cuda.synchronize()
-    st = h.device_status()
-    if st != 0:
-        raise RuntimeError(f"device status {svdq.STATUS.get(st)} after warm-up")
+    for d in L:
+        st = d["h"].device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {svdq.STATUS.get(st)} after warm-up")
 
+    # timed pass 1: whole steps, events only at step boundaries (consecutive
+    # kernels overlap through programmatic dependent launch)
     clocks = ClockSampler(local)
     clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    ev_step = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     clocks.mark(True)
     for i in range(args.steps):
-        step(evs[i])
+        flush()
+        ev_step[i][0].record(stream)
+        run_layers()
+        ev_step[i][1].record(stream)
     torch.cuda.synchronize()
     barrier()
     clocks.mark(False)
+    # timed pass 2: the same steps with an event after every kernel, for the
+    # per-kernel durations (the events keep consecutive kernels apart)
+    nk = 2 * len(L)
+    ev_k = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush()
+        ev_k[i][0].record(stream)
+        run_layers(ev_k[i])
+    torch.cuda.synchronize()
+    barrier()
     clk = clocks.stop()
-    st = h.device_status()
-    if st != 0:
-        raise RuntimeError(f"device status {svdq.STATUS.get(st)} in the timed region")
-    t_kq = [e[0].elapsed_time(e[1]) for e in evs]
-    t_kg = [e[1].elapsed_time(e[2]) for e in evs]
-    ms_step = statistics.mean(a + b for a, b in zip(t_kq, t_kg))
-    ms_kg = statistics.mean(t_kg)
-    ms_kq = statistics.mean(t_kq)
-    ms_step, ms_kg, ms_kq = max_over_ranks([ms_step, ms_kg, ms_kq], "cuda")
+    for d in L:
+        st = d["h"].device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {svdq.STATUS.get(st)} in the timed region")
+    ms_step = statistics.mean(e[0].elapsed_time(e[1]) for e in ev_step)
+    per_k = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev_k) for j in range(nk)]
+    ms_sum = sum(per_k)
+    vals = max_over_ranks([ms_step, ms_sum] + per_k, "cuda")
+    ms_step, ms_sum, per_k = vals[0], vals[1], vals[2:]
 
-    flops = layer.flops()
+    flops = sum(d["layer"].flops() for d in L)
     value = job_throughput(world, flops, ms_step)
 
-    # end to end through the host entry point (pinned buffers, copies timed)
-    xh = torch.from_numpy(x_bits.view(np.int16)).pin_memory()
-    yh = torch.empty((M, N), dtype=torch.int16).pin_memory()
+    # end to end through the host entry point (pinned buffers, copies timed):
+    # every layer takes its input from host memory and returns its output there
     e2e_steps = max(3, min(args.steps, 20))
+    hx = [torch.from_numpy(d["x_bits"].view(np.int16)).pin_memory() for d in L]
+    hy = [torch.empty((d["layer"].M, d["layer"].N), dtype=torch.int16).pin_memory() for d in L]
+
+    def host_step():
+        for d, xh, yh in zip(L, hx, hy):
+            d["h"].linear_forward_host(xh, yh, d["layer"].M)
+
     for _ in range(2):
-        h.linear_forward_host(xh, yh, M)
+        host_step()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     e0.record(stream)
     for _ in range(e2e_steps):
-        h.linear_forward_host(xh, yh, M)
+        host_step()
     e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / e2e_steps
     (ms_e2e,) = max_over_ranks([ms_e2e], "cuda")
-    if h.device_status() != 0:
-        raise RuntimeError("device status error in the end-to-end loop")
+    for d in L:
+        if d["h"].device_status() != 0:
+            raise RuntimeError("device status error in the end-to-end loop")
 
     pk, pk_src = peaks()
-    # dominant kernel: the 4-bit GEMM.  NVFP4 runs on the FP4 tensor path (dense
-    # peak = measured bf16 burst x 4, the 9 : 2.25 PF nominal ratio); INT4 on
-    # the int8 path (x 2, 4.5 : 2.25), or with fp16 operands on the 16-bit
-    # path (the measured bf16 burst itself)
-    nvfp4 = layer.variant == W.NVFP4
+    # dominant kernel: the 4-bit GEMM of the layer with the most work.  NVFP4
+    # runs on the FP4 tensor path (dense peak = measured bf16 burst x 4, the
+    # 9 : 2.25 PF nominal ratio); INT4 on the int8 path (x 2), or with fp16
+    # operands on the 16-bit path (the measured bf16 burst itself)
+    di = max(range(len(L)), key=lambda i: L[i]["layer"].flops())
+    dl, f16 = L[di]["layer"], L[di]["f16"]
+    M, K, N, r = dl.M, dl.K, dl.N, dl.r
+    nvfp4 = dl.variant == W.NVFP4
+    ms_kg = per_k[2 * di + 1]
     kg_flops = 2.0 * M * K * N + 2.0 * M * N * r
     achieved = kg_flops / (ms_kg * 1e-3) / 1e12
     ratio = 4.0 if nvfp4 else (1.0 if f16 else 2.0)
@@ -305,37 +386,58 @@ def run_ours(args, layer):
         peak_src = f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s (fp16 = bf16 rate)"
     else:
         peak_src = f"{pk_src} bf16 burst {pk['bf16_tflops']} TFLOP/s x 2 (INT8:BF16 nominal 4.5:2.25)"
+    # the nominal dense 4-bit / 8-bit tensor rate at the sampled SM clock
+    # (2 x 128 x 256 x 64 per SM per 128 cycles for FP4; half that for INT8)
+    sm_mhz = clk.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
+    nominal = 148 * 2 * 128 * 256 * 64 / 128 * sm_mhz * 1e6 / 1e12 / (1.0 if nvfp4 else 2.0)
     traffic_key = args.workload + ("/int4_f16" if f16 else "")
+    wl = " + ".join(layer_desc(d["layer"], d["f16"]) for d in L)
+    kernels = {}
+    for i, d in enumerate(L):
+        pre = d["layer"].name + "." if len(L) > 1 else ""
+        kernels[pre + "quantize_act_lowrank_down"] = per_k[2 * i]
+        kernels[pre + "w4a4_gemm_lowrank_up"] = per_k[2 * i + 1]
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "metric": metric_name(args.workload, [d["layer"] for d in L]), "value": value, "unit": "TFLOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "nvfp4" if nvfp4 else ("int4 (fp16 operands)" if f16 else "int4"), "data": "synthetic",
-        "config": {"workload": f"{layer.name} M{M} K{K} N{N} r{r}{' GELU' if layer.gelu else ''} "
-                               f"{W.VARIANT_NAME[layer.variant]}{' fp16-operand GEMM' if f16 else ''}",
-                   "l2": "flushed before every step (256 MB write, outside the timed events)",
-                   "parallelism": f"replicas x{world}", "tokens_per_step": M * world},
-        "tokens_per_s": world * M / (ms_step * 1e-3),
+        "config": {"workload": wl,
+                   "l2": "flushed before every step (256 MB write, then 256 MB read; outside the timed events)",
+                   "parallelism": f"replicas x{world}", "tokens_per_step": L[0]["layer"].M * world,
+                   "chained": [d["layer"].name for d in L if d["chained"]],
+                   "timing": "ms_per_step: events at step boundaries only (kernels overlap through "
+                             "programmatic dependent launch); kernels_ms: a second timed pass with an "
+                             "event after every kernel"},
+        "tokens_per_s": world * L[0]["layer"].M / (ms_step * 1e-3),
         "frac_of_fp4_roofline": None,
-        "kernels_ms": {"quantize_act_lowrank_down": ms_kq, "w4a4_gemm_lowrank_up": ms_kg},
+        "kernels_ms": kernels,
+        "kernels_sum_ms": ms_sum,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic("w4a4_gemm_lowrank_up", traffic_key),
-                     "peak_source": peak_src},
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic("w4a4_gemm_lowrank_up", traffic_key),
+                     "peak_source": peak_src, "kernel": f"w4a4_gemm_lowrank_up ({dl.name})",
+                     "nominal_peak": nominal, "frac_of_nominal": achieved / nominal,
+                     "nominal_source": f"{'FP4' if nvfp4 else 'INT8'} dense tcgen05 rate at {sm_mhz:.0f} MHz "
+                                       "(128x256x64 per SM per 128 cycles)"},
         "e2e": {"value": job_throughput(world, flops, ms_e2e), "unit": "TFLOPS",
-                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
-        "gpu_launches": 2 * args.steps,
+                "h2d_bytes_per_step": sum(d["layer"].M * d["layer"].K * 2 for d in L),
+                "d2h_bytes_per_step": sum(d["layer"].M * d["layer"].N * 2 for d in L)},
+        "gpu_launches": 2 * len(L) * args.steps,
         "clocks": clk,
     }
-    # whole-layer roofline: the slower of FP4 compute and the layer's HBM bytes
-    bytes_alg = (M * K * 2 + 2 * (M * K // 2) + 2 * (M * K // 16) + N * K // 2 + N * K // 16
-                 + K * r * 2 + r * N * 2 + 2 * M * r * 4 + M * N * 2)
+    # whole-step roofline: the slower of 4-bit compute and the step's HBM bytes
+    bytes_alg = sum(layer_bytes(d["layer"]) for d in L)
     t_star = max(flops / (peak * 1e12), bytes_alg / (pk["hbm_gbs"] * 1e9))
     line["frac_of_fp4_roofline"] = t_star / (ms_step * 1e-3)
+    line["frac_of_nominal_roofline"] = max(flops / (nominal * 1e12),
+                                           bytes_alg / (pk["hbm_gbs"] * 1e9)) / (ms_step * 1e-3)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(layer, pw, x_bits, 1024)
+        line["cpu_baseline"] = cpu_baseline(L[0]["layer"], L[0]["pw"], L[0]["x_bits"], 1024)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    h.close()
+    for d in L:
+        d["h"].close()
     if world > 1:
         dist.destroy_process_group()
 
@@ -343,11 +445,11 @@ def run_ours(args, layer):
 def main():
     args = parse()
     from bit_diffusion_transformer_w4a4_b200 import workloads as W
-    layer = W.workloads()[args.workload][0]
+    layers = W.workloads()[args.workload]
     if args.impl == "reference":
-        run_reference(args, layer)
+        run_reference(args, layers)
     else:
-        run_ours(args, layer)
+        run_ours(args, layers)
 
 
 if __name__ == "__main__":

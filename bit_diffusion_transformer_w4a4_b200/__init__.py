@@ -3,4 +3,4 @@
 The compute lives in ``libsvdq.so`` (CUDA, include/svdq.h); ``svdq`` is its
 Python binding and ``workloads`` the seeded synthetic inputs.
 """
-__version__ = "0.1.0"
+__version__ = "0.2.0"

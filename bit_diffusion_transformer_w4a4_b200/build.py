@@ -49,8 +49,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     if not force and not stale():
         return LIB
     cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", os.path.join(ROOT, "include"),
-           os.path.join(CSRC, "svdq_api.cu"), "-o", LIB + ".tmp", "-lcuda" if False else ""]
-    cmd = [c for c in cmd if c]
+           os.path.join(CSRC, "svdq_api.cu"), "-o", LIB + ".tmp"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     r = subprocess.run(cmd, capture_output=True, text=True)

@@ -116,6 +116,9 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // inputs written by the activation kernel: see griddep_wait()
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer

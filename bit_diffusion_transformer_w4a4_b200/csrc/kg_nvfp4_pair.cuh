@@ -23,8 +23,9 @@
 //               counted on the leader's full barrier
 //   warp 1      leader: MMAs for the pair; both CTAs: tensor-memory
 //               allocation (cta_group::2, same warp in both)
-//   warps 2, 3  leader: scale-factor copies for the pair (A's, B's), a stage
-//               ahead of the MMAs, from threads other than the MMA issuer
+//   warps 2, 3  leader: scale-factor copies for the pair (first and second
+//               half of each stage's k-blocks), a stage ahead of the MMAs,
+//               from threads other than the MMA issuer
 //   warps 4-19  epilogue (both CTAs): drain this SM's accumulator half,
 //               prepare the next tile's low-rank operand rows, store
 // Cross-CTA signals: MMA completion is committed to the barrier at the same
@@ -86,8 +87,8 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   const uint32_t bar_drain = smem_u32(bars + 2 * NST + 3);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NST + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const uint32_t bar_sfa = smem_u32(bars + 2 * NST + 5);        // leader: A's scales copied
-  const uint32_t bar_sfb = smem_u32(bars + 3 * NST + 5);        // leader: B's scales copied
+  const uint32_t bar_sfa = smem_u32(bars + 2 * NST + 5);        // leader: k-blocks 0-1 scales copied
+  const uint32_t bar_sfb = smem_u32(bars + 3 * NST + 5);        // leader: k-blocks 2-3 scales copied
   const uint32_t bar_sf_drain = smem_u32(bars + 4 * NST + 5);   // two barriers
 
   const int warp = threadIdx.x >> 5;
@@ -126,6 +127,11 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The activation codes, scales and T come from the previous kernel of the
+  // stream (see griddep_wait()); the producer first issues the weight halves
+  // of the first stages, which do not depend on it.
+  if (!(warp == 0 && lane == 0)) griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -139,17 +145,43 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_par = 0;
       bool ok = true;
+      // Weight half (B codes, B scale atoms) of the first tile's first stages,
+      // issued before the dependency wait: the stage's full barrier completes
+      // only when its activation half has landed too.
+      const int pre = (cid < num_tiles && !(p.debug_mask & 1u)) ? min(NST, nks) : 0;
+      if (pre > 0) {
+        const int nb = cid / p.num_m;
+        const int brow = nb * 256 + static_cast<int>(rank) * 128;
+        for (int ks = 0; ks < pre; ++ks) {  // fresh ring: every slot is free
+          const uint32_t st = sbase + ks * S::STAGE;
+          const uint32_t fb = full0 + 8 * ks;
+          if (rank == 0) mbar_expect_tx(bar_full + 8 * ks, S::TX);
+          tma_load_2d_pair(st + S::A_BYTES, &tm_b, fb, ks * S::ROWB, brow);
+          tma_load_2d_pair(st + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, &tm_sfb, fb, 0,
+                           2 * nb * kblk + KB * ks);
+          tma_load_2d_pair(st + S::A_BYTES + S::B_BYTES + S::SFA_BYTES + KB * 512, &tm_sfb, fb, 0,
+                           (2 * nb + 1) * kblk + KB * ks);
+          issued |= 1u << ks;
+        }
+      }
+      griddep_wait();
       for (int tile = cid, j = 0; tile < num_tiles && ok; tile += nclu, ++j) {
         const int mb = tile % p.num_m, nb = tile / p.num_m;
         const int arow = mb * 256 + static_cast<int>(rank) * 128;   // this CTA's A rows
         const int brow = nb * 256 + static_cast<int>(rank) * 128;   // this CTA's B rows
         const int sfa_atom = (2 * mb + static_cast<int>(rank)) * kblk;
         for (int ks = 0; ks < nks; ++ks) {
+          const uint32_t st = sbase + s * S::STAGE;
+          const uint32_t fb = full0 + 8 * s;
+          if (j == 0 && ks < pre) {  // weight half already in flight: the activation half
+            tma_load_2d_pair(st, &tm_a, fb, ks * S::ROWB, arow);
+            tma_load_2d_pair(st + S::A_BYTES + S::B_BYTES, &tm_sfa, fb, 0, sfa_atom + KB * ks);
+            if (++s == NST) { s = 0; ph ^= 1; }
+            continue;
+          }
           if (!(ok = wait_bounded(bar_empty + 8 * s, ph ^ 1, guard, 0x221))) break;
           issued &= ~(1u << s);
           if (!((p.debug_mask & 1u) && j == 0 && ks == 1)) {  // test hook: leave one stage empty
-            const uint32_t st = sbase + s * S::STAGE;
-            const uint32_t fb = full0 + 8 * s;
             if (rank == 0) mbar_expect_tx(bar_full + 8 * s, S::TX);
             // whole boxes always: rows past M, N or the last k-block are zero-filled
             tma_load_2d_pair(st, &tm_a, fb, ks * S::ROWB, arow);
@@ -195,20 +227,25 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         if (j > 0 && !(ok = wait_bounded_cl(bar_acc_empty, (j - 1) & 1, guard, 0x223))) break;
         tc_fence_after();
         for (int ks = 0; ks < nks; ++ks) {
-          if (!(ok = wait_bounded(bar_sfa + 8 * s, ph, guard, 0x224) &&
-                     wait_bounded(bar_sfb + 8 * s, ph, guard, 0x228)))
-            break;
-          tc_fence_after();
           const uint64_t so = kStage * s;
           const int kv = min(KB, kblk - KB * ks);
           const uint32_t ca = tmem + S::SFA_COL + KB * 4 * s;
           const uint32_t cb = tmem + S::SFB_COL + KB * 8 * s;
+          // first half of the k-blocks once warp 2's copies are in, the second
+          // half once warp 3's are
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) {
-            if (kb >= kv) break;
-            mma_nvf4_pair(tmem, dA0 + so + 2 * kb, dB0 + so + 2 * kb, id_f4, ca + 4 * kb, cb + 8 * kb,
-                          (ks | kb) != 0);
+            if (kb == 0 || kb == KB / 2) {
+              if (!(ok = wait_bounded(kb == 0 ? bar_sfa + 8 * s : bar_sfb + 8 * s, ph, guard,
+                                      kb == 0 ? 0x224 : 0x228)))
+                break;
+              tc_fence_after();
+            }
+            if (kb < kv)
+              mma_nvf4_pair(tmem, dA0 + so + 2 * kb, dB0 + so + 2 * kb, id_f4, ca + 4 * kb, cb + 8 * kb,
+                            (ks | kb) != 0);
           }
+          if (!ok) break;
           tc_commit_pair(bar_empty + 8 * s, 0x3);
           if (++s == NST) { s = 0; ph ^= 1; }
         }
@@ -246,34 +283,35 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     // Each copy lands in both CTAs' tensor memory, from each CTA's own stage;
     // every stage completes the leader's ready barrier once, after the
     // pair's data has landed (the leader's full barrier counts both CTAs).
+    // Warp 2 copies the scale atoms of the stage's first half of k-blocks
+    // (A's and both of B's), warp 3 those of the second half: six copies per
+    // warp and stage, which one warp issues in less time than the stage's
+    // four MMAs take.
     if (lane == 0 && rank == 0) {
-      const bool is_a = warp == 2;
-      const uint32_t ready = is_a ? bar_sfa : bar_sfb;
-      const uint64_t d0 = is_a ? smem_desc(sbase + S::A_BYTES + S::B_BYTES, 0, 128, SWZ_NONE)
-                               : smem_desc(sbase + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, 0, 128, SWZ_NONE);
+      const int h = warp - 2;
+      const uint32_t ready = h == 0 ? bar_sfa : bar_sfb;
+      const uint64_t dA = smem_desc(sbase + S::A_BYTES + S::B_BYTES, 0, 128, SWZ_NONE);
+      const uint64_t dB = smem_desc(sbase + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, 0, 128, SWZ_NONE);
       constexpr uint64_t kStage = S::STAGE >> 4;
+      constexpr int KH = KB / 2;
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
       for (int tile = cid; tile < num_tiles && ok; tile += nclu) {
         for (int ks = 0; ks < nks; ++ks) {
-          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, is_a ? 0x22a : 0x22b))) break;
+          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, h == 0 ? 0x22a : 0x22b))) break;
           tc_fence_after();
-          const uint64_t d = d0 + kStage * s;
           const int kv = min(KB, kblk - KB * ks);
-          if (is_a) {
-            const uint32_t ca = tmem + S::SFA_COL + KB * 4 * s;
+          const uint32_t ca = tmem + S::SFA_COL + KB * 4 * s;
+          const uint32_t cb = tmem + S::SFB_COL + KB * 8 * s;
 #pragma unroll
-            for (int kb = 0; kb < KB; ++kb)
-              if (kb < kv) tmem_cp_32x128b_warpx4_pair(ca + 4 * kb, d + 32 * kb);
-          } else {
-            const uint32_t cb = tmem + S::SFB_COL + KB * 8 * s;
-#pragma unroll
-            for (int kb = 0; kb < KB; ++kb)
-              if (kb < kv) {
-                tmem_cp_32x128b_warpx4_pair(cb + 8 * kb, d + 32 * kb);
-                tmem_cp_32x128b_warpx4_pair(cb + 8 * kb + 4, d + 32 * (KB + kb));
-              }
+          for (int i = 0; i < KH; ++i) {
+            const int kb = h * KH + i;
+            if (kb < kv) {
+              tmem_cp_32x128b_warpx4_pair(ca + 4 * kb, dA + kStage * s + 32 * kb);
+              tmem_cp_32x128b_warpx4_pair(cb + 8 * kb, dB + kStage * s + 32 * kb);
+              tmem_cp_32x128b_warpx4_pair(cb + 8 * kb + 4, dB + kStage * s + 32 * (KB + kb));
+            }
           }
           tc_commit_pair(ready + 8 * s, 0x1);
           if (++s == NST) { s = 0; ph ^= 1; }
@@ -285,7 +323,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         }
       }
       // this warp's copies have completed before tensor memory is freed
-      const uint32_t drain = bar_sf_drain + (is_a ? 0 : 8);
+      const uint32_t drain = bar_sf_drain + 8 * h;
       tc_commit_pair(drain, 0x1);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < p.timeout_ns) {

@@ -183,6 +183,10 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = R > 0 ? *tmem_slot : 0;
+  // X may still be being written by the previous kernel of the stream, and
+  // the outputs may still be read by it: see griddep_wait()
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == PRODUCER) {
     // ---------------------------------------------------------------- producer

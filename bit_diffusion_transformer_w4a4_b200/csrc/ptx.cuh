@@ -120,6 +120,20 @@ __device__ __forceinline__ bool wait_bounded_impl(uint32_t bar, uint32_t parity,
   }
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while
+// the previous kernel of the stream is still running.  griddep_wait() blocks
+// the calling thread until every grid it depends on has completed and its
+// memory writes are visible (it returns at once when there is none), so each
+// thread calls it before touching global memory that the previous kernel
+// writes or reads.  griddep_launch_dependents() lets the next kernel of the
+// stream, if it was launched that way, begin its own prologue once every CTA
+// of this grid has issued it or exited.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // --------------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -109,6 +110,51 @@ svdq_status set_smem(K kernel, int bytes) {
   return SVDQ_OK;
 }
 
+// The dynamic shared-memory opt-in of kernel `Kern` on the current device.
+// The attribute belongs to the device's context, so it is set once per
+// device ordinal (bit `dev` of a per-kernel mask); two threads that race on a
+// first call both set it, which is harmless.
+template <auto Kern>
+svdq_status ensure_smem(int bytes) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SVDQ_ERR_CUDA;
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return SVDQ_OK;
+  svdq_status s = set_smem(Kern, bytes);
+  if (s == SVDQ_OK) done.fetch_or(bit, std::memory_order_release);
+  return s;
+}
+
+// Launch configuration with programmatic stream serialisation: the kernel may
+// start (prologue: barrier set-up, tensor-memory allocation, tensor-map
+// prefetch, weight loads) while the previous kernel of the stream finishes;
+// every kernel of the library waits for that kernel (griddepcontrol.wait)
+// before it reads or writes global memory the previous kernel may touch.
+// `cluster` > 1 adds a cluster dimension.
+struct LaunchCfg {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  LaunchCfg(dim3 grid, dim3 block, int smem, cudaStream_t st, int cluster = 1) {
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int n = 1;
+    if (cluster > 1) {
+      attr[1].id = cudaLaunchAttributeClusterDimension;
+      attr[1].val.clusterDim.x = cluster;
+      attr[1].val.clusterDim.y = 1;
+      attr[1].val.clusterDim.z = 1;
+      n = 2;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+  }
+};
+
 }  // namespace
 
 struct svdq_weights {
@@ -176,12 +222,7 @@ template <int V, int R>
 svdq_status launch_kq_t(svdq_weights* h, const CUtensorMap& tmx, int64_t M, uint8_t* codes,
                         void* scales, float* t, cudaStream_t st) {
   using S = KQSmem<V, R>;
-  static bool attr = false;
-  if (!attr) {
-    svdq_status s = set_smem(kq_kernel<V, R>, S::TOTAL);
-    if (s != SVDQ_OK) return s;
-    attr = true;
-  }
+  if (svdq_status s = ensure_smem<kq_kernel<V, R>>(S::TOTAL); s != SVDQ_OK) return s;
   const int num_m = static_cast<int>(cdiv(M, 128));
   const int kch = static_cast<int>(h->K / 64);
   // split the K range so that the grid fills the SMs in one wave
@@ -204,12 +245,8 @@ svdq_status launch_kq_t(svdq_weights* h, const CUtensorMap& tmx, int64_t M, uint
   p.err = h->err;
   p.debug_mask = h->debug_mask;
   p.timeout_ns = h->timeout_ns;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ksplit, num_m, 1);
-  cfg.blockDim = dim3(KQ_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = S::TOTAL;
-  cfg.stream = st;
-  SVDQ_TRY(cudaLaunchKernelEx(&cfg, kq_kernel<V, R>, tmx, h->tm_l1t, p));
+  LaunchCfg lc(dim3(ksplit, num_m, 1), dim3(KQ_THREADS, 1, 1), S::TOTAL, st);
+  SVDQ_TRY(cudaLaunchKernelEx(&lc.cfg, kq_kernel<V, R>, tmx, h->tm_l1t, p));
   return SVDQ_OK;
 }
 
@@ -230,12 +267,7 @@ template <int R>
 svdq_status launch_kg_int4h_t(svdq_weights* h, const CUtensorMap& tma, int64_t M, const uint8_t* sfa,
                               const float* t, void* y, cudaStream_t st) {
   using S = KGI4HSmem<R>;
-  static bool attr = false;
-  if (!attr) {
-    svdq_status s = set_smem(kg_int4h_kernel<R>, S::TOTAL);
-    if (s != SVDQ_OK) return s;
-    attr = true;
-  }
+  if (svdq_status s = ensure_smem<kg_int4h_kernel<R>>(S::TOTAL); s != SVDQ_OK) return s;
   KGParams p;
   p.sfa = sfa;
   p.sfb = h->wscales;
@@ -253,8 +285,8 @@ svdq_status launch_kg_int4h_t(svdq_weights* h, const CUtensorMap& tma, int64_t M
   p.timeout_ns = h->timeout_ns;
   const int tiles = p.num_m * p.num_n;
   const int grid = tiles < h->sms ? tiles : h->sms;
-  kg_int4h_kernel<R><<<grid, KGI4H_THREADS, S::TOTAL, st>>>(tma, h->tm_bh, h->tm_blrh, p);
-  SVDQ_TRY(cudaGetLastError());
+  LaunchCfg lc(dim3(grid), dim3(KGI4H_THREADS), S::TOTAL, st);
+  SVDQ_TRY(cudaLaunchKernelEx(&lc.cfg, kg_int4h_kernel<R>, tma, h->tm_bh, h->tm_blrh, p));
   return SVDQ_OK;
 }
 
@@ -266,12 +298,9 @@ svdq_status launch_kg_t(svdq_weights* h, const CUtensorMap& tma, int64_t M, cons
   }
   const int smem = V == 1 ? KGF4Smem<R>::TOTAL : KGI4Smem<R>::TOTAL;
   auto kern = V == 1 ? kg_nvfp4_kernel<R> : kg_int4_kernel<R>;
-  static bool attr = false;
-  if (!attr) {
-    svdq_status s = set_smem(kern, smem);
-    if (s != SVDQ_OK) return s;
-    attr = true;
-  }
+  if (svdq_status s = V == 1 ? ensure_smem<kg_nvfp4_kernel<R>>(smem) : ensure_smem<kg_int4_kernel<R>>(smem);
+      s != SVDQ_OK)
+    return s;
   KGParams p;
   p.sfa = sfa;
   p.sfb = h->wscales;
@@ -289,20 +318,22 @@ svdq_status launch_kg_t(svdq_weights* h, const CUtensorMap& tma, int64_t M, cons
   p.timeout_ns = h->timeout_ns;
   const int tiles = p.num_m * p.num_n;
   const int grid = tiles < h->sms ? tiles : h->sms;
-  kern<<<grid, KG_THREADS, smem, st>>>(tma, h->tm_b, h->tm_blr, p);
-  SVDQ_TRY(cudaGetLastError());
+  LaunchCfg lc(dim3(grid), dim3(KG_THREADS), smem, st);
+  SVDQ_TRY(cudaLaunchKernelEx(&lc.cfg, kern, tma, h->tm_b, h->tm_blr, p));
   return SVDQ_OK;
 }
 
-// Clusters of two CTAs that fit on the device at once for this kernel
-// (0 if the pair kernel cannot be resident).
+// Clusters of two CTAs that fit on the handle's device at once for this
+// kernel (0 if the pair kernel cannot be resident), cached per device
+// ordinal (stored + 1, so 0 means not yet known).
 template <int R>
 int pair_clusters(svdq_weights* h) {
   using S = KGF4PairSmem<R>;
-  static int clusters = -1;
-  if (clusters >= 0) return clusters;
-  clusters = 0;
-  if (set_smem(kg_nvfp4_pair_kernel<R>, S::TOTAL) != SVDQ_OK) return 0;
+  static std::atomic<int> cache[64];
+  if (h->device < 0 || h->device >= 64) return 0;
+  const int known = cache[h->device].load(std::memory_order_acquire);
+  if (known > 0) return known - 1;
+  if (ensure_smem<kg_nvfp4_pair_kernel<R>>(S::TOTAL) != SVDQ_OK) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (h->sms / 2));
   cfg.blockDim = dim3(KG_THREADS);
@@ -317,10 +348,10 @@ int pair_clusters(svdq_weights* h) {
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, kg_nvfp4_pair_kernel<R>, &cfg) != cudaSuccess) {
     cudaGetLastError();
-    n = 0;
+    return 0;  // not cached: the next call asks again
   }
-  clusters = n;
-  return clusters;
+  cache[h->device].store(n + 1, std::memory_order_release);
+  return n;
 }
 
 template <int R>
@@ -344,19 +375,8 @@ svdq_status launch_kg_pair_t(svdq_weights* h, int64_t M, const uint8_t* sfa, con
   p.timeout_ns = h->timeout_ns;
   const int tiles = p.num_m * p.num_n;
   const int n = tiles < clusters ? tiles : clusters;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * n);
-  cfg.blockDim = dim3(KG_THREADS);
-  cfg.dynamicSmemBytes = S::TOTAL;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  SVDQ_TRY(cudaLaunchKernelEx(&cfg, kg_nvfp4_pair_kernel<R>, h->tm_a2, h->tm_b2, h->tm_blr2,
+  LaunchCfg lc(dim3(2 * n), dim3(KG_THREADS), S::TOTAL, st, 2);
+  SVDQ_TRY(cudaLaunchKernelEx(&lc.cfg, kg_nvfp4_pair_kernel<R>, h->tm_a2, h->tm_b2, h->tm_blr2,
                               h->tm_sfa2, h->tm_sfb2, p));
   return SVDQ_OK;
 }
@@ -530,12 +550,7 @@ svdq_status launch_kq_static(const CUtensorMap& tmx, const CUtensorMap& tml, con
                              int64_t M, int64_t K, int sms, uint8_t* codes, void* scales, float* t,
                              unsigned char* scratch, int* err, cudaStream_t st) {
   using S = KQSmem<V, R>;
-  static bool attr = false;
-  if (!attr) {
-    svdq_status s = set_smem(kq_kernel<V, R>, S::TOTAL);
-    if (s != SVDQ_OK) return s;
-    attr = true;
-  }
+  if (svdq_status s = ensure_smem<kq_kernel<V, R>>(S::TOTAL); s != SVDQ_OK) return s;
   const int num_m = static_cast<int>(cdiv(M, 128));
   const int kch = static_cast<int>(K / 64);
   int ksplit = 1;  // same split rule as the handle-based entry point
@@ -600,7 +615,7 @@ const char* svdq_status_string(svdq_status s) {
   return "SVDQ_ERR_UNKNOWN";
 }
 
-const char* svdq_version(void) { return "svdq 0.1.0 sm_100a"; }
+const char* svdq_version(void) { return "svdq 0.2.0 sm_100a"; }
 
 svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, void* stream) {
   if (!d || !out) return SVDQ_ERR_INVALID_ARG;

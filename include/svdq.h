@@ -116,6 +116,13 @@ typedef struct {
 } svdq_weight_desc;
 
 /*
+ * Defined by: "Nunchaku Lite ..." (axbrief.com), section "The Mechanics of
+ * 4-Bit Efficiency and SVDQuant" -- the layer's weights are the smoothing
+ * (outliers shifted from activations into weights), a 16-bit low-rank branch
+ * and a 4-bit residual; section "Hardware Specialization and the Compression
+ * Workflow" -- INT4 or NVFP4 precision, a CUDA capability check that refuses
+ * unsupported devices; "Nunchaku 1.3.0 ..." (note.com), section "SVDQ-FP4 on
+ * Blackwell", item "1. INT4" -- INT4 codes are -8..+7 times a scale.
  * Copy and re-tile the weights into library-owned device memory on the
  * current device and size the forward workspace for max_M tokens.
  * The weight scales of the NVFP4 variant are re-tiled into the tensor-core
@@ -126,10 +133,12 @@ typedef struct {
  */
 svdq_status svdq_weights_load(const svdq_weight_desc* desc, svdq_weights_t* out, void* stream);
 
-/* Free a handle (NULL is a no-op).  Synchronises the device first. */
+/* Free a handle (NULL is a no-op).  Synchronises the device first.  No
+ * counterpart on the pages: resource release for svdq_weights_load. */
 svdq_status svdq_weights_free(svdq_weights_t h);
 
 /*
+ * Layout helper for kernel 1's output (no counterpart on the pages).
  * Size in bytes of the activation-scale buffer for M tokens:
  *   INT4 : M * (K/64) * 2          canonical [M x K/64] bf16
  *   NVFP4: ceil(M/128)*128 * (K/16) the tensor-core tiled layout (below)
@@ -137,6 +146,12 @@ svdq_status svdq_weights_free(svdq_weights_t h);
 svdq_status svdq_act_scales_bytes(svdq_weights_t h, int64_t M, size_t* bytes);
 
 /*
+ * Defined by: "Problemas do Nunchaku Qwen ..." (apatero.com), section "O que
+ * e Nunchaku e como acelera modelos Qwen" -- the low-rank down projection is
+ * fused with the activation quantisation kernel so both branches share the
+ * activations; "Nunchaku Lite ..." (axbrief.com), section "The Mechanics of
+ * 4-Bit Efficiency and SVDQuant" -- activation outliers are divided out
+ * before the activations are quantised to 4 bits (W4A4).
  * Kernel 1: smooth, quantise and pack the activations, and compute the
  * rank-r down projection from the same tiles.
  *   x          bf16 [M x K]
@@ -157,6 +172,11 @@ svdq_status svdq_quantize_act_lowrank_down(svdq_weights_t h, const void* x, int6
                                            void* stream);
 
 /*
+ * Defined by: "Problemas do Nunchaku Qwen ..." (apatero.com), section "O que
+ * e Nunchaku e como acelera modelos Qwen" -- the up projection is fused with
+ * the 4-bit compute kernel; "Nunchaku Lite ..." (axbrief.com), section "The
+ * Mechanics of 4-Bit Efficiency and SVDQuant" -- the 4-bit residual branch
+ * with 4-bit weights and activations, added to the 16-bit low-rank branch.
  * Kernel 2: the 4-bit GEMM on the packed residual with the low-rank up
  * projection, optional bias and GELU fused into the epilogue.
  *   act_codes, act_scales, t  as written by kernel 1 (t ignored when r == 0)
@@ -168,11 +188,21 @@ svdq_status svdq_w4a4_gemm_lowrank_up(svdq_weights_t h, const uint8_t* act_codes
                                       const void* act_scales, const float* t, int64_t M,
                                       void* y, void* stream);
 
-/* Both kernels back to back through the handle's workspace: y = layer(x). */
+/*
+ * Defined by: "Nunchaku Lite ..." (axbrief.com), section "The Mechanics of
+ * 4-Bit Efficiency and SVDQuant" -- the quantised layer replaces a standard
+ * linear layer (SVDQW4A4Linear in place of nn.Linear): y = layer(x).
+ * Both kernels back to back through the handle's workspace.  Kernel 2 is
+ * launched as a programmatic dependent of kernel 1 (its set-up overlaps
+ * kernel 1's tail); every kernel of the library waits for the previous
+ * kernel of the stream before it touches global memory.
+ *   x  bf16 [M x K], y  bf16 [M x N]
+ */
 svdq_status svdq_linear_forward(svdq_weights_t h, const void* x, void* y, int64_t M,
                                 void* stream);
 
 /*
+ * Defined by: the same layer as svdq_linear_forward.
  * Same as svdq_linear_forward with HOST input and output (pinned memory is
  * recommended): copies x_host to the device, runs the layer and copies y back
  * on `stream`.  Returns after enqueueing; synchronise the stream before
@@ -194,7 +224,9 @@ svdq_status svdq_linear_forward_host(svdq_weights_t h, const void* x_host, void*
  *   l1t         device bf16 [r x K]  L1 transposed (NULL when r == 0)
  *   x, act_codes, act_scales, t      as for svdq_quantize_act_lowrank_down
  *   device_error device int, set to a nonzero wait-site code if a bounded
- *               wait expires (never cleared by the library); may be NULL
+ *               wait expires (never cleared by the library).  May be NULL:
+ *               such a failure is then reported to no one, and the outputs
+ *               of that call may be incomplete without any sign of it
  * The split-K scratch (partial T tiles and per-row-block arrival counters)
  * lives in a static device array of the library: 10 MiB of partial tiles
  * plus counters for M <= 524288 tokens, held by every GPU that loads the
@@ -215,14 +247,15 @@ svdq_status svdq_quantize_act_lowrank_down_static(svdq_variant variant, int64_t 
                                                   void* stream);
 
 /*
+ * Failure reporting (no counterpart on the pages).
  * Synchronise `stream` and report device-side failures recorded by earlier
  * calls on this handle (SVDQ_ERR_DEVICE_TIMEOUT), clearing the record.
  */
 svdq_status svdq_device_status(svdq_weights_t h, void* stream);
 
 /*
- * Test hook: make the next launches wait on a pipeline stage that is never
- * filled (mask bit 0: GEMM producer skips one stage; bit 1: activation
+ * Test hook (no counterpart on the pages): make the next launches wait on a
+ * pipeline stage that is never filled (mask bit 0: GEMM producer skips one stage; bit 1: activation
  * kernel producer skips one stage) and use `timeout_us` as the bounded-wait
  * limit (0 restores the default of 2 s).  The kernels then return early and
  * record SVDQ_ERR_DEVICE_TIMEOUT; no GPU fault is involved.
@@ -230,6 +263,7 @@ svdq_status svdq_device_status(svdq_weights_t h, void* stream);
 svdq_status svdq_debug_set_fault(svdq_weights_t h, uint32_t mask, uint32_t timeout_us);
 
 /*
+ * Test hook (no counterpart on the pages).
  * Self-test of the activation quantiser's division (x / s is computed with a
  * reciprocal and one fma correction step).  Runs it against IEEE fp32
  * division for every bf16 dividend and every positive finite scale of
@@ -244,10 +278,11 @@ svdq_status svdq_debug_set_fault(svdq_weights_t h, uint32_t mask, uint32_t timeo
  */
 svdq_status svdq_selftest_division(int variant, unsigned long long* mismatches);
 
-/* Human-readable name of a status code (static storage). */
+/* Human-readable name of a status code (static storage); no counterpart on
+ * the pages. */
 const char* svdq_status_string(svdq_status s);
 
-/* Library version, e.g. "svdq 0.1.0 sm_100a". */
+/* Library version, e.g. "svdq 0.2.0 sm_100a"; no counterpart on the pages. */
 const char* svdq_version(void);
 
 #ifdef __cplusplus
