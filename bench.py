@@ -442,9 +442,130 @@ def run_ours(args, layers):
         dist.destroy_process_group()
 
 
+def run_awq(args, layer):
+    """The AWQ W4A16 modulation linear: one call per step, HBM-bound on the
+    4-bit weight stream."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from bit_diffusion_transformer_w4a4_b200 import svdq
+    from bit_diffusion_transformer_w4a4_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    M, K, N = layer.M, layer.K, layer.N
+    if args.impl == "reference":
+        if rank == 0:
+            from oracle import awq as A
+            p = W.synthetic_awq(layer)
+            xb = W.awq_activations(layer)
+            for _ in range(min(args.warmup, 3)):
+                A.forward(xb, p)
+            ts = []
+            for _ in range(min(args.steps, 20)):
+                t = time.perf_counter()
+                A.forward(xb, p)
+                ts.append(time.perf_counter() - t)
+            ms = statistics.median(ts) * 1e3
+            v = (layer.weight_bytes() + M * K * 2 + M * N * 2) / (ms * 1e-3) / 1e9
+            print(json.dumps({"metric": f"AWQ W4A16 linear weight-stream GB/s at M{M} K{K} N{N}", "value": v,
+                              "unit": "GB/s", "n_gpus": args.gpus, "steps": len(ts), "warmup": min(args.warmup, 3),
+                              "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                              "dtype": "f64", "data": "synthetic", "impl": "reference",
+                              "config": {"workload": f"{layer.name} M{M} K{K} N{N} awq_w4a16_g64"},
+                              "cpu_baseline": {"value": v, "unit": "GB/s", "kind": "oracle",
+                                               "cores": os.cpu_count(), "sample": "the whole call"},
+                              "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    p = W.synthetic_awq(layer, seed=rank)
+    xb = W.awq_activations(layer, seed=rank)
+    h = svdq.AWQWeights(p, M)
+    x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush_w.zero_(); flush_r.sum()
+        h.forward(x, y, M)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush_w.zero_(); flush_r.sum()
+        evs[i][0].record(stream)
+        h.forward(x, y, M)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    (ms,) = max_over_ranks([ms], "cuda")
+    nbytes = layer.weight_bytes() + M * K * 2 + M * N * 2 + K * 4 + (N * 2 if p.bias is not None else 0)
+    gbs = world * nbytes / (ms * 1e-3) / 1e9
+    xh = torch.from_numpy(xb.view(np.int16)).pin_memory()
+    yh = torch.empty((M, N), dtype=torch.int16).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    xd = torch.empty_like(x)
+    n_e2e = max(3, min(args.steps, 50))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        xd.view(torch.int16).copy_(xh, non_blocking=True)
+        h.forward(xd, y, M)
+        yh.copy_(y.view(torch.int16), non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / n_e2e
+    (ms_e2e,) = max_over_ranks([ms_e2e], "cuda")
+    pk, pk_src = peaks()
+    line = {"metric": f"AWQ W4A16 linear weight-stream GB/s at M{M} K{K} N{N}", "value": gbs, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x int4",
+            "data": "synthetic",
+            "config": {"workload": f"{layer.name} M{M} K{K} N{N} awq_w4a16_g64",
+                       "l2": "flushed before every step (256 MB write, then 256 MB read; outside the timed events)",
+                       "parallelism": f"replicas x{world}"},
+            "tokens_per_s": world * M / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "traffic": recorded_traffic("awq_w4a16_forward", args.workload),
+                         "peak_source": f"{pk_src} copy bandwidth", "kernel": "kawq_kernel",
+                         "bytes_per_launch": nbytes},
+            "e2e": {"value": world * nbytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+            "gpu_launches": args.steps, "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import awq as A
+        t = time.perf_counter()
+        A.forward(xb, p)
+        dt = time.perf_counter() - t
+        line["cpu_baseline"] = {"value": nbytes / dt / 1e9, "unit": "GB/s", "kind": "oracle",
+                                "cores": os.cpu_count(), "sample": f"the whole call (numpy fp64), {dt:.2f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     from bit_diffusion_transformer_w4a4_b200 import workloads as W
+    if args.workload in W.awq_workloads():
+        run_awq(args, W.awq_workloads()[args.workload])
+        return
     layers = W.workloads()[args.workload]
     if args.impl == "reference":
         run_reference(args, layers)

@@ -1,0 +1,162 @@
+// AWQ W4A16 linear layer: 4-bit weights with group scales and integer zero
+// points, 16-bit activations, y = (x / a) . W_deq^T (+ bias).
+//
+// Method: "Nunchaku Lite ... integrated into Diffusers" (axbrief.com),
+// section "The Mechanics of 4-Bit Efficiency and SVDQuant" (AWQW4A16Linear:
+// 4-bit weights, 16-bit activations) and section "The Trade-off Between Fused
+// Kernels and Generality" (the scanner gives modulation linear layers AWQ
+// W4A16).  Modulation layers take one token per image (M = batch), so the
+// layer is a matrix-vector product bound by the HBM stream of the 4-bit
+// weights: it runs on the CUDA cores, not the tensor cores.
+//
+// Per element: x' = fp32(x) *_RN fp32(1/a_k) (fp32, not rounded further);
+// for each group g of 64 along K: part = sum_{k in g} x'_k (q_k - z_g) in
+// fp32 (q - z is an exact small integer), y += s_g * part.
+//
+// Layout: codes [N x K/2] bytes (element 2j in the low nibble), group
+// parameters [N x K/64] 32-bit words (bf16 scale in the high half, zero
+// point in the low byte), 1/a fp32 [K], bias bf16 [N] or null.
+//
+// Work split: a CTA stages x' of up to MT tokens in shared memory (one
+// 32-element chunk per 36 floats, so the lanes' 16-byte reads of their own
+// chunks hit distinct banks), then each warp takes RW weight rows at a time;
+// lane l reads the 16-byte code chunks l, l+32, ... of each row (a warp reads
+// 512 contiguous bytes per load), decodes eight codes per word with byte
+// permutes into fp32 2^23 + q, subtracts 2^23 + z and accumulates
+// x' (q - z) with packed fp32x2 FMAs; the row's partial sums meet in a warp
+// shuffle reduction.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace svdq {
+
+constexpr int AWQ_THREADS = 256;
+constexpr int AWQ_G = 64;
+constexpr int AWQ_RW = 4;  // weight rows per warp and pass
+
+// byte `sel` of a, as the fp32 bit pattern 0x4B0000bb (= 2^23 + byte)
+template <int SEL>
+__device__ __forceinline__ uint32_t byte_as_magic(uint32_t a) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(0x4B000000u), "n"(0x7440 + SEL));
+  return d;
+}
+
+struct AWQParams {
+  const uint8_t* codes;   // [N x K/2]
+  const uint32_t* gp;     // [N x K/64]: (bf16 scale << 16) | zero
+  const float* inv_a;     // [K]
+  const uint16_t* x;      // bf16 [M x K]
+  const uint16_t* bias;   // bf16 [N] or null
+  uint16_t* y;            // bf16 [M x N]
+  int M, K, N;
+};
+
+template <int MT>
+struct AWQSmem {
+  static size_t bytes(int K) { return static_cast<size_t>(MT) * (K / 32) * 36 * 4; }
+};
+
+template <int MT>
+__global__ void __launch_bounds__(AWQ_THREADS)
+    kawq_kernel(AWQParams p) {
+  extern __shared__ __align__(16) float xs[];  // [MT][K/32][36]
+  const int nck = p.K / 32;                    // 16-byte code chunks per row
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpb = AWQ_THREADS / 32;
+  const int gstride = gridDim.x * wpb * AWQ_RW;
+  // x may still be written by the previous kernel of the stream
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int m0 = 0; m0 < p.M; m0 += MT) {
+    const int mt = min(MT, p.M - m0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < MT * (p.K / 2); i += AWQ_THREADS) {
+      const int m = i / (p.K / 2), k = 2 * (i % (p.K / 2));
+      float v0 = 0.f, v1 = 0.f;
+      if (m < mt) {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p.x + static_cast<size_t>(m0 + m) * p.K + k));
+        const float2 ia = __ldg(reinterpret_cast<const float2*>(p.inv_a + k));
+        v0 = __fmul_rn(bf16lo(w), ia.x);
+        v1 = __fmul_rn(bf16hi(w), ia.y);
+      }
+      *reinterpret_cast<float2*>(xs + (m * nck + k / 32) * 36 + (k % 32)) = make_float2(v0, v1);
+    }
+    __syncthreads();
+    for (int n0 = (blockIdx.x * wpb + warp) * AWQ_RW; n0 < p.N; n0 += gstride) {
+      float acc[AWQ_RW][MT];
+#pragma unroll
+      for (int r = 0; r < AWQ_RW; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
+      for (int ci = lane; ci < nck; ci += 32) {
+        uint4 cw[AWQ_RW];
+        uint32_t gw[AWQ_RW];
+#pragma unroll
+        for (int r = 0; r < AWQ_RW; ++r) {
+          const int n = min(n0 + r, p.N - 1);  // rows past N recompute row N-1, never stored
+          cw[r] = __ldcs(reinterpret_cast<const uint4*>(p.codes + static_cast<size_t>(n) * (p.K / 2)) + ci);
+          gw[r] = __ldg(p.gp + static_cast<size_t>(n) * (p.K / AWQ_G) + ci / 2);
+        }
+        const float* xc = xs + ci * 36;
+#pragma unroll
+        for (int r = 0; r < AWQ_RW; ++r) {
+          const float nz = -(8388608.0f + static_cast<float>(gw[r] & 0xFFu));
+          const uint64_t nzz = f2_pack(nz, nz);
+          uint64_t part[MT];
+#pragma unroll
+          for (int m = 0; m < MT; ++m) part[m] = 0ull;
+          const uint32_t words[4] = {cw[r].x, cw[r].y, cw[r].z, cw[r].w};
+#pragma unroll
+          for (int wi = 0; wi < 4; ++wi) {
+            const uint32_t lo = words[wi] & 0x0F0F0F0Fu;         // codes 8wi + 2b
+            const uint32_t hi = (words[wi] >> 4) & 0x0F0F0F0Fu;  // codes 8wi + 2b + 1
+            uint64_t q[4];
+            q[0] = f2_add(f2_pack(__uint_as_float(byte_as_magic<0>(lo)), __uint_as_float(byte_as_magic<0>(hi))), nzz);
+            q[1] = f2_add(f2_pack(__uint_as_float(byte_as_magic<1>(lo)), __uint_as_float(byte_as_magic<1>(hi))), nzz);
+            q[2] = f2_add(f2_pack(__uint_as_float(byte_as_magic<2>(lo)), __uint_as_float(byte_as_magic<2>(hi))), nzz);
+            q[3] = f2_add(f2_pack(__uint_as_float(byte_as_magic<3>(lo)), __uint_as_float(byte_as_magic<3>(hi))), nzz);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              const float4 xa = *reinterpret_cast<const float4*>(xc + m * nck * 36 + 8 * wi);
+              const float4 xb = *reinterpret_cast<const float4*>(xc + m * nck * 36 + 8 * wi + 4);
+              part[m] = f2_fma(f2_pack(xa.x, xa.y), q[0], part[m]);
+              part[m] = f2_fma(f2_pack(xa.z, xa.w), q[1], part[m]);
+              part[m] = f2_fma(f2_pack(xb.x, xb.y), q[2], part[m]);
+              part[m] = f2_fma(f2_pack(xb.z, xb.w), q[3], part[m]);
+            }
+          }
+          const float s = __uint_as_float(gw[r] & 0xFFFF0000u);
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const float ps = __fadd_rn(f2_lo(part[m]), f2_hi(part[m]));
+            acc[r][m] = __fmaf_rn(s, ps, acc[r][m]);
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < AWQ_RW; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          float v = acc[r][m];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          acc[r][m] = v;
+        }
+      // lane r*MT + m stores output (m, n0 + r)
+#pragma unroll
+      for (int r = 0; r < AWQ_RW; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+          if (lane == r * MT + m && m < mt && n0 + r < p.N) {
+            float v = acc[r][m];
+            if (p.bias) v = __fadd_rn(v, bf16lo(p.bias[n0 + r]));
+            const __nv_bfloat16 b = __float2bfloat16_rn(v);
+            p.y[static_cast<size_t>(m0 + m) * p.N + n0 + r] = *reinterpret_cast<const uint16_t*>(&b);
+          }
+    }
+  }
+}
+
+}  // namespace svdq

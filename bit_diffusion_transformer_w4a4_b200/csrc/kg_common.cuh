@@ -28,6 +28,18 @@ struct KGParams {
   int M, N, K;
   int num_m, num_n;
   int gelu;
+  // NVFP4 weights with a per-tensor scale 2^e: the accumulator is multiplied
+  // by out_scale = 2^e before bias / GELU and T by t_scale = 2^-e before the
+  // low-rank MMAs (both exact powers of two; 1 otherwise)
+  float out_scale, t_scale;
+  // fused QKV epilogue (qkv_hd > 0): columns [Q | K | V] of qkv_hd each; Q
+  // and K heads (128 features) RMS-normalised (times gq / gk, bf16 [128]) and
+  // rotated pairwise by rope (fp32 [M x 64 x 2]: cos, sin per token and pair)
+  int qkv_hd;
+  float norm_eps;
+  const uint16_t* gq;
+  const uint16_t* gk;
+  const float* rope;
   int* err;
   uint32_t debug_mask;
   uint64_t timeout_ns;
@@ -47,7 +59,7 @@ __device__ __forceinline__ float gelu_tanh(float x) {
 // Called by NT epilogue threads (etid = 0..NT-1).
 template <int R, int NT = KG_EPI_WARPS * 32>
 __device__ __forceinline__ void prep_lowrank_a(uint8_t* alr, const float* __restrict__ t, int m0,
-                                               int M, int etid) {
+                                               int M, int etid, float tsc = 1.0f) {
   constexpr int SEG = R / 8;  // 8 values of T per item
   for (int it = etid; it < 128 * SEG; it += NT) {
     const int row = it / SEG;
@@ -59,7 +71,8 @@ __device__ __forceinline__ void prep_lowrank_a(uint8_t* alr, const float* __rest
       a = __ldg(src);
       b = __ldg(src + 1);
     }
-    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const float v[8] = {__fmul_rn(a.x, tsc), __fmul_rn(a.y, tsc), __fmul_rn(a.z, tsc), __fmul_rn(a.w, tsc),
+                        __fmul_rn(b.x, tsc), __fmul_rn(b.y, tsc), __fmul_rn(b.z, tsc), __fmul_rn(b.w, tsc)};
     uint32_t hi[4], lo[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -87,6 +100,8 @@ __device__ __forceinline__ void prep_lowrank_a(uint8_t* alr, const float* __rest
 // leaves lane 8g+c with chunk c of the rows of lanes 8g..8g+7.  Store k then
 // writes, per 8-lane group, one contiguous 128-byte row segment, instead of
 // 32 scattered 16-byte pieces.  All 32 lanes must call it.
+// With FINAL the 64 values are already the outputs (no scale, bias or GELU).
+template <bool FINAL = false>
 __device__ __forceinline__ void store_rows64_coalesced(const KGParams& p, int row0, int n_base,
                                                        const float* acc, int lane) {
   uint32_t w[32];
@@ -95,8 +110,8 @@ __device__ __forceinline__ void store_rows64_coalesced(const KGParams& p, int ro
     const int n = n_base + 8 * j8;
     float v[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = acc[8 * j8 + e];
-    if (p.bias != nullptr && n < p.N) {
+    for (int e = 0; e < 8; ++e) v[e] = FINAL ? acc[8 * j8 + e] : __fmul_rn(acc[8 * j8 + e], p.out_scale);
+    if (!FINAL && p.bias != nullptr && n < p.N) {
       const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
       const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
@@ -105,7 +120,7 @@ __device__ __forceinline__ void store_rows64_coalesced(const KGParams& p, int ro
         v[2 * e + 1] = __fadd_rn(v[2 * e + 1], bf16hi(bw[e]));
       }
     }
-    if (p.gelu) {
+    if (!FINAL && p.gelu) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = gelu_tanh(v[e]);
     }
@@ -150,7 +165,7 @@ __device__ __forceinline__ void store_rows32_coalesced(const KGParams& p, int ro
     const int n = n_base + 8 * j8;
     float v[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = acc[8 * j8 + e];
+    for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(acc[8 * j8 + e], p.out_scale);
     if (p.bias != nullptr && n < p.N) {
       const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
       const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
@@ -192,6 +207,80 @@ __device__ __forceinline__ void store_rows32_coalesced(const KGParams& p, int ro
       *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(gm) * p.N + n) =
           make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
   }
+}
+
+// Fused QKV epilogue for one epilogue warp's 32 rows x 64 columns
+// [n_base, n_base + 64) (row = row0 + lane), then the coalesced store.
+// "Nunchaku Lite ..." (axbrief.com), section "The Trade-off Between Fused
+// Kernels and Generality": the QKV projection, the Q/K normalisation and the
+// rotary embedding in one kernel.  Per value: v = acc * out_scale (+ bias);
+// for Q and K columns, per 128-feature head: v <- v / sqrt(mean(v^2) + eps)
+// * g, then pairs (2i, 2i+1) rotated by token row's (cos, sin) of pair i.
+// A head spans two warps (slices cs and cs ^ 1 of the same lane quarter q).
+// Each publishes its rows' partial sums of squares in red ([4][4][32]
+// floats) and the pair exchanges them through mbarrier xbar[q + 4 (cs/2)]
+// (64 arrivals a phase): phase 2k when both have written, 2k + 1 when both
+// have read, so the next tile's write cannot overtake the partner's read.
+// The two partials are added in slice order (both warps use the same sum).
+// Waits are bounded; false means the CTA is aborting.
+__device__ __forceinline__ bool epilogue_qkv64(const KGParams& p, int row0, int n_base, const float* acc,
+                                               int lane, int q, int cs, float* red, uint32_t xbar,
+                                               uint32_t& xph, const Guard& guard) {
+  float v[64];
+#pragma unroll
+  for (int c = 0; c < 64; ++c) v[c] = __fmul_rn(acc[c], p.out_scale);
+  if (p.bias != nullptr && n_base < p.N) {
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+      const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n_base + 8 * c8));
+      const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[8 * c8 + 2 * e] = __fadd_rn(v[8 * c8 + 2 * e], bf16lo(bw[e]));
+        v[8 * c8 + 2 * e + 1] = __fadd_rn(v[8 * c8 + 2 * e + 1], bf16hi(bw[e]));
+      }
+    }
+  }
+  if (n_base < 2 * p.qkv_hd && n_base < p.N) {
+    const uint16_t* g = n_base < p.qkv_hd ? p.gq : p.gk;
+    const int d0 = n_base % 128;  // first feature of this slice within its head
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) ss = __fmaf_rn(v[c], v[c], ss);
+    const uint32_t xb = xbar + 8 * (q + 4 * (cs >> 1));
+    red[(q * 4 + cs) * 32 + lane] = ss;
+    mbar_arrive(xb);
+    if (!__all_sync(0xffffffffu, wait_bounded(xb, xph & 1, guard, 0x240))) return false;
+    const float tot = __fadd_rn(red[(q * 4 + (cs & ~1)) * 32 + lane], red[(q * 4 + (cs | 1)) * 32 + lane]);
+    mbar_arrive(xb);
+    if (!__all_sync(0xffffffffu, wait_bounded(xb, (xph + 1) & 1, guard, 0x241))) return false;
+    xph += 2;
+    const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, 128.0f), p.norm_eps)));
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+      const uint4 gg = __ldg(reinterpret_cast<const uint4*>(g + d0 + 8 * c8));
+      const uint32_t gw[4] = {gg.x, gg.y, gg.z, gg.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[8 * c8 + 2 * e] = __fmul_rn(__fmul_rn(v[8 * c8 + 2 * e], inv), bf16lo(gw[e]));
+        v[8 * c8 + 2 * e + 1] = __fmul_rn(__fmul_rn(v[8 * c8 + 2 * e + 1], inv), bf16hi(gw[e]));
+      }
+    }
+    const int row = row0 + lane;
+    const float4* cs4 =
+        reinterpret_cast<const float4*>(p.rope + (static_cast<size_t>(row < p.M ? row : 0) * 64 + d0 / 2) * 2);
+#pragma unroll
+    for (int i2 = 0; i2 < 16; ++i2) {  // two pairs per 16-byte load: (cos, sin, cos, sin)
+      const float4 t = row < p.M ? __ldg(cs4 + i2) : make_float4(1.f, 0.f, 1.f, 0.f);
+      const float a0 = v[4 * i2], b0 = v[4 * i2 + 1], a1 = v[4 * i2 + 2], b1 = v[4 * i2 + 3];
+      v[4 * i2] = __fsub_rn(__fmul_rn(a0, t.x), __fmul_rn(b0, t.y));
+      v[4 * i2 + 1] = __fadd_rn(__fmul_rn(a0, t.y), __fmul_rn(b0, t.x));
+      v[4 * i2 + 2] = __fsub_rn(__fmul_rn(a1, t.z), __fmul_rn(b1, t.w));
+      v[4 * i2 + 3] = __fadd_rn(__fmul_rn(a1, t.w), __fmul_rn(b1, t.z));
+    }
+  }
+  store_rows64_coalesced<true>(p, row0, n_base, v, lane);
+  return true;
 }
 
 // Wait for the producer's outstanding loads before the CTA exits (abort path).

@@ -50,25 +50,6 @@ struct KGI4Smem {
   static_assert(TOTAL <= 232448, "shared memory per CTA");
 };
 
-// Paired fp32 arithmetic (one instruction per two lanes of data).
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ float f2_lo(uint64_t a) { return __uint_as_float(static_cast<uint32_t>(a)); }
-__device__ __forceinline__ float f2_hi(uint64_t a) { return __uint_as_float(static_cast<uint32_t>(a >> 32)); }
-
 // 8 two's-complement nibbles (element 0 in the low nibble) -> 8 int8 bytes.
 __device__ __forceinline__ uint2 unpack_s4x8(uint32_t w) {
   uint32_t lo = w & 0x0F0F0F0Fu;          // elements 0, 2, 4, 6

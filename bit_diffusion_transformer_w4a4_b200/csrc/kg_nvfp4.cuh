@@ -50,7 +50,9 @@ struct KGF4Smem {
   static constexpr int LR_STAGES = (LR_STEPS + KB - 1) / KB;  // a stage row holds KB k-steps
   static constexpr int ALR_OFF = STAGES * STAGE;
   static constexpr int BAR_OFF = ALR_OFF + LR_CHUNKS * 16384;
-  static constexpr int TOTAL = BAR_OFF + 256 + 1024;
+  static constexpr int RED_OFF = BAR_OFF + 256;      // QKV epilogue: [4][4][32] partial sums
+  static constexpr int XBAR_OFF = RED_OFF + 2048;    // QKV epilogue: 8 exchange mbarriers
+  static constexpr int TOTAL = XBAR_OFF + 64 + 1024;
   // tensor memory columns: accumulator [0, 256), then scale factors
   static constexpr int SFA_COL = 256;
   static constexpr int SFB_COL = 256 + 4 * KB * STAGES;
@@ -105,6 +107,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     }
     mbar_init(bar_sf_drain, 1);
     mbar_init(bar_sf_drain + 8, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(smem_u32(smem + S::XBAR_OFF) + 8 * i, 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -287,9 +290,12 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     const int cs = e >> 2;         // 64-column slice
     const int etid = threadIdx.x - 128;
     uint8_t* alr = smem + S::ALR_OFF;
+    float* red = reinterpret_cast<float*>(smem + S::RED_OFF);  // QKV epilogue partial sums
+    const uint32_t xbar = smem_u32(smem + S::XBAR_OFF);
+    uint32_t xph = 0;
     if constexpr (R > 0) {
       if (static_cast<int>(blockIdx.x) < num_tiles) {
-        prep_lowrank_a<R>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid);
+        prep_lowrank_a<R>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid, p.t_scale);
         fence_proxy_async_smem();
         mbar_arrive(bar_lr_full);
       }
@@ -309,13 +315,18 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       if constexpr (R > 0) {
         const int next = tile + gridDim.x;
         if (next < num_tiles) {
-          prep_lowrank_a<R>(alr, p.t, (next % p.num_m) * KG_BM, p.M, etid);
+          prep_lowrank_a<R>(alr, p.t, (next % p.num_m) * KG_BM, p.M, etid, p.t_scale);
           fence_proxy_async_smem();
           mbar_arrive(bar_lr_full);
         }
       }
-      store_rows64_coalesced(p, mb * KG_BM + q * 32, nb * KG_BN + cs * 64,
-                             reinterpret_cast<const float*>(v), lane);
+      if (p.qkv_hd > 0) {
+        if (!epilogue_qkv64(p, mb * KG_BM + q * 32, nb * KG_BN + cs * 64, reinterpret_cast<const float*>(v),
+                            lane, q, cs, red, xbar, xph, guard))
+          break;
+      } else
+        store_rows64_coalesced(p, mb * KG_BM + q * 32, nb * KG_BN + cs * 64,
+                               reinterpret_cast<const float*>(v), lane);
     }
   }
 

@@ -57,7 +57,9 @@ struct KGF4PairSmem {
   static constexpr int LR_STAGES = (LR_STEPS + KB - 1) / KB;
   static constexpr int ALR_OFF = STAGES * STAGE;
   static constexpr int BAR_OFF = ALR_OFF + LR_CHUNKS * 16384;
-  static constexpr int TOTAL = BAR_OFF + 256 + 1024;
+  static constexpr int RED_OFF = BAR_OFF + 256;      // QKV epilogue: [4][4][32] partial sums
+  static constexpr int XBAR_OFF = RED_OFF + 2048;    // QKV epilogue: 8 exchange mbarriers
+  static constexpr int TOTAL = XBAR_OFF + 64 + 1024;
   static constexpr int SFA_COL = 256;
   static constexpr int SFB_COL = 256 + 4 * KB * STAGES;
   static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
@@ -116,6 +118,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     }
     mbar_init(bar_sf_drain, 1);
     mbar_init(bar_sf_drain + 8, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(smem_u32(smem + S::XBAR_OFF) + 8 * i, 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -336,11 +339,14 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     const int cs = e >> 2;         // 64-column slice
     const int etid = threadIdx.x - 128;
     uint8_t* alr = smem + S::ALR_OFF;
+    float* red = reinterpret_cast<float*>(smem + S::RED_OFF);  // QKV epilogue partial sums
+    const uint32_t xbar = smem_u32(smem + S::XBAR_OFF);
+    uint32_t xph = 0;
     const uint32_t acc_empty0 = mapa_shared(bar_acc_empty, 0);
     const uint32_t lr_full0 = mapa_shared(bar_lr_full, 0);
     if constexpr (R > 0) {
       if (cid < num_tiles) {
-        prep_lowrank_a<R>(alr, p.t, (cid % p.num_m) * 256 + static_cast<int>(rank) * 128, p.M, etid);
+        prep_lowrank_a<R>(alr, p.t, (cid % p.num_m) * 256 + static_cast<int>(rank) * 128, p.M, etid, p.t_scale);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(lr_full0);
@@ -361,14 +367,19 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       if constexpr (R > 0) {
         const int next = tile + nclu;
         if (next < num_tiles) {
-          prep_lowrank_a<R>(alr, p.t, (next % p.num_m) * 256 + static_cast<int>(rank) * 128, p.M, etid);
+          prep_lowrank_a<R>(alr, p.t, (next % p.num_m) * 256 + static_cast<int>(rank) * 128, p.M, etid, p.t_scale);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(lr_full0);
         }
       }
-      store_rows64_coalesced(p, mb * 256 + static_cast<int>(rank) * 128 + q * 32, nb * KG_BN + cs * 64,
-                             reinterpret_cast<const float*>(v), lane);
+      if (p.qkv_hd > 0) {
+        if (!epilogue_qkv64(p, mb * 256 + static_cast<int>(rank) * 128 + q * 32, nb * KG_BN + cs * 64, reinterpret_cast<const float*>(v),
+                            lane, q, cs, red, xbar, xph, guard))
+          break;
+      } else
+        store_rows64_coalesced(p, mb * 256 + static_cast<int>(rank) * 128 + q * 32, nb * KG_BN + cs * 64,
+                               reinterpret_cast<const float*>(v), lane);
     }
   }
 

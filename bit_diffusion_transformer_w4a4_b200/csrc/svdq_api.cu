@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -15,6 +16,8 @@
 #include <vector>
 
 #include "../../include/svdq.h"
+#include "kawq.cuh"
+#include "kprep.cuh"
 #include "kg_int4.cuh"
 #include "kg_int4h.cuh"
 #include "kg_nvfp4.cuh"
@@ -164,6 +167,13 @@ struct svdq_weights {
   uint32_t stage_row_bytes = 64;  // bytes per operand row in one GEMM pipeline stage
   uint32_t flags;
   int device, sms;
+  float out_scale = 1.0f, t_scale = 1.0f;  // 2^e and 2^-e of the NVFP4 per-tensor scale
+  // fused QKV epilogue (SVDQ_EPI_QKV_NORM_ROPE): norm weights, epsilon, and
+  // the rotary table of the call being launched
+  uint16_t* gq = nullptr;
+  uint16_t* gk = nullptr;
+  float norm_eps = 0.f;
+  const float* rope = nullptr;
   // device weights (library-owned)
   float* inv_lam = nullptr;
   uint16_t* l1t = nullptr;     // [r x K]
@@ -212,7 +222,8 @@ size_t act_scale_bytes(const svdq_weights* h, int64_t M) {
 
 void free_all(svdq_weights* h) {
   void* ptrs[] = {h->inv_lam, h->l1t, h->l2dup, h->wcodes, h->wscales, h->wh, h->bias, h->ws_codes,
-                  h->ws_scales, h->ws_t, h->x_dev, h->y_dev, h->err, h->kq_tpart, h->kq_counters};
+                  h->ws_scales, h->ws_t, h->x_dev, h->y_dev, h->err, h->kq_tpart, h->kq_counters,
+                  h->gq, h->gk};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -280,6 +291,13 @@ svdq_status launch_kg_int4h_t(svdq_weights* h, const CUtensorMap& tma, int64_t M
   p.num_m = static_cast<int>(cdiv(M, KG_BM));
   p.num_n = static_cast<int>(cdiv(h->N, KG_BN));
   p.gelu = (h->flags & SVDQ_EPI_GELU) ? 1 : 0;
+  p.out_scale = h->out_scale;
+  p.t_scale = h->t_scale;
+  p.qkv_hd = (h->flags & SVDQ_EPI_QKV_NORM_ROPE) ? static_cast<int>(h->N / 3) : 0;
+  p.norm_eps = h->norm_eps;
+  p.gq = h->gq;
+  p.gk = h->gk;
+  p.rope = h->rope;
   p.err = h->err;
   p.debug_mask = h->debug_mask;
   p.timeout_ns = h->timeout_ns;
@@ -313,6 +331,13 @@ svdq_status launch_kg_t(svdq_weights* h, const CUtensorMap& tma, int64_t M, cons
   p.num_m = static_cast<int>(cdiv(M, KG_BM));
   p.num_n = static_cast<int>(cdiv(h->N, V == 1 ? KG_BN : KGI4_BN));
   p.gelu = (h->flags & SVDQ_EPI_GELU) ? 1 : 0;
+  p.out_scale = h->out_scale;
+  p.t_scale = h->t_scale;
+  p.qkv_hd = (h->flags & SVDQ_EPI_QKV_NORM_ROPE) ? static_cast<int>(h->N / 3) : 0;
+  p.norm_eps = h->norm_eps;
+  p.gq = h->gq;
+  p.gk = h->gk;
+  p.rope = h->rope;
   p.err = h->err;
   p.debug_mask = h->debug_mask;
   p.timeout_ns = h->timeout_ns;
@@ -370,6 +395,13 @@ svdq_status launch_kg_pair_t(svdq_weights* h, int64_t M, const uint8_t* sfa, con
   p.num_m = static_cast<int>(cdiv(M, 256));
   p.num_n = static_cast<int>(cdiv(h->N, KG_BN));
   p.gelu = (h->flags & SVDQ_EPI_GELU) ? 1 : 0;
+  p.out_scale = h->out_scale;
+  p.t_scale = h->t_scale;
+  p.qkv_hd = (h->flags & SVDQ_EPI_QKV_NORM_ROPE) ? static_cast<int>(h->N / 3) : 0;
+  p.norm_eps = h->norm_eps;
+  p.gq = h->gq;
+  p.gk = h->gk;
+  p.rope = h->rope;
   p.err = h->err;
   p.debug_mask = h->debug_mask;
   p.timeout_ns = h->timeout_ns;
@@ -597,6 +629,189 @@ svdq_status launch_kq_static_v(int64_t r, const CUtensorMap& tmx, const CUtensor
 
 }  // namespace
 
+struct svdq_awq {
+  int64_t K, N, max_M;
+  int device, sms;
+  uint8_t* codes = nullptr;   // [N x K/2]
+  uint32_t* gp = nullptr;     // [N x K/64]: (bf16 scale << 16) | zero point
+  float* inv_a = nullptr;     // [K]
+  uint16_t* bias = nullptr;   // [N] or null
+};
+
+namespace {
+
+void awq_free_all(svdq_awq* h) {
+  void* ptrs[] = {h->codes, h->gp, h->inv_a, h->bias};
+  for (void* q : ptrs)
+    if (q) cudaFree(q);
+}
+
+template <int MT>
+svdq_status launch_awq(svdq_awq* h, const void* x, void* y, int64_t M, cudaStream_t st) {
+  const size_t smem = AWQSmem<MT>::bytes(static_cast<int>(h->K));
+  if (svdq_status s = ensure_smem<kawq_kernel<MT>>(static_cast<int>(smem)); s != SVDQ_OK) return s;
+  AWQParams p;
+  p.codes = h->codes;
+  p.gp = h->gp;
+  p.inv_a = h->inv_a;
+  p.x = static_cast<const uint16_t*>(x);
+  p.bias = h->bias;
+  p.y = static_cast<uint16_t*>(y);
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(h->K);
+  p.N = static_cast<int>(h->N);
+  const int64_t rows_per_cta = (AWQ_THREADS / 32) * AWQ_RW;
+  const int64_t want = cdiv(h->N, rows_per_cta);
+  const int grid = static_cast<int>(want < 4 * h->sms ? want : 4 * h->sms);
+  LaunchCfg lc(dim3(grid), dim3(AWQ_THREADS), static_cast<int>(smem), st);
+  SVDQ_TRY(cudaLaunchKernelEx(&lc.cfg, kawq_kernel<MT>, p));
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+
+// ------------------------------------------------------------ weight prep
+namespace {
+
+// fp64 -> bf16 bits, round to nearest even (values in bf16's normal range
+// or zero; the prep only rounds factor entries of moderate magnitude).
+uint16_t bf16_bits_rn(double v) {
+  if (v == 0.0) return std::signbit(v) ? 0x8000u : 0u;
+  int ex;
+  std::frexp(v, &ex);
+  const int lead = std::max(ex - 1, -126);
+  const int ue = lead - 7;
+  const double q = std::ldexp(std::nearbyint(std::ldexp(v, -ue)), ue);  // default rounding mode: to nearest even
+  const float f = static_cast<float>(q);                                  // exact
+  uint32_t b;
+  std::memcpy(&b, &f, 4);
+  return static_cast<uint16_t>(b >> 16);
+}
+
+// Upper-triangular R with R^T R = G (G symmetric positive definite, l x l,
+// row-major) and its inverse; false if G is not numerically positive.
+bool cholesky_inv(const std::vector<double>& G, int l, std::vector<double>& Rinv) {
+  std::vector<double> R(static_cast<size_t>(l) * l, 0.0);
+  for (int i = 0; i < l; ++i) {
+    double d = G[i * l + i];
+    for (int k = 0; k < i; ++k) d -= R[k * l + i] * R[k * l + i];
+    if (!(d > 0.0)) return false;
+    R[i * l + i] = std::sqrt(d);
+    for (int j = i + 1; j < l; ++j) {
+      double v = G[i * l + j];
+      for (int k = 0; k < i; ++k) v -= R[k * l + i] * R[k * l + j];
+      R[i * l + j] = v / R[i * l + i];
+    }
+  }
+  Rinv.assign(static_cast<size_t>(l) * l, 0.0);
+  for (int j = 0; j < l; ++j) {  // solve R x = e_j by back substitution
+    for (int i = l - 1; i >= 0; --i) {
+      double v = (i == j) ? 1.0 : 0.0;
+      for (int k = i + 1; k < l; ++k) v -= R[i * l + k] * Rinv[k * l + j];
+      Rinv[i * l + j] = v / R[i * l + i];
+    }
+  }
+  return true;
+}
+
+// Eigen-decomposition of a symmetric l x l matrix by cyclic Jacobi rotations:
+// A = V diag(ev) V^T, eigenvalues in descending order, V's columns the vectors.
+void jacobi_eig(std::vector<double> A, int l, std::vector<double>& ev, std::vector<double>& V) {
+  V.assign(static_cast<size_t>(l) * l, 0.0);
+  for (int i = 0; i < l; ++i) V[i * l + i] = 1.0;
+  for (int sweep = 0; sweep < 100; ++sweep) {
+    double off = 0.0, tot = 0.0;
+    for (int i = 0; i < l; ++i)
+      for (int j = 0; j < l; ++j) {
+        tot += A[i * l + j] * A[i * l + j];
+        if (i != j) off += A[i * l + j] * A[i * l + j];
+      }
+    if (off <= 1e-30 * tot) break;
+    for (int p = 0; p < l - 1; ++p)
+      for (int q = p + 1; q < l; ++q) {
+        const double apq = A[p * l + q];
+        if (apq == 0.0) continue;
+        const double theta = (A[q * l + q] - A[p * l + p]) / (2.0 * apq);
+        const double t = (theta >= 0 ? 1.0 : -1.0) / (std::fabs(theta) + std::sqrt(theta * theta + 1.0));
+        const double c = 1.0 / std::sqrt(t * t + 1.0), sn = t * c;
+        for (int k = 0; k < l; ++k) {  // A = J^T A J
+          const double akp = A[k * l + p], akq = A[k * l + q];
+          A[k * l + p] = c * akp - sn * akq;
+          A[k * l + q] = sn * akp + c * akq;
+        }
+        for (int k = 0; k < l; ++k) {
+          const double apk = A[p * l + k], aqk = A[q * l + k];
+          A[p * l + k] = c * apk - sn * aqk;
+          A[q * l + k] = sn * apk + c * aqk;
+        }
+        for (int k = 0; k < l; ++k) {
+          const double vkp = V[k * l + p], vkq = V[k * l + q];
+          V[k * l + p] = c * vkp - sn * vkq;
+          V[k * l + q] = sn * vkp + c * vkq;
+        }
+      }
+  }
+  std::vector<int> idx(l);
+  for (int i = 0; i < l; ++i) idx[i] = i;
+  std::sort(idx.begin(), idx.end(), [&](int a, int b) { return A[a * l + a] > A[b * l + b]; });
+  std::vector<double> V2(static_cast<size_t>(l) * l);
+  ev.resize(l);
+  for (int c = 0; c < l; ++c) {
+    ev[c] = A[idx[c] * l + idx[c]];
+    for (int k = 0; k < l; ++k) V2[k * l + c] = V[k * l + idx[c]];
+  }
+  V.swap(V2);
+}
+
+struct DevBuf {
+  void* p = nullptr;
+  ~DevBuf() { if (p) cudaFree(p); }
+  bool alloc(size_t bytes) {
+    if (cudaMalloc(&p, bytes < 256 ? 256 : bytes) != cudaSuccess) {
+      cudaGetLastError();
+      p = nullptr;
+      return false;
+    }
+    return true;
+  }
+  template <class T> T* as() const { return static_cast<T*>(p); }
+};
+
+// C = op(A) op(B) (fp32) with split-K over the contraction, C zeroed first.
+svdq_status gemm_f32(const float* A, int64_t as0, int64_t as1, const float* B, int64_t bs0, int64_t bs1,
+                     float* C, int64_t Mr, int64_t Nc, int64_t Kd, int sms, cudaStream_t st) {
+  SVDQ_TRY(cudaMemsetAsync(C, 0, static_cast<size_t>(Mr) * Nc * 4, st));
+  const int64_t tiles = cdiv(Mr, 64) * cdiv(Nc, 64);
+  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(cdiv(4 * sms, tiles), cdiv(Kd, 256)));
+  const int64_t kslice = cdiv(cdiv(Kd, splits), 16) * 16;
+  splits = cdiv(Kd, kslice);
+  dim3 grid(static_cast<unsigned>(cdiv(Nc, 64)), static_cast<unsigned>(cdiv(Mr, 64)), static_cast<unsigned>(splits));
+  prep_gemm_f32_kernel<<<grid, 256, 0, st>>>(A, as0, as1, B, bs0, bs1, C, Nc, Mr, Nc, Kd, kslice);
+  SVDQ_TRY(cudaGetLastError());
+  return SVDQ_OK;
+}
+
+// Y [rows x l] := an orthonormal basis of its column span, by two rounds of
+// Cholesky QR (Gram matrix in fp64 on the GPU, its factor on the host).
+svdq_status orthonormalize(float* Y, int64_t rows, int l, double* G_dev, cudaStream_t st) {
+  for (int round = 0; round < 2; ++round) {
+    prep_gram_f64_kernel<<<dim3(l, l), 256, 0, st>>>(Y, rows, l, G_dev);
+    SVDQ_TRY(cudaGetLastError());
+    std::vector<double> G(static_cast<size_t>(l) * l), Rinv;
+    SVDQ_TRY(cudaMemcpyAsync(G.data(), G_dev, G.size() * 8, cudaMemcpyDeviceToHost, st));
+    SVDQ_TRY(cudaStreamSynchronize(st));
+    if (!cholesky_inv(G, l, Rinv)) return SVDQ_ERR_RANGE;
+    SVDQ_TRY(cudaMemcpyAsync(G_dev, Rinv.data(), Rinv.size() * 8, cudaMemcpyHostToDevice, st));
+    prep_rmul_small_kernel<<<static_cast<unsigned>(cdiv(rows, 128)), 128, l * l * 8, st>>>(Y, rows, l, G_dev);
+    SVDQ_TRY(cudaGetLastError());
+    SVDQ_TRY(cudaStreamSynchronize(st));  // Rinv (host) outlives the copy
+  }
+  return SVDQ_OK;
+}
+
+}  // namespace
+
 // ====================================================================== C ABI
 extern "C" {
 
@@ -621,13 +836,21 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
   if (!d || !out) return SVDQ_ERR_INVALID_ARG;
   *out = nullptr;
   if (d->variant != SVDQ_INT4_G64_BF16 && d->variant != SVDQ_NVFP4_G16_E4M3) return SVDQ_ERR_INVALID_ARG;
-  if (d->flags & ~(SVDQ_EPI_GELU | SVDQ_GEMM_SINGLE_SM | SVDQ_INT4_F16)) return SVDQ_ERR_INVALID_ARG;
+  if (d->flags & ~(SVDQ_EPI_GELU | SVDQ_GEMM_SINGLE_SM | SVDQ_INT4_F16 | SVDQ_EPI_QKV_NORM_ROPE))
+    return SVDQ_ERR_INVALID_ARG;
+  if (d->flags & SVDQ_EPI_QKV_NORM_ROPE) {
+    if (d->variant != SVDQ_NVFP4_G16_E4M3 || (d->flags & SVDQ_EPI_GELU)) return SVDQ_ERR_INVALID_ARG;
+    if (!d->q_norm || !d->k_norm || !(d->norm_eps > 0.0f) || !(d->norm_eps < 1.0f)) return SVDQ_ERR_INVALID_ARG;
+    if (d->N % 384 != 0) return SVDQ_ERR_SHAPE;
+  }
   const int64_t K = d->K, N = d->N, r = d->r;
   if (K < 128 || K % 128 != 0 || K > (1 << 20)) return SVDQ_ERR_SHAPE;
   if (N < 16 || N % 16 != 0 || N > (1 << 20)) return SVDQ_ERR_SHAPE;
   if (!(r == 0 || r == 16 || r == 32 || r == 64 || r == 128)) return SVDQ_ERR_SHAPE;
   if (d->max_M < 1 || d->max_M > (1ll << 30)) return SVDQ_ERR_SHAPE;
   if (!d->lambda || !d->w_codes || !d->w_scales) return SVDQ_ERR_INVALID_ARG;
+  if (d->w_scale_exp != 0 && d->variant != SVDQ_NVFP4_G16_E4M3) return SVDQ_ERR_INVALID_ARG;
+  if (d->w_scale_exp < -100 || d->w_scale_exp > 100) return SVDQ_ERR_INVALID_ARG;
   if (r > 0 && (!d->L1 || !d->L2)) return SVDQ_ERR_INVALID_ARG;
   for (int64_t k = 0; k < K; ++k)
     if (!(d->lambda[k] > 0.0f) || !(d->lambda[k] < INFINITY)) return SVDQ_ERR_INVALID_ARG;
@@ -644,6 +867,8 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
   h->max_M = d->max_M;
   h->npad = cdiv(N, 256) * 256;
   h->flags = d->flags;
+  h->out_scale = std::ldexp(1.0f, d->w_scale_exp);
+  h->t_scale = std::ldexp(1.0f, -d->w_scale_exp);
   h->device = dev;
   h->sms = sms;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -733,6 +958,14 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
                 !dmalloc(reinterpret_cast<void**>(&h->ws_t), static_cast<size_t>(h->max_M) * r * 4)))
     return fail(SVDQ_ERR_OOM);
   if (d->bias && !dmalloc(reinterpret_cast<void**>(&h->bias), N * 2)) return fail(SVDQ_ERR_OOM);
+  if (d->flags & SVDQ_EPI_QKV_NORM_ROPE) {
+    if (!dmalloc(reinterpret_cast<void**>(&h->gq), 256) || !dmalloc(reinterpret_cast<void**>(&h->gk), 256))
+      return fail(SVDQ_ERR_OOM);
+    if (cudaMemcpy(h->gq, d->q_norm, 256, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(h->gk, d->k_norm, 256, cudaMemcpyHostToDevice) != cudaSuccess)
+      return fail(SVDQ_ERR_CUDA);
+    h->norm_eps = d->norm_eps;
+  }
   if (!wh.empty() && !dmalloc(reinterpret_cast<void**>(&h->wh), wh.size() * 2)) return fail(SVDQ_ERR_OOM);
   if (r > 0 && (!dmalloc(reinterpret_cast<void**>(&h->kq_tpart), static_cast<size_t>(sms) * 128 * r * 4) ||
                 !dmalloc(reinterpret_cast<void**>(&h->kq_counters), cdiv(h->max_M, 128) * 4)))
@@ -846,6 +1079,7 @@ svdq_status svdq_w4a4_gemm_lowrank_up(svdq_weights_t h, const uint8_t* act_codes
                                       void* stream) {
   svdq_status s = check_call(h, M);
   if (s != SVDQ_OK) return s;
+  if ((h->flags & SVDQ_EPI_QKV_NORM_ROPE) && !h->rope) return SVDQ_ERR_INVALID_ARG;  // use the _qkv call
   if (!act_codes || !act_scales || !y || (h->r > 0 && !t)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(y) || (t && !aligned16(t)))
     return SVDQ_ERR_ALIGNMENT;
@@ -862,6 +1096,25 @@ svdq_status svdq_linear_forward(svdq_weights_t h, const void* x, void* y, int64_
                                                  stream);
   if (s != SVDQ_OK) return s;
   return svdq_w4a4_gemm_lowrank_up(h, h->ws_codes, h->ws_scales, h->ws_t, M, y, stream);
+}
+
+svdq_status svdq_w4a4_gemm_lowrank_up_qkv(svdq_weights_t h, const uint8_t* act_codes,
+                                          const void* act_scales, const float* t, int64_t M,
+                                          const float* rope, void* y, void* stream) {
+  if (!h || !(h->flags & SVDQ_EPI_QKV_NORM_ROPE) || !rope) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(rope)) return SVDQ_ERR_ALIGNMENT;
+  h->rope = rope;
+  const svdq_status s = svdq_w4a4_gemm_lowrank_up(h, act_codes, act_scales, t, M, y, stream);
+  h->rope = nullptr;
+  return s;
+}
+
+svdq_status svdq_linear_forward_qkv(svdq_weights_t h, const void* x, const float* rope, void* y, int64_t M,
+                                    void* stream) {
+  if (!h || !(h->flags & SVDQ_EPI_QKV_NORM_ROPE) || !rope) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = svdq_quantize_act_lowrank_down(h, x, M, h->ws_codes, h->ws_scales, h->ws_t, stream);
+  if (s != SVDQ_OK) return s;
+  return svdq_w4a4_gemm_lowrank_up_qkv(h, h->ws_codes, h->ws_scales, h->ws_t, M, rope, y, stream);
 }
 
 svdq_status svdq_linear_forward_host(svdq_weights_t h, const void* x_host, void* y_host, int64_t M,
@@ -943,6 +1196,211 @@ svdq_status svdq_quantize_act_lowrank_down_static(svdq_variant variant, int64_t 
   return variant == SVDQ_NVFP4_G16_E4M3
              ? launch_kq_static_v<1>(r, tmx, tml, inv_lambda, M, K, sms, act_codes, act_scales, t, scratch, err, st)
              : launch_kq_static_v<0>(r, tmx, tml, inv_lambda, M, K, sms, act_codes, act_scales, t, scratch, err, st);
+}
+
+svdq_status svdq_awq_load(const svdq_awq_desc* d, svdq_awq_t* out, void* stream) {
+  if (!d || !out) return SVDQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  const int64_t K = d->K, N = d->N;
+  if (K < 64 || K % 64 != 0 || K > 32768) return SVDQ_ERR_SHAPE;
+  if (N < 1 || N > (1 << 24)) return SVDQ_ERR_SHAPE;
+  if (d->max_M < 1 || d->max_M > (1ll << 30)) return SVDQ_ERR_SHAPE;
+  if (!d->a || !d->codes || !d->scales || !d->zeros) return SVDQ_ERR_INVALID_ARG;
+  for (int64_t k = 0; k < K; ++k)
+    if (!(d->a[k] > 0.0f) || !(d->a[k] < INFINITY)) return SVDQ_ERR_INVALID_ARG;
+  const int64_t ng = K / 64;
+  for (int64_t i = 0; i < N * ng; ++i)
+    if (d->zeros[i] > 15) return SVDQ_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  svdq_status ds = check_device(&dev, &sms);
+  if (ds != SVDQ_OK) return ds;
+  svdq_awq* h = new (std::nothrow) svdq_awq();
+  if (!h) return SVDQ_ERR_OOM;
+  h->K = K;
+  h->N = N;
+  h->max_M = d->max_M;
+  h->device = dev;
+  h->sms = sms;
+  auto fail = [&](svdq_status st) {
+    cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    awq_free_all(h);
+    delete h;
+    return st;
+  };
+  std::vector<float> inv(K);
+  for (int64_t k = 0; k < K; ++k) inv[k] = 1.0f / d->a[k];  // IEEE fp32 division
+  std::vector<uint32_t> gp(static_cast<size_t>(N) * ng);
+  for (size_t i = 0; i < gp.size(); ++i)
+    gp[i] = (static_cast<uint32_t>(d->scales[i]) << 16) | d->zeros[i];
+  if (cudaMalloc(reinterpret_cast<void**>(&h->codes), static_cast<size_t>(N) * (K / 2)) != cudaSuccess ||
+      cudaMalloc(reinterpret_cast<void**>(&h->gp), gp.size() * 4) != cudaSuccess ||
+      cudaMalloc(reinterpret_cast<void**>(&h->inv_a), K * 4) != cudaSuccess ||
+      (d->bias && cudaMalloc(reinterpret_cast<void**>(&h->bias), N * 2) != cudaSuccess)) {
+    cudaGetLastError();
+    return fail(SVDQ_ERR_OOM);
+  }
+  if (cudaMemcpy(h->codes, d->codes, static_cast<size_t>(N) * (K / 2), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(h->gp, gp.data(), gp.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(h->inv_a, inv.data(), K * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      (d->bias && cudaMemcpy(h->bias, d->bias, N * 2, cudaMemcpyHostToDevice) != cudaSuccess))
+    return fail(SVDQ_ERR_CUDA);
+  *out = h;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_awq_free(svdq_awq_t h) {
+  if (!h) return SVDQ_OK;
+  cudaDeviceSynchronize();
+  awq_free_all(h);
+  delete h;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_awq_w4a16_forward(svdq_awq_t h, const void* x, void* y, int64_t M, void* stream) {
+  if (!h) return SVDQ_ERR_INVALID_ARG;
+  if (M < 1 || M > h->max_M) return SVDQ_ERR_SHAPE;
+  if (!x || !y) return SVDQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 1u)) return SVDQ_ERR_ALIGNMENT;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (dev != h->device) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // tokens staged per pass: as many as fit, up to 8
+  const size_t cap = 200 * 1024;
+  if (M >= 5 && AWQSmem<8>::bytes(static_cast<int>(h->K)) <= cap) return launch_awq<8>(h, x, y, M, st);
+  if (M >= 3 && AWQSmem<4>::bytes(static_cast<int>(h->K)) <= cap) return launch_awq<4>(h, x, y, M, st);
+  if (M >= 2 && AWQSmem<2>::bytes(static_cast<int>(h->K)) <= cap) return launch_awq<2>(h, x, y, M, st);
+  return launch_awq<1>(h, x, y, M, st);
+}
+
+svdq_status svdq_prep_calibrate(const void* x, int64_t M, const void* w, int64_t K, int64_t N, float alpha,
+                                float* lambda, void* stream) {
+  if (!x || !w || !lambda) return SVDQ_ERR_INVALID_ARG;
+  if (M < 1 || K < 1 || N < 1 || M > (1ll << 31) || K > (1ll << 24) || N > (1ll << 24)) return SVDQ_ERR_SHAPE;
+  if (!(alpha >= 0.0f && alpha <= 1.0f)) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_device(nullptr, nullptr);
+  if (s != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevBuf ax, aw;
+  if (!ax.alloc(K * 4) || !aw.alloc(K * 4)) return SVDQ_ERR_OOM;
+  SVDQ_TRY(cudaMemsetAsync(ax.p, 0, K * 4, st));
+  const int rows_per = 256;
+  prep_col_amax_kernel<<<dim3(static_cast<unsigned>(cdiv(K, 256)), static_cast<unsigned>(cdiv(M, rows_per))), 256, 0, st>>>(
+      static_cast<const uint16_t*>(x), M, K, rows_per, ax.as<unsigned>());
+  prep_row_amax_kernel<<<static_cast<unsigned>(K), 256, 0, st>>>(static_cast<const uint16_t*>(w), K, N, aw.as<unsigned>());
+  prep_lambda_kernel<<<static_cast<unsigned>(cdiv(K, 256)), 256, 0, st>>>(ax.as<unsigned>(), aw.as<unsigned>(), K,
+                                                                           static_cast<double>(alpha), lambda);
+  SVDQ_TRY(cudaGetLastError());
+  SVDQ_TRY(cudaStreamSynchronize(st));  // the scratch is freed on return
+  return SVDQ_OK;
+}
+
+svdq_status svdq_prep_lowrank(const void* w, const float* lambda, int64_t K, int64_t N, int64_t r,
+                              const float* omega, int64_t l, int power_iters, uint16_t* L1, uint16_t* L2,
+                              void* stream) {
+  if (!w || !lambda || !omega || !L1 || !L2) return SVDQ_ERR_INVALID_ARG;
+  if (K < 1 || N < 1 || K > (1 << 20) || N > (1 << 20)) return SVDQ_ERR_SHAPE;
+  if (r < 1 || l < r || l > 64 || l > K || l > N) return SVDQ_ERR_SHAPE;
+  if (power_iters < 0 || power_iters > 8) return SVDQ_ERR_INVALID_ARG;
+  int sms = 0;
+  svdq_status s = check_device(nullptr, &sms);
+  if (s != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int li = static_cast<int>(l);
+  DevBuf wh, Y, Z, B, G;
+  if (!wh.alloc(static_cast<size_t>(K) * N * 4) || !Y.alloc(static_cast<size_t>(K) * l * 4) ||
+      !Z.alloc(static_cast<size_t>(N) * l * 4) || !B.alloc(static_cast<size_t>(l) * N * 4) || !G.alloc(l * l * 8))
+    return SVDQ_ERR_OOM;
+  float* W = wh.as<float>();
+  prep_smooth_kernel<<<static_cast<unsigned>(cdiv(K * N, 256)), 256, 0, st>>>(static_cast<const uint16_t*>(w), lambda,
+                                                                               K, N, W);
+  SVDQ_TRY(cudaGetLastError());
+  // range finder: Y = W_hat Omega, then power iterations Y = W_hat (W_hat^T Y)
+  if ((s = gemm_f32(W, N, 1, omega, l, 1, Y.as<float>(), K, l, N, sms, st)) != SVDQ_OK) return s;
+  if ((s = orthonormalize(Y.as<float>(), K, li, G.as<double>(), st)) != SVDQ_OK) return s;
+  for (int it = 0; it < power_iters; ++it) {
+    if ((s = gemm_f32(W, 1, N, Y.as<float>(), l, 1, Z.as<float>(), N, l, K, sms, st)) != SVDQ_OK) return s;
+    if ((s = orthonormalize(Z.as<float>(), N, li, G.as<double>(), st)) != SVDQ_OK) return s;
+    if ((s = gemm_f32(W, N, 1, Z.as<float>(), l, 1, Y.as<float>(), K, l, N, sms, st)) != SVDQ_OK) return s;
+    if ((s = orthonormalize(Y.as<float>(), K, li, G.as<double>(), st)) != SVDQ_OK) return s;
+  }
+  // B = Q^T W_hat [l x N]
+  if ((s = gemm_f32(Y.as<float>(), 1, l, W, N, 1, B.as<float>(), l, N, K, sms, st)) != SVDQ_OK) return s;
+  std::vector<float> Bh(static_cast<size_t>(l) * N), Qh(static_cast<size_t>(K) * l);
+  SVDQ_TRY(cudaMemcpyAsync(Bh.data(), B.p, Bh.size() * 4, cudaMemcpyDeviceToHost, st));
+  SVDQ_TRY(cudaMemcpyAsync(Qh.data(), Y.p, Qh.size() * 4, cudaMemcpyDeviceToHost, st));
+  SVDQ_TRY(cudaStreamSynchronize(st));
+  // small SVD of B on the host (fp64): B B^T = U diag(sigma^2) U^T, V = B^T U / sigma
+  std::vector<double> C(static_cast<size_t>(l) * l, 0.0);
+  for (int a = 0; a < li; ++a)
+    for (int b = a; b < li; ++b) {
+      double t = 0.0;
+      for (int64_t n = 0; n < N; ++n) t += static_cast<double>(Bh[a * N + n]) * Bh[b * N + n];
+      C[a * l + b] = C[b * l + a] = t;
+    }
+  std::vector<double> ev, U;
+  jacobi_eig(C, li, ev, U);
+  std::vector<uint16_t> l1(static_cast<size_t>(K) * r), l2(static_cast<size_t>(r) * N);
+  for (int64_t i = 0; i < r; ++i) {
+    const double sig = std::sqrt(std::max(ev[i], 0.0));
+    const double rs = std::sqrt(sig);
+    for (int64_t k = 0; k < K; ++k) {  // L1 = Q U_r sqrt(S)
+      double t = 0.0;
+      for (int a = 0; a < li; ++a) t += static_cast<double>(Qh[k * l + a]) * U[a * l + i];
+      l1[k * r + i] = bf16_bits_rn(t * rs);
+    }
+    for (int64_t n = 0; n < N; ++n) {  // L2 = sqrt(S) V_r^T, V = B^T U / sigma
+      double t = 0.0;
+      for (int a = 0; a < li; ++a) t += static_cast<double>(Bh[a * N + n]) * U[a * l + i];
+      l2[i * N + n] = bf16_bits_rn(sig > 0.0 ? t / rs : 0.0);
+    }
+  }
+  SVDQ_TRY(cudaMemcpyAsync(L1, l1.data(), l1.size() * 2, cudaMemcpyHostToDevice, st));
+  SVDQ_TRY(cudaMemcpyAsync(L2, l2.data(), l2.size() * 2, cudaMemcpyHostToDevice, st));
+  SVDQ_TRY(cudaStreamSynchronize(st));
+  return SVDQ_OK;
+}
+
+svdq_status svdq_prep_residual_quantize(svdq_variant variant, const void* w, const float* lambda,
+                                        const uint16_t* L1, const uint16_t* L2, int64_t K, int64_t N, int64_t r,
+                                        int tensor_scale, uint8_t* codes, void* scales, int32_t* w_scale_exp,
+                                        void* stream) {
+  if (variant != SVDQ_INT4_G64_BF16 && variant != SVDQ_NVFP4_G16_E4M3) return SVDQ_ERR_INVALID_ARG;
+  if (!w || !lambda || !codes || !scales || !w_scale_exp || (r > 0 && (!L1 || !L2))) return SVDQ_ERR_INVALID_ARG;
+  if (tensor_scale && variant != SVDQ_NVFP4_G16_E4M3) return SVDQ_ERR_INVALID_ARG;
+  const int G = group_of(variant);
+  if (K < G || K % G != 0 || K > (1 << 20) || N < 1 || N > (1 << 20)) return SVDQ_ERR_SHAPE;
+  if (r < 0 || r > 128) return SVDQ_ERR_SHAPE;
+  svdq_status s = check_device(nullptr, nullptr);
+  if (s != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int ri = static_cast<int>(r);
+  const uint16_t* wb = static_cast<const uint16_t*>(w);
+  int e = 0;
+  if (tensor_scale) {
+    DevBuf am;
+    if (!am.alloc(8)) return SVDQ_ERR_OOM;
+    SVDQ_TRY(cudaMemsetAsync(am.p, 0, 8, st));
+    prep_residual_amax_kernel<<<dim3(static_cast<unsigned>(cdiv(N, 128)), static_cast<unsigned>(cdiv(K, 16))), 128, 0, st>>>(
+        wb, lambda, L1, L2, K, N, ri, am.as<unsigned long long>());
+    SVDQ_TRY(cudaGetLastError());
+    double amax = 0.0;
+    SVDQ_TRY(cudaMemcpyAsync(&amax, am.p, 8, cudaMemcpyDeviceToHost, st));
+    SVDQ_TRY(cudaStreamSynchronize(st));
+    if (amax > 0.0) {  // smallest e with amax / 6 <= 448 * 2^e
+      int x;
+      const double m = std::frexp(amax / 6.0 / 448.0, &x);
+      e = (m == 0.5) ? x - 1 : x;
+    }
+  }
+  dim3 grid(static_cast<unsigned>(cdiv(N, 128)), static_cast<unsigned>(K / G));
+  if (variant == SVDQ_INT4_G64_BF16)
+    prep_residual_quant_kernel<0><<<grid, 128, 0, st>>>(wb, lambda, L1, L2, K, N, ri, 0, codes, scales);
+  else
+    prep_residual_quant_kernel<1><<<grid, 128, 0, st>>>(wb, lambda, L1, L2, K, N, ri, e, codes, scales);
+  SVDQ_TRY(cudaGetLastError());
+  *w_scale_exp = e;
+  return SVDQ_OK;
 }
 
 svdq_status svdq_selftest_division(int variant, unsigned long long* mismatches) {

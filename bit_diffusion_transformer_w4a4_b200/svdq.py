@@ -19,6 +19,7 @@ NVFP4 = 1
 EPI_GELU = 1
 GEMM_SINGLE_SM = 2
 INT4_F16 = 4
+EPI_QKV_NORM_ROPE = 8
 
 STATUS = {
     0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_SHAPE", 3: "SVDQ_ERR_ALIGNMENT",
@@ -32,6 +33,9 @@ EXPORTED = [
     "svdq_linear_forward_host", "svdq_device_status", "svdq_debug_set_fault",
     "svdq_selftest_division", "svdq_status_string", "svdq_version",
     "svdq_quantize_act_lowrank_down_static",
+    "svdq_awq_load", "svdq_awq_free", "svdq_awq_w4a16_forward",
+    "svdq_prep_calibrate", "svdq_prep_lowrank", "svdq_prep_residual_quantize",
+    "svdq_w4a4_gemm_lowrank_up_qkv", "svdq_linear_forward_qkv",
 ]
 
 
@@ -49,6 +53,16 @@ class WeightDesc(ctypes.Structure):
         ("flags", ctypes.c_uint32),
         ("lam", ctypes.c_void_p), ("L1", ctypes.c_void_p), ("L2", ctypes.c_void_p),
         ("w_codes", ctypes.c_void_p), ("w_scales", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+        ("w_scale_exp", ctypes.c_int32),
+        ("q_norm", ctypes.c_void_p), ("k_norm", ctypes.c_void_p), ("norm_eps", ctypes.c_float),
+    ]
+
+
+class AWQDesc(ctypes.Structure):
+    _fields_ = [
+        ("K", ctypes.c_int64), ("N", ctypes.c_int64), ("max_M", ctypes.c_int64),
+        ("a", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+        ("zeros", ctypes.c_void_p), ("bias", ctypes.c_void_p),
     ]
 
 
@@ -78,6 +92,15 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
     L.svdq_device_status.argtypes = [vp, vp]
     L.svdq_debug_set_fault.argtypes = [vp, ctypes.c_uint32, ctypes.c_uint32]
     L.svdq_selftest_division.argtypes = [ctypes.c_int, ctypes.c_void_p]
+    L.svdq_w4a4_gemm_lowrank_up_qkv.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp]
+    L.svdq_linear_forward_qkv.argtypes = [vp, vp, vp, vp, i64, vp]
+    L.svdq_awq_load.argtypes = [ctypes.POINTER(AWQDesc), ctypes.POINTER(vp), vp]
+    L.svdq_awq_free.argtypes = [vp]
+    L.svdq_awq_w4a16_forward.argtypes = [vp, vp, vp, i64, vp]
+    L.svdq_prep_calibrate.argtypes = [vp, i64, vp, i64, i64, ctypes.c_float, vp, vp]
+    L.svdq_prep_lowrank.argtypes = [vp, vp, i64, i64, i64, vp, i64, ctypes.c_int, vp, vp, vp]
+    L.svdq_prep_residual_quantize.argtypes = [st, vp, vp, vp, vp, i64, i64, i64, ctypes.c_int, vp, vp,
+                                              ctypes.POINTER(ctypes.c_int32), vp]
     L.svdq_quantize_act_lowrank_down_static.argtypes = [st, i64, i64, vp, vp, vp, i64, vp, vp, vp, vp, vp]
     L.svdq_status_string.argtypes = [st]
     L.svdq_status_string.restype = ctypes.c_char_p
@@ -124,12 +147,13 @@ class SVDQWeights:
     """A loaded layer: owns a library handle (``svdq_weights_t``)."""
 
     def __init__(self, pw, max_M: int, stream=None, single_sm: bool = False,
-                 int4_f16: bool = False):
+                 int4_f16: bool = False, qkv_norm=None):
         """``pw`` has fields variant, K, N, r, lam, L1, L2, codes, scales, bias, gelu
         (host numpy arrays in the formats of ``svdq_weight_desc``).  ``single_sm``
         sets SVDQ_GEMM_SINGLE_SM (NVFP4 GEMM on single SMs; by default it runs on
         pairs of SMs when M > 128).  ``int4_f16`` sets SVDQ_INT4_F16 (INT4 GEMM as
-        one fp16 GEMM of the exactly dequantised operands)."""
+        one fp16 GEMM of the exactly dequantised operands).  ``qkv_norm`` =
+        (q_norm bf16 [128], k_norm bf16 [128], eps) sets SVDQ_EPI_QKV_NORM_ROPE."""
         self._keep = [np.ascontiguousarray(pw.lam, dtype=np.float32),
                       np.ascontiguousarray(pw.L1, dtype=np.uint16),
                       np.ascontiguousarray(pw.L2, dtype=np.uint16),
@@ -137,14 +161,23 @@ class SVDQWeights:
                       np.ascontiguousarray(pw.scales),
                       None if pw.bias is None else np.ascontiguousarray(pw.bias, dtype=np.uint16)]
         lam, L1, L2, codes, scales, bias = self._keep
+        qn = kn = None
+        eps = 0.0
+        if qkv_norm is not None:
+            qn = np.ascontiguousarray(qkv_norm[0], dtype=np.uint16)
+            kn = np.ascontiguousarray(qkv_norm[1], dtype=np.uint16)
+            eps = float(qkv_norm[2])
+            self._keep += [qn, kn]
+        self.qkv = qkv_norm is not None
         self.variant, self.K, self.N, self.r = int(pw.variant), int(pw.K), int(pw.N), int(pw.r)
         self.max_M = int(max_M)
         self.gelu = bool(pw.gelu)
         d = WeightDesc(self.variant, self.K, self.N, self.r, self.max_M,
                        (EPI_GELU if self.gelu else 0) | (GEMM_SINGLE_SM if single_sm else 0)
-                       | (INT4_F16 if int4_f16 else 0),
+                       | (INT4_F16 if int4_f16 else 0) | (EPI_QKV_NORM_ROPE if self.qkv else 0),
                        _ptr(lam), _ptr(L1) if self.r else 0, _ptr(L2) if self.r else 0,
-                       _ptr(codes), _ptr(scales), _ptr(bias))
+                       _ptr(codes), _ptr(scales), _ptr(bias), int(getattr(pw, "w_scale_exp", 0)),
+                       _ptr(qn), _ptr(kn), eps)
         h = ctypes.c_void_p(0)
         self._lib = lib()
         _check(self._lib.svdq_weights_load(ctypes.byref(d), ctypes.byref(h), _stream(stream)),
@@ -170,6 +203,15 @@ class SVDQWeights:
         _check(self._lib.svdq_w4a4_gemm_lowrank_up(
             self.handle, _ptr(act_codes), _ptr(act_scales), _ptr(t), int(M), _ptr(y),
             _stream(stream)), "svdq_w4a4_gemm_lowrank_up")
+
+    def w4a4_gemm_lowrank_up_qkv(self, act_codes, act_scales, t, M, rope, y, stream=None):
+        _check(self._lib.svdq_w4a4_gemm_lowrank_up_qkv(
+            self.handle, _ptr(act_codes), _ptr(act_scales), _ptr(t), int(M), _ptr(rope), _ptr(y),
+            _stream(stream)), "svdq_w4a4_gemm_lowrank_up_qkv")
+
+    def linear_forward_qkv(self, x, rope, y, M, stream=None):
+        _check(self._lib.svdq_linear_forward_qkv(self.handle, _ptr(x), _ptr(rope), _ptr(y), int(M),
+                                                 _stream(stream)), "svdq_linear_forward_qkv")
 
     def linear_forward(self, x, y, M, stream=None):
         _check(self._lib.svdq_linear_forward(self.handle, _ptr(x), _ptr(y), int(M), _stream(stream)),
@@ -204,6 +246,71 @@ class SVDQWeights:
             self.close()
         except Exception:
             pass
+
+
+class AWQWeights:
+    """A loaded AWQ W4A16 layer: owns a library handle (``svdq_awq_t``)."""
+
+    def __init__(self, p, max_M: int, stream=None):
+        """``p`` has fields K, N, a, codes, scales, zeros, bias (host numpy
+        arrays in the formats of ``svdq_awq_desc``)."""
+        self._keep = [np.ascontiguousarray(p.a, dtype=np.float32),
+                      np.ascontiguousarray(p.codes, dtype=np.uint8),
+                      np.ascontiguousarray(p.scales, dtype=np.uint16),
+                      np.ascontiguousarray(p.zeros, dtype=np.uint8),
+                      None if p.bias is None else np.ascontiguousarray(p.bias, dtype=np.uint16)]
+        a, codes, scales, zeros, bias = self._keep
+        self.K, self.N, self.max_M = int(p.K), int(p.N), int(max_M)
+        d = AWQDesc(self.K, self.N, self.max_M, _ptr(a), _ptr(codes), _ptr(scales), _ptr(zeros),
+                    _ptr(bias))
+        h = ctypes.c_void_p(0)
+        self._lib = lib()
+        _check(self._lib.svdq_awq_load(ctypes.byref(d), ctypes.byref(h), _stream(stream)), "svdq_awq_load")
+        self.handle = h
+
+    def forward(self, x, y, M, stream=None):
+        _check(self._lib.svdq_awq_w4a16_forward(self.handle, _ptr(x), _ptr(y), int(M), _stream(stream)),
+               "svdq_awq_w4a16_forward")
+
+    def close(self) -> None:
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            self._lib.svdq_awq_free(self.handle)
+            self.handle = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ------------------------------------------------------------- weight prep
+def prep_calibrate(x, M, w, K, N, lam, alpha=0.5, stream=None):
+    """lambda (fp32 [K], written) from calibration activations x (bf16
+    [M x K]) and the weight w (bf16 [K x N]), all device tensors."""
+    _check(lib().svdq_prep_calibrate(_ptr(x), int(M), _ptr(w), int(K), int(N), float(alpha), _ptr(lam),
+                                     _stream(stream)), "svdq_prep_calibrate")
+
+
+def prep_lowrank(w, lam, K, N, r, omega, l, power_iters, L1, L2, stream=None):
+    """Rank-r bf16 factors L1 [K x r], L2 [r x N] (written) of diag(lam) w by
+    a randomized SVD with the caller's Gaussian test matrix omega (fp32
+    [N x l])."""
+    _check(lib().svdq_prep_lowrank(_ptr(w), _ptr(lam), int(K), int(N), int(r), _ptr(omega), int(l),
+                                   int(power_iters), _ptr(L1), _ptr(L2), _stream(stream)), "svdq_prep_lowrank")
+
+
+def prep_residual_quantize(variant, w, lam, L1, L2, K, N, r, codes, scales, tensor_scale=False,
+                           stream=None) -> int:
+    """Codes [N x K/2] and scales [N x K/G] (written) of the residual
+    diag(lam) w - L1 L2; returns the per-tensor scale exponent (0 without
+    tensor_scale)."""
+    e = ctypes.c_int32(0)
+    _check(lib().svdq_prep_residual_quantize(int(variant), _ptr(w), _ptr(lam), _ptr(L1), _ptr(L2), int(K),
+                                             int(N), int(r), int(bool(tensor_scale)), _ptr(codes),
+                                             _ptr(scales), ctypes.byref(e), _stream(stream)),
+           "svdq_prep_residual_quantize")
+    return int(e.value)
 
 
 def untile_nvfp4_scales(buf: np.ndarray, M: int, K: int) -> np.ndarray:

@@ -171,6 +171,7 @@ class PackedWeights:
     bias: np.ndarray | None = None
     gelu: bool = False
     meta: dict = field(default_factory=dict)
+    w_scale_exp: int = 0        # NVFP4 per-tensor scale 2^e of the residual weights
 
 
 def synthetic_packed(layer: Layer, seed: int = 0, int4_min: int = -7) -> PackedWeights:
@@ -203,3 +204,74 @@ def synthetic_packed(layer: Layer, seed: int = 0, int4_min: int = -7) -> PackedW
     codes = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
     return PackedWeights(layer.variant, K, N, r, lam, L1, L2, codes, scales,
                          bias(layer, seed), layer.gelu, {"source": "synthetic"})
+
+
+# ------------------------------------------------------------ AWQ W4A16 layers
+@dataclass(frozen=True)
+class AWQLayer:
+    """A W4A16 modulation linear: x[M,K] @ W[K,N] with M = tokens per call
+    (one conditioning vector per image: the batch)."""
+    name: str
+    M: int
+    K: int
+    N: int
+    bias: bool = True
+    config_id: int = 90
+    layer_id: int = 0
+
+    def flops(self) -> int:
+        return 2 * self.M * self.K * self.N
+
+    def weight_bytes(self) -> int:
+        """Bytes of the packed weights: codes, bf16 scales and u8 zeros."""
+        return self.N * self.K // 2 + self.N * (self.K // 64) * 3
+
+
+def awq_workloads() -> dict[str, AWQLayer]:
+    """DiT adaLN modulation (hidden 3072 -> 6 x 3072) at batch 1, 2 (CFG) and 4."""
+    return {f"awq_mod_m{m}": AWQLayer(f"mod_m{m}", M=m, K=3072, N=18432, layer_id=m) for m in (1, 2, 4)}
+
+
+def awq_activations(layer: AWQLayer, seed: int = 0) -> np.ndarray:
+    """x [M,K] bf16 bits ~N(0,1) (a SiLU'd conditioning embedding's scale)."""
+    g = _rng(seed, layer.config_id, 10 * layer.layer_id + 1)
+    return to_bf16_bits(g.standard_normal((layer.M, layer.K), dtype=np.float32))
+
+
+def awq_weight(layer: AWQLayer, seed: int = 0) -> np.ndarray:
+    """W [K,N] fp32 on the bf16 grid ~N(0, 0.02^2)."""
+    g = _rng(seed, layer.config_id, 10 * layer.layer_id + 2)
+    w = g.standard_normal((layer.K, layer.N), dtype=np.float32) * np.float32(0.02)
+    return bf16_bits_to_f32(to_bf16_bits(w))
+
+
+@dataclass
+class PackedAWQ:
+    """AWQ W4A16 load format (host arrays): a fp32 [K]; codes u8 [N, K/2]
+    (element 2j low nibble, 0..15); scales bf16 bits [N, K/64]; zeros u8
+    [N, K/64] (0..15); bias bf16 bits [N] or None."""
+    K: int
+    N: int
+    a: np.ndarray
+    codes: np.ndarray
+    scales: np.ndarray
+    zeros: np.ndarray
+    bias: np.ndarray | None = None
+
+
+def synthetic_awq(layer: AWQLayer, seed: int = 0) -> PackedAWQ:
+    """Random AWQ-packed weights for timing runs, sampled as raw bit patterns:
+    codes 0..15 bell-shaped around the zero point, zero points 6..9, bf16
+    scales in a band around 0.005, log-normal channel factors."""
+    K, N = layer.K, layer.N
+    g = _rng(seed, layer.config_id, 10 * layer.layer_id + 7)
+    a = np.exp(g.normal(0.0, 0.3, K)).astype(np.float32)
+    zeros = g.integers(6, 10, (N, K // 64)).astype(np.uint8)
+    q = np.clip(np.rint(g.normal(0.0, 3.0, (N, K)) + np.repeat(zeros, 64, axis=1)), 0, 15).astype(np.uint8)
+    codes = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
+    scales = to_bf16_bits(np.exp(g.normal(np.log(0.005), 0.3, (N, K // 64))).astype(np.float32))
+    b = None
+    if layer.bias:
+        b = to_bf16_bits(_rng(seed, layer.config_id, 10 * layer.layer_id + 3)
+                         .standard_normal(N, dtype=np.float32) * np.float32(0.1))
+    return PackedAWQ(K, N, a, codes, scales, zeros, b)

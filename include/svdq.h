@@ -88,6 +88,18 @@ typedef enum {
  * which an activation scale exceeded 9357 (7 s > 65504).  Activation scales
  * below 2^-17 lose low bits of s q (absolute error below 2^-25 s). */
 #define SVDQ_INT4_F16 4u
+/* NVFP4 only, not with SVDQ_EPI_GELU: the layer is a merged QKV projection
+ * whose N = 3 H 128 output columns are [Q | K | V] (heads of 128 features);
+ * the GEMM epilogue RMS-normalises every head of Q and of K,
+ *   v <- v / sqrt(mean_head(v^2) + norm_eps) * g   (g = q_norm or k_norm),
+ * and rotates its interleaved pairs (2i, 2i+1) by the token's rotary angle
+ * for pair i: (a, b) <- (a cos - b sin, a sin + b cos).  V is stored as is.
+ * Defined by "Nunchaku Lite ..." (axbrief.com), section "The Trade-off
+ * Between Fused Kernels and Generality": QKV projection, Q/K normalisation
+ * and rotary embeddings bundled into one kernel over a merged to_qkv module.
+ * Such a layer runs through svdq_linear_forward_qkv /
+ * svdq_w4a4_gemm_lowrank_up_qkv only.  N % 384 == 0. */
+#define SVDQ_EPI_QKV_NORM_ROPE 8u
 
 typedef struct svdq_weights* svdq_weights_t;   /* opaque, library-owned */
 
@@ -101,6 +113,12 @@ typedef struct svdq_weights* svdq_weights_t;   /* opaque, library-owned */
  *   w_codes  u8   [N x K/2]  residual codes, one row per output feature
  *   w_scales INT4: bf16 [N x K/64]; NVFP4: E4M3 bytes [N x K/16]
  *   bias     bf16 [N] or NULL
+ *   w_scale_exp  NVFP4 only: per-tensor second-level scale 2^w_scale_exp of
+ *            the residual weights (a weight is code * E4M3 scale *
+ *            2^w_scale_exp); 0 = none.  |w_scale_exp| <= 100, else
+ *            SVDQ_ERR_INVALID_ARG (also for INT4 with a nonzero value).
+ *            The GEMM multiplies its accumulator by 2^e and T by 2^-e, both
+ *            exact, so y is the same function of the dequantised weights.
  * L1 / L2 may be NULL when r == 0.
  */
 typedef struct {
@@ -113,6 +131,12 @@ typedef struct {
   const uint8_t* w_codes;
   const void* w_scales;
   const uint16_t* bias;
+  int32_t w_scale_exp;
+  /* SVDQ_EPI_QKV_NORM_ROPE only (else ignored): host bf16 [128] RMS-norm
+   * weights of the Q and K heads and the epsilon (0 < norm_eps < 1) */
+  const uint16_t* q_norm;
+  const uint16_t* k_norm;
+  float norm_eps;
 } svdq_weight_desc;
 
 /*
@@ -202,6 +226,22 @@ svdq_status svdq_linear_forward(svdq_weights_t h, const void* x, void* y, int64_
                                 void* stream);
 
 /*
+ * Defined by: the fused path of "Nunchaku Lite ..." (axbrief.com), section
+ * "The Trade-off Between Fused Kernels and Generality" (see
+ * SVDQ_EPI_QKV_NORM_ROPE).  Kernel 2 / the whole layer for a handle loaded
+ * with SVDQ_EPI_QKV_NORM_ROPE:
+ *   rope  device fp32 [M x 64 x 2], 16-byte aligned: (cos, sin) of the
+ *         rotary angle of token m for pair i at rope[(m * 64 + i) * 2]
+ * Other arguments as svdq_w4a4_gemm_lowrank_up / svdq_linear_forward.  The
+ * table is read while the kernel runs (it must stay valid until then).
+ */
+svdq_status svdq_w4a4_gemm_lowrank_up_qkv(svdq_weights_t h, const uint8_t* act_codes,
+                                          const void* act_scales, const float* t, int64_t M,
+                                          const float* rope, void* y, void* stream);
+svdq_status svdq_linear_forward_qkv(svdq_weights_t h, const void* x, const float* rope, void* y,
+                                    int64_t M, void* stream);
+
+/*
  * Defined by: the same layer as svdq_linear_forward.
  * Same as svdq_linear_forward with HOST input and output (pinned memory is
  * recommended): copies x_host to the device, runs the layer and copies y back
@@ -245,6 +285,101 @@ svdq_status svdq_quantize_act_lowrank_down_static(svdq_variant variant, int64_t 
                                                   const void* x, int64_t M, uint8_t* act_codes,
                                                   void* act_scales, float* t, int* device_error,
                                                   void* stream);
+
+/* ------------------------------------------------------------------------
+ * AWQ W4A16 linear layer: 4-bit weights, 16-bit activations.
+ *
+ * Defined by: "Nunchaku Lite ..." (axbrief.com), section "The Mechanics of
+ * 4-Bit Efficiency and SVDQuant" -- besides SVDQW4A4Linear the runtime
+ * patching installs AWQW4A16Linear layers (4-bit weights, 16-bit
+ * activations); section "The Trade-off Between Fused Kernels and
+ * Generality" -- the scanner assigns AWQ W4A16 to modulation linear layers.
+ * The pages give no arithmetic; the library computes (readings: activation-
+ * aware channel factors a, groups of 64 along K, asymmetric unsigned codes
+ * with an integer zero point):
+ *   x' = fp32(x) * fp32(1/a_k)                       (kept in fp32)
+ *   y[m,n] = sum_g s[n,g] sum_{k in g} x'[m,k] (q[n,k] - z[n,g])  (+ bias)
+ * accumulated in fp32 and rounded once to bf16.  Modulation layers see one
+ * token per image, so the call is a matrix-vector product bound by reading
+ * the 4-bit weights; it runs on the CUDA cores.
+ */
+typedef struct svdq_awq* svdq_awq_t;   /* opaque, library-owned */
+
+/* HOST memory, read only during svdq_awq_load:
+ *   a       fp32 [K]        activation-aware channel factors (> 0)
+ *   codes   u8   [N x K/2]  codes 0..15, element 2j in the low nibble
+ *   scales  bf16 [N x K/64] group scales s
+ *   zeros   u8   [N x K/64] integer zero points 0..15 (else INVALID_ARG)
+ *   bias    bf16 [N] or NULL
+ * Shapes: K % 64 == 0, 64 <= K <= 32768, 1 <= N, 1 <= M <= max_M. */
+typedef struct {
+  int64_t K, N, max_M;
+  const float* a;
+  const uint8_t* codes;
+  const uint16_t* scales;
+  const uint8_t* zeros;
+  const uint16_t* bias;
+} svdq_awq_desc;
+
+/* Copy the weights into library-owned device memory on the current device
+ * (1/a is computed once, by IEEE fp32 division).  On error *out is NULL. */
+svdq_status svdq_awq_load(const svdq_awq_desc* desc, svdq_awq_t* out, void* stream);
+
+/* Free a handle (NULL is a no-op).  Synchronises the device first. */
+svdq_status svdq_awq_free(svdq_awq_t h);
+
+/* y = layer(x): x bf16 [M x K] (4-byte aligned), y bf16 [M x N] (2-byte
+ * aligned), device memory owned by the caller; asynchronous on `stream`,
+ * launched as a programmatic dependent of the previous kernel (it waits for
+ * that kernel before reading x). */
+svdq_status svdq_awq_w4a16_forward(svdq_awq_t h, const void* x, void* y, int64_t M, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Weight preparation on the GPU (offline compression; not on the layer's
+ * timed path: these calls allocate scratch, copy small results to the host
+ * and synchronise `stream` before returning).
+ *
+ * Defined by: "Nunchaku Lite ..." (axbrief.com), section "Hardware
+ * Specialization and the Compression Workflow" -- inspect, calibrate the
+ * data distribution to find outliers, quantize the weights, package, at INT4
+ * or NVFP4 precision; section "The Mechanics of 4-Bit Efficiency and
+ * SVDQuant" -- activation outliers shifted into the weights, the weights
+ * split into a 16-bit low-rank branch and a 4-bit residual; "Problemas do
+ * Nunchaku Qwen ..." (apatero.com), section "O que e Nunchaku ..." -- the
+ * low-rank branch from a singular value decomposition.  The outputs are the
+ * inputs of svdq_weights_load.  All pointers are device memory unless named
+ * otherwise.
+ */
+
+/* Calibration and smoothing factors: lambda_k = max_m|x[m,k]|^alpha /
+ * max_n|w[k,n]|^(1-alpha) (fp64, then fp32), 1 where either maximum is 0,
+ * clamped to [2^-20, 2^20].  x bf16 [M x K] calibration activations, w bf16
+ * [K x N] the layer's weight, lambda fp32 [K] (written). */
+svdq_status svdq_prep_calibrate(const void* x, int64_t M, const void* w, int64_t K, int64_t N,
+                                float alpha, float* lambda, void* stream);
+
+/* Rank-r factors of W_hat = diag(lambda) w by a randomized SVD: the range
+ * of W_hat Omega (omega fp32 [N x l], the caller's Gaussian test matrix,
+ * r <= l <= 64, l <= min(K, N)) refined by `power_iters` power iterations
+ * with re-orthonormalisation (Cholesky QR twice, fp64 Gram matrices), then
+ * the small SVD of Q^T W_hat on the host in fp64.  The singular values are
+ * split evenly: L1 = Q U_r S_r^(1/2) bf16 [K x r], L2 = S_r^(1/2) V_r^T bf16
+ * [r x N] (round to nearest even).  The products with W_hat run in fp32. */
+svdq_status svdq_prep_lowrank(const void* w, const float* lambda, int64_t K, int64_t N, int64_t r,
+                              const float* omega, int64_t l, int power_iters, uint16_t* L1,
+                              uint16_t* L2, void* stream);
+
+/* Residual R = diag(lambda) w - L1 L2 (fp64) quantised per output feature n
+ * in groups of G along K: INT4 s = bf16(amax / 7), q = clamp(rint(R / s),
+ * -8, 7); NVFP4 s = E4M3(amax / 6 / 2^e) (satfinite), q = E2M1(R / (s 2^e)).
+ * With tensor_scale (NVFP4 only) e is the smallest integer with
+ * max|R| / 6 <= 448 * 2^e, else 0; *w_scale_exp (HOST int) receives e.
+ * codes u8 [N x K/2] (element 2j low nibble), scales [N x K/G] (bf16 bits or
+ * E4M3 bytes), written.  r may be 0 (L1, L2 unused). */
+svdq_status svdq_prep_residual_quantize(svdq_variant variant, const void* w, const float* lambda,
+                                        const uint16_t* L1, const uint16_t* L2, int64_t K, int64_t N,
+                                        int64_t r, int tensor_scale, uint8_t* codes, void* scales,
+                                        int32_t* w_scale_exp, void* stream);
 
 /*
  * Failure reporting (no counterpart on the pages).

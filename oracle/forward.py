@@ -21,6 +21,7 @@ pages say nothing:
       NVFP4 q = E2M1_RN_satfinite(v);  s == 0 gives q = +0
   s5  T = X' L1, summed exactly (fp64), stored fp32
   s6  acc = sum_g s_x s_w sum_{k in g} q_x q_w  +  T L2  (+ bias)   (fp64)
+      (an NVFP4 weight with a per-tensor scale 2^e has s_w = E4M3 scale * 2^e)
   s7  y = GELU_tanh(acc) when the layer has GELU;  Y = bf16_RN(y)
 
 Parity: pinned by brute force on 8x8 problems, by the exact-reconstruction
@@ -73,8 +74,8 @@ def quantize_groups(xp: np.ndarray, variant: int):
     return nib.reshape(rows, K).astype(np.uint8), s_store
 
 
-def dequantize(nib: np.ndarray, scales: np.ndarray, variant: int) -> np.ndarray:
-    """nibbles [rows,K] + scales -> exact fp64 values q*s."""
+def dequantize(nib: np.ndarray, scales: np.ndarray, variant: int, scale_exp: int = 0) -> np.ndarray:
+    """nibbles [rows,K] + scales (times 2^scale_exp) -> exact fp64 values q*s."""
     G = GROUP[variant]
     rows, K = nib.shape
     if variant == INT4:
@@ -82,7 +83,7 @@ def dequantize(nib: np.ndarray, scales: np.ndarray, variant: int) -> np.ndarray:
         s = F.bf16_from_bits(scales)
     else:
         q = F.e2m1_decode(nib)
-        s = F.e4m3_decode(scales)
+        s = np.ldexp(F.e4m3_decode(scales), scale_exp)
     return (q.reshape(rows, K // G, G) * s[:, :, None]).reshape(rows, K)
 
 
@@ -108,7 +109,7 @@ def gelu_tanh(x):
 
 
 def gemm_lowrank_up(codes, scales, T, w_codes, w_scales, L2_bits, variant,
-                    bias_bits=None, gelu=False, rows=None):
+                    bias_bits=None, gelu=False, rows=None, w_scale_exp: int = 0):
     """Weight side (steps s6-s7).
 
     codes [M,K/2], scales (activation), T fp32 [M,r]; w_codes [N,K/2],
@@ -118,7 +119,7 @@ def gemm_lowrank_up(codes, scales, T, w_codes, w_scales, L2_bits, variant,
     if rows is not None:
         codes, scales, T = codes[rows], scales[rows], T[rows]
     xa = dequantize(F.unpack_nibbles(codes), scales, variant)
-    wq = dequantize(F.unpack_nibbles(w_codes), w_scales, variant)
+    wq = dequantize(F.unpack_nibbles(w_codes), w_scales, variant, w_scale_exp)
     acc = xa @ wq.T
     L2 = F.bf16_from_bits(L2_bits)
     if L2.shape[0] > 0:
@@ -140,7 +141,7 @@ def linear_forward(x_bits, pw, rows=None):
         x_bits = x_bits[rows]
     codes, scales, T = quantize_act_lowrank_down(x_bits, inv_lam, pw.L1, pw.variant)
     y, Y = gemm_lowrank_up(codes, scales, T, pw.codes, pw.scales, pw.L2, pw.variant,
-                           pw.bias, pw.gelu)
+                           pw.bias, pw.gelu, w_scale_exp=getattr(pw, "w_scale_exp", 0))
     return {"codes": codes, "scales": scales, "T": T, "y": y, "Y": Y}
 
 

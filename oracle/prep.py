@@ -19,6 +19,14 @@ quantize -> package; INT4 or NVFP4 precision.
   c6  per output column n, groups of G along K: s = amax/7 -> bf16 (INT4) or
       amax/6 -> E4M3 (NVFP4), codes = round(R/s) in fp64 (same rule as the
       runtime activation quantiser, in fp64)
+  c7  NVFP4 with a per-tensor second-level scale (optional): a power of two
+      2^e with e the smallest integer such that max|R| / 6 <= 448 * 2^e (e = 0
+      when R = 0); group scales s = E4M3_RN_satfinite((amax / 6) * 2^-e), codes
+      = E2M1_RN_satfinite(R / (s 2^e)); a weight dequantises to q s 2^e.
+      Reading: the pages name NVFP4 but not its second level; the format's own
+      tensor scale is an fp32 value, taken here as a power of two so that the
+      scaling stays exact through the low-rank branch (the GEMM scales its
+      accumulator by 2^e and the low-rank operand T by 2^-e).
 
 Parity: smoothing invariance, the Eckart-Young residual norm and exact
 reconstruction at r = min(K, N) are pinned in tests/test_oracle_pins.py.
@@ -51,18 +59,31 @@ def svd_factors(w_hat: np.ndarray, r: int):
     return U[:, :r] * rs[None, :], rs[:, None] * Vt[:r, :], S
 
 
-def quantize_weight_groups(Rt: np.ndarray, variant: int):
-    """c6 on R^T [N,K] (fp64): returns (nibbles [N,K], scales)."""
+def tensor_scale_exponent(R: np.ndarray) -> int:
+    """c7: the smallest integer e with max|R| / 6 <= 448 * 2^e (0 for R = 0)."""
+    amax = float(np.max(np.abs(R))) if R.size else 0.0
+    if amax == 0.0:
+        return 0
+    t = amax / 6.0 / 448.0
+    m, x = np.frexp(t)                       # t = m 2^x, 0.5 <= m < 1
+    return int(x - 1) if m == 0.5 else int(x)
+
+
+def quantize_weight_groups(Rt: np.ndarray, variant: int, scale_exp: int = 0):
+    """c6 (and c7 when scale_exp != 0) on R^T [N,K] (fp64): returns
+    (nibbles [N,K], scales)."""
     G = GROUP[variant]
     N, K = Rt.shape
     g = Rt.reshape(N, K // G, G)
     a = np.max(np.abs(g), axis=2)
     if variant == INT4:
+        assert scale_exp == 0, "the per-tensor scale is an NVFP4 option"
         s = F.bf16_round(a / 7.0)
         s_store = F.bf16_bits(s)
     else:
-        s = F.e4m3_round(a / 6.0)
+        s = F.e4m3_round(np.ldexp(a / 6.0, -scale_exp))
         s_store = F.e4m3_encode(s)
+        s = np.ldexp(s, scale_exp)               # the group's full scale s 2^e
     nz = s > 0
     with np.errstate(divide="ignore", invalid="ignore"):
         v = np.where(nz[:, :, None], g / np.where(nz, s, 1.0)[:, :, None], 0.0)
@@ -79,8 +100,10 @@ class Prepared:
 
 
 def prepare(x_bits: np.ndarray, w: np.ndarray, r: int, variant: int,
-            alpha: float = 0.5, bias_bits=None, gelu: bool = False) -> Prepared:
-    """c2-c6 for weight W [K,N] (fp64 values) calibrated on X (bf16 bits)."""
+            alpha: float = 0.5, bias_bits=None, gelu: bool = False,
+            tensor_scale: bool = False) -> Prepared:
+    """c2-c6 (c7 with ``tensor_scale``, NVFP4 only) for weight W [K,N] (fp64
+    values) calibrated on X (bf16 bits)."""
     x = F.bf16_from_bits(x_bits)
     w = np.asarray(w, dtype=np.float64)
     K, N = w.shape
@@ -95,7 +118,8 @@ def prepare(x_bits: np.ndarray, w: np.ndarray, r: int, variant: int,
         L1b = np.zeros((K, 0), dtype=np.uint16)
         L2b = np.zeros((0, N), dtype=np.uint16)
         R = w_hat
-    nib, scales = quantize_weight_groups(R.T.copy(), variant)
+    e = tensor_scale_exponent(R) if tensor_scale else 0
+    nib, scales = quantize_weight_groups(R.T.copy(), variant, e)
     return Prepared(variant=variant, K=K, N=N, r=r, lam=lam, L1=L1b, L2=L2b,
                     codes=F.pack_nibbles(nib), scales=scales, bias=bias_bits,
-                    gelu=gelu, R=R, S=S, w_hat=w_hat)
+                    gelu=gelu, R=R, S=S, w_hat=w_hat, w_scale_exp=e)

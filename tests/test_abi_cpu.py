@@ -94,3 +94,47 @@ def test_no_gpu_no_fallback():
     assert L.svdq_weights_load(ctypes.byref(d), ctypes.byref(h), None) == 4
     n = (ctypes.c_ulonglong * 2)()
     assert L.svdq_selftest_division(1, n) == 4
+
+
+def _awq_desc(**kw):
+    lay = W.AWQLayer("t", M=2, K=128, N=16, config_id=93)
+    p = W.synthetic_awq(lay)
+    zeros = kw.get("zeros", p.zeros)
+    keep = [p.a, p.codes, p.scales, zeros]
+    d = svdq.AWQDesc(kw.get("K", 128), kw.get("N", 16), kw.get("max_M", 2),
+                     p.a.ctypes.data, p.codes.ctypes.data, p.scales.ctypes.data, zeros.ctypes.data, 0)
+    return d, keep
+
+
+@pytest.mark.parametrize("kw,code", [
+    ({"K": 96}, 2), ({"K": 0}, 2), ({"N": 0}, 2), ({"max_M": 0}, 2),
+    ({"zeros": np.full((16, 2), 16, np.uint8)}, 1),
+])
+def test_awq_load_validation(kw, code):
+    """Host-side validation of svdq_awq_load runs before any device work."""
+    L = svdq.lib()
+    d, keep = _awq_desc(**kw)
+    h = ctypes.c_void_p(0)
+    assert L.svdq_awq_load(ctypes.byref(d), ctypes.byref(h), None) == code
+    assert not h.value
+    assert L.svdq_awq_free(None) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    ({"variant": 0, "flags": 8}, 1),           # QKV epilogue: NVFP4 only
+    ({"variant": 1, "flags": 8 | 1}, 1),       # not with GELU
+    ({"variant": 1, "flags": 8, "N": 256}, 2),  # N must be a multiple of 3 x 128
+])
+def test_qkv_flag_validation(kw, code):
+    L = svdq.lib()
+    variant = kw["variant"]
+    N = kw.get("N", 384)
+    lay = W.Layer("t", M=64, K=256, N=N, r=16, variant=variant, config_id=9)
+    pw = W.synthetic_packed(lay)
+    g = np.full(128, 0x3F80, np.uint16)
+    d = svdq.WeightDesc(variant, 256, N, 16, 64, kw["flags"], pw.lam.ctypes.data, pw.L1.ctypes.data,
+                        pw.L2.ctypes.data, pw.codes.ctypes.data, pw.scales.ctypes.data, 0, 0,
+                        g.ctypes.data, g.ctypes.data, 1e-6)
+    h = ctypes.c_void_p(0)
+    assert L.svdq_weights_load(ctypes.byref(d), ctypes.byref(h), None) == code
+    assert not h.value

@@ -241,3 +241,20 @@ def test_int4_weight_code_minus8(opts):
     PT.check_act(got, ref, r=r, label="int4 -8")
     PT.check_y(got["Y"], ref["y"], ref["Y"], label=f"int4 -8 {opts}")
     h.close()
+
+
+@pytest.mark.parametrize("opts", [{}, {"single_sm": True}], ids=["nvfp4-pair", "nvfp4-1sm"])
+@pytest.mark.parametrize("M,K,N,r", [(300, 512, 448, 32), (129, 1024, 272, 0)])
+def test_nvfp4_tensor_scale(opts, M, K, N, r):
+    """NVFP4 weights with a per-tensor second-level scale 2^e (e < 0 for these
+    residuals): the GEMM scales its accumulator by 2^e and T by 2^-e; Y within
+    the bars of the oracle, whose weights dequantise to q s 2^e."""
+    lay, x, _ = _prepped(M, K, N, r, NVFP4, gelu=True, with_bias=True, cid=68)
+    pw = P.prepare(x, W.weight(lay), r, NVFP4, bias_bits=W.bias(lay), gelu=True, tensor_scale=True)
+    assert pw.w_scale_exp < 0
+    h = svdq.SVDQWeights(pw, M, **opts)
+    got = PT.gpu_forward(h, x, M)
+    ref = O.linear_forward(x, pw)
+    PT.check_act(got, ref, r=r, label="tensor scale")
+    PT.check_y(got["Y"], ref["y"], ref["Y"], label=f"tensor scale e{pw.w_scale_exp} {opts}")
+    h.close()

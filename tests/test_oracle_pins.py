@@ -222,11 +222,12 @@ def _brute_layer(x, inv_lam, L1, L2, wq, ws, variant, gelu, bias=None):
     return qx, sx, T, y
 
 
-@pytest.mark.parametrize("variant", [INT4, NVFP4])
+@pytest.mark.parametrize("variant,scale_exp", [(INT4, 0), (NVFP4, 0), (NVFP4, -7)])
 @pytest.mark.parametrize("gelu,with_bias", [(False, False), (True, False), (False, True),
                                             (True, True)])
-def test_brute_force_8x8(variant, gelu, with_bias):
-    g = np.random.default_rng(10 + variant + 2 * gelu + 4 * with_bias)
+def test_brute_force_8x8(variant, scale_exp, gelu, with_bias):
+    """scale_exp: the NVFP4 weights' per-tensor scale 2^e (weights q s 2^e)."""
+    g = np.random.default_rng(10 + variant + 2 * gelu + 4 * with_bias - scale_exp)
     G = O.GROUP[variant]
     M = N = 8
     K, r = G, 3
@@ -253,7 +254,8 @@ def test_brute_force_8x8(variant, gelu, with_bias):
     bias_bits = F.bf16_bits(g.standard_normal(N) * 2.0) if with_bias else None
     codes, scales, T = O.quantize_act_lowrank_down(x_bits, inv_lam, L1b, variant)
     y, Y = O.gemm_lowrank_up(codes, scales, T, F.pack_nibbles(wq_nib), ws, L2b, variant,
-                             bias_bits=bias_bits, gelu=gelu)
+                             bias_bits=bias_bits, gelu=gelu, w_scale_exp=scale_exp)
+    wsv = wsv * 2.0 ** scale_exp
 
     fr = lambda a: [[Fraction(float(v)) for v in row] for row in a]
     qx, sx, Tb, yb = _brute_layer(
@@ -375,3 +377,45 @@ def test_prepare_full_rank_reconstructs_xw(K, N, variant):
     out = O.linear_forward(x_bits, pw)
     e = np.linalg.norm(out["y"] - ref) / np.linalg.norm(ref)
     assert e < 1e-2, e
+
+
+# --------------------------------------- NVFP4 per-tensor second-level scale
+def test_tensor_scale_exponent():
+    """e is the smallest integer with max|R| / 6 <= 448 * 2^e."""
+    assert P.tensor_scale_exponent(np.zeros((4, 4))) == 0
+    for e in (-20, -10, -1, 0, 3):
+        R = np.full((2, 2), 2688.0 * 2.0 ** e)          # max|R| / 6 = 448 * 2^e exactly
+        assert P.tensor_scale_exponent(R) == e
+        R[0, 0] = np.nextafter(R[0, 0], np.inf)          # just above: one more
+        assert P.tensor_scale_exponent(R) == e + 1
+        R = -np.full((3,), 2688.0 * 2.0 ** e * 0.75)     # sign does not matter
+        assert P.tensor_scale_exponent(R) == e
+
+
+def test_tensor_scale_quantisation():
+    """With the per-tensor scale a small residual keeps normal E4M3 group
+    scales (no zero or subnormal scales where global scale 1 has many), no
+    scale saturates, and each group obeys the E2M1 rounding bound; e = 0
+    reproduces the plain quantiser bit for bit."""
+    g = np.random.default_rng(31)
+    N, K = 64, 256
+    Rt = g.standard_normal((N, K)) * 3e-3
+    Rt[5, 16:32] = 0.0                                   # an all-zero group
+    e = P.tensor_scale_exponent(Rt)
+    assert e < -5
+    nib0, sc0 = P.quantize_weight_groups(Rt, NVFP4)
+    nib, sc = P.quantize_weight_groups(Rt, NVFP4, e)
+    s0 = F.e4m3_decode(sc0)
+    s = F.e4m3_decode(sc)
+    assert (s0 < 2.0 ** -6).mean() > 0.9                 # global scale 1: subnormal or zero
+    live = np.abs(Rt).reshape(N, K // 16, 16).max(axis=2) > 0
+    assert np.all(s[live] >= 2.0 ** -6) and np.all(s <= 448.0)
+    assert np.all(s[~live] == 0)
+    deq = O.dequantize(nib, sc, NVFP4, e)
+    full = np.repeat(s * 2.0 ** e, 16, axis=1)
+    v = np.abs(Rt) / np.where(full > 0, full, 1.0)
+    half = np.where(v < 2, 0.25, np.where(v < 4, 0.5, 1.0))
+    assert np.all(np.abs(np.abs(Rt) - np.abs(deq)) <= full * half * (1 + 1e-12))
+    assert np.linalg.norm(Rt - deq) < 0.2 * np.linalg.norm(Rt - O.dequantize(nib0, sc0, NVFP4))
+    nib_z, sc_z = P.quantize_weight_groups(Rt, NVFP4, 0)
+    assert np.array_equal(nib_z, nib0) and np.array_equal(sc_z, sc0)
