@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="fc1_nvfp4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-scheme-error", action="store_true",
+                    help="skip the (untimed) quantisation-error report")
     ap.add_argument("--int4-f16", action="store_true",
                     help="INT4 workloads: kernel 2 as one fp16 GEMM of the dequantised operands "
                          "(SVDQ_INT4_F16) instead of int8 MMAs")
@@ -204,6 +206,64 @@ def run_reference(args, layers):
             | {"value": tflops},
             "e2e": {"value": tflops, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def scheme_error(layer, f16: bool = False) -> dict:
+    """The method's own quantisation error on this layer, reported (not a
+    gate): weights prepared by the library's GPU preparation from the
+    layer's seeded full-precision W (calibration on its X, randomized SVD of
+    rank r, residual quantisation), the layer run through the library, and
+    the result compared with the dense fp32 product X W (relative Frobenius
+    norm).  For NVFP4 also with the per-tensor weight scale, and the
+    fraction of weight groups whose E4M3 scale is subnormal or zero without
+    it."""
+    import numpy as np
+    import torch
+    from bit_diffusion_transformer_w4a4_b200 import svdq
+    from bit_diffusion_transformer_w4a4_b200 import workloads as W
+    M, K, N, r, G = layer.M, layer.K, layer.N, layer.r, layer.G
+    x_bits = W.activations(layer)
+    w = W.weight(layer)
+    xd = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    wd = torch.from_numpy(W.to_bf16_bits(w).view(np.int16)).cuda().view(torch.bfloat16)
+    lam = torch.empty(K, dtype=torch.float32, device="cuda")
+    svdq.prep_calibrate(xd, M, wd, K, N, lam)
+    L1 = torch.zeros((K, max(r, 1)), dtype=torch.int16, device="cuda")
+    L2 = torch.zeros((max(r, 1), N), dtype=torch.int16, device="cuda")
+    if r > 0:
+        omega = torch.from_numpy(np.random.default_rng([layer.config_id, 77]).standard_normal(
+            (N, r + 16)).astype(np.float32)).cuda()
+        svdq.prep_lowrank(wd, lam, K, N, r, omega, r + 16, 2, L1, L2)
+    torch.backends.cuda.matmul.allow_tf32 = False
+    ref = xd.float() @ wd.float()
+    out = {"reference": "dense fp32 X W (tf32 off)", "weights": "seeded full-precision W, prepared on the GPU"}
+    sb = 2 if layer.variant == W.INT4 else 1
+    for ts in ([False, True] if layer.variant == W.NVFP4 else [False]):
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty(N * (K // G) * sb, dtype=torch.uint8, device="cuda")
+        e = svdq.prep_residual_quantize(layer.variant, wd, lam, L1 if r else None, L2 if r else None, K, N,
+                                        r, codes, scales, tensor_scale=ts)
+        torch.cuda.synchronize()
+        sc = scales.cpu().numpy()
+        pw = W.PackedWeights(layer.variant, K, N, r, lam.cpu().numpy(),
+                             L1.cpu().numpy().view(np.uint16)[:, :r], L2.cpu().numpy().view(np.uint16)[:r],
+                             codes.cpu().numpy(),
+                             sc.view(np.uint16).reshape(N, -1) if sb == 2 else sc.reshape(N, -1),
+                             gelu=False, w_scale_exp=e)
+        h = svdq.SVDQWeights(pw, M, int4_f16=f16)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        h.linear_forward(xd, y, M)
+        torch.cuda.synchronize()
+        h.close()
+        rel = float(torch.linalg.norm(y.float() - ref) / torch.linalg.norm(ref))
+        out["rel_fro_tensor_scale" if ts else "rel_fro"] = rel
+        if layer.variant == W.NVFP4 and not ts:
+            exp0 = (sc & 0x78) == 0
+            out["w_scale_subnormal_frac"] = float(np.mean(exp0 & (sc != 0)))
+            out["w_scale_zero_frac"] = float(np.mean(sc == 0))
+        if ts:
+            out["w_scale_exp"] = e
+    return out
 
 
 def metric_name(workload: str, layers) -> str:
@@ -425,6 +485,7 @@ def run_ours(args, layers):
                 "d2h_bytes_per_step": sum(d["layer"].M * d["layer"].N * 2 for d in L)},
         "gpu_launches": 2 * len(L) * args.steps,
         "clocks": clk,
+        "kernel_source_hash": kernel_source_hash(),
     }
     # whole-step roofline: the slower of 4-bit compute and the step's HBM bytes
     bytes_alg = sum(layer_bytes(d["layer"]) for d in L)
@@ -434,6 +495,8 @@ def run_ours(args, layers):
                                            bytes_alg / (pk["hbm_gbs"] * 1e9)) / (ms_step * 1e-3)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(L[0]["layer"], L[0]["pw"], L[0]["x_bits"], 1024)
+    if rank == 0 and world == 1 and not args.no_scheme_error:
+        line["scheme_error"] = {d["layer"].name: scheme_error(d["layer"], d["f16"]) for d in L}
     if rank == 0:
         print(json.dumps(line), flush=True)
     for d in L:
@@ -545,7 +608,7 @@ def run_awq(args, layer):
                          "bytes_per_launch": nbytes},
             "e2e": {"value": world * nbytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
-            "gpu_launches": args.steps, "clocks": clk}
+            "gpu_launches": args.steps, "clocks": clk, "kernel_source_hash": kernel_source_hash()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import awq as A
         t = time.perf_counter()

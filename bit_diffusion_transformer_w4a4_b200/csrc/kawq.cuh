@@ -17,14 +17,15 @@
 // parameters [N x K/64] 32-bit words (bf16 scale in the high half, zero
 // point in the low byte), 1/a fp32 [K], bias bf16 [N] or null.
 //
-// Work split: a CTA stages x' of up to MT tokens in shared memory (one
-// 32-element chunk per 36 floats, so the lanes' 16-byte reads of their own
-// chunks hit distinct banks), then each warp takes RW weight rows at a time;
-// lane l reads the 16-byte code chunks l, l+32, ... of each row (a warp reads
-// 512 contiguous bytes per load), decodes eight codes per word with byte
-// permutes into fp32 2^23 + q, subtracts 2^23 + z and accumulates
-// x' (q - z) with packed fp32x2 FMAs; the row's partial sums meet in a warp
-// shuffle reduction.
+// Work split: a persistent grid (one or two CTAs per SM) in which each CTA stages
+// x' of up to MT tokens once in shared memory (one 32-element chunk per 36
+// floats, so the lanes' 16-byte reads of their own chunks hit distinct
+// banks), then each warp takes RW weight rows at a time; lane l reads the
+// 16-byte code chunks l, l+32, ... of each row (a warp reads 512 contiguous
+// bytes per load), CB chunks of every row loaded before any is decoded;
+// decoding turns eight codes per word with byte permutes into fp32 2^23 + q,
+// subtracts 2^23 + z and accumulates x' (q - z) with packed fp32x2 FMAs; the
+// row's partial sums meet in a warp shuffle reduction.
 #pragma once
 
 #include "ptx.cuh"
@@ -34,6 +35,10 @@ namespace svdq {
 constexpr int AWQ_THREADS = 256;
 constexpr int AWQ_G = 64;
 constexpr int AWQ_RW = 4;  // weight rows per warp and pass
+// code chunks per lane and row loaded ahead of the arithmetic, and resident
+// CTAs per SM, by tokens per pass (registers: more tokens, more partial sums)
+template <int MT> constexpr int awq_cb() { return MT <= 2 ? 3 : 1; }
+template <int MT> constexpr int awq_ctas() { return MT == 1 ? 2 : 1; }
 
 // byte `sel` of a, as the fp32 bit pattern 0x4B0000bb (= 2^23 + byte)
 template <int SEL>
@@ -59,8 +64,9 @@ struct AWQSmem {
 };
 
 template <int MT>
-__global__ void __launch_bounds__(AWQ_THREADS)
+__global__ void __launch_bounds__(AWQ_THREADS, awq_ctas<MT>())
     kawq_kernel(AWQParams p) {
+  constexpr int AWQ_CB = awq_cb<MT>();
   extern __shared__ __align__(16) float xs[];  // [MT][K/32][36]
   const int nck = p.K / 32;                    // 16-byte code chunks per row
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -72,16 +78,25 @@ __global__ void __launch_bounds__(AWQ_THREADS)
   for (int m0 = 0; m0 < p.M; m0 += MT) {
     const int mt = min(MT, p.M - m0);
     __syncthreads();
-    for (int i = threadIdx.x; i < MT * (p.K / 2); i += AWQ_THREADS) {
-      const int m = i / (p.K / 2), k = 2 * (i % (p.K / 2));
-      float v0 = 0.f, v1 = 0.f;
+    // x' = fp32(x) * (1/a) for MT tokens, eight elements per item
+    for (int i = threadIdx.x; i < MT * (p.K / 8); i += AWQ_THREADS) {
+      const int m = i / (p.K / 8), k = 8 * (i % (p.K / 8));
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (m < mt) {
-        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p.x + static_cast<size_t>(m0 + m) * p.K + k));
-        const float2 ia = __ldg(reinterpret_cast<const float2*>(p.inv_a + k));
-        v0 = __fmul_rn(bf16lo(w), ia.x);
-        v1 = __fmul_rn(bf16hi(w), ia.y);
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(m0 + m) * p.K + k));
+        const float4 a0 = __ldg(reinterpret_cast<const float4*>(p.inv_a + k));
+        const float4 a1 = __ldg(reinterpret_cast<const float4*>(p.inv_a + k + 4));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        const float ia[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[2 * e] = __fmul_rn(bf16lo(ww[e]), ia[2 * e]);
+          v[2 * e + 1] = __fmul_rn(bf16hi(ww[e]), ia[2 * e + 1]);
+        }
       }
-      *reinterpret_cast<float2*>(xs + (m * nck + k / 32) * 36 + (k % 32)) = make_float2(v0, v1);
+      float* dst = xs + (m * nck + k / 32) * 36 + (k % 32);
+      *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
     }
     __syncthreads();
     for (int n0 = (blockIdx.x * wpb + warp) * AWQ_RW; n0 < p.N; n0 += gstride) {
@@ -90,48 +105,61 @@ __global__ void __launch_bounds__(AWQ_THREADS)
       for (int r = 0; r < AWQ_RW; ++r)
 #pragma unroll
         for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
-      for (int ci = lane; ci < nck; ci += 32) {
-        uint4 cw[AWQ_RW];
-        uint32_t gw[AWQ_RW];
+      // AWQ_CB chunks of each of the RW rows per lane are loaded before any
+      // of them is decoded (up to 12 independent 16-byte loads per lane)
+      for (int cb = 0; cb < nck; cb += 32 * AWQ_CB) {
+        uint4 cw[AWQ_CB][AWQ_RW];
+        uint32_t gw[AWQ_CB][AWQ_RW];
 #pragma unroll
-        for (int r = 0; r < AWQ_RW; ++r) {
-          const int n = min(n0 + r, p.N - 1);  // rows past N recompute row N-1, never stored
-          cw[r] = __ldcs(reinterpret_cast<const uint4*>(p.codes + static_cast<size_t>(n) * (p.K / 2)) + ci);
-          gw[r] = __ldg(p.gp + static_cast<size_t>(n) * (p.K / AWQ_G) + ci / 2);
-        }
-        const float* xc = xs + ci * 36;
+        for (int c = 0; c < AWQ_CB; ++c) {
+          const int ci = cb + 32 * c + lane;
 #pragma unroll
-        for (int r = 0; r < AWQ_RW; ++r) {
-          const float nz = -(8388608.0f + static_cast<float>(gw[r] & 0xFFu));
-          const uint64_t nzz = f2_pack(nz, nz);
-          uint64_t part[MT];
-#pragma unroll
-          for (int m = 0; m < MT; ++m) part[m] = 0ull;
-          const uint32_t words[4] = {cw[r].x, cw[r].y, cw[r].z, cw[r].w};
-#pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
-            const uint32_t lo = words[wi] & 0x0F0F0F0Fu;         // codes 8wi + 2b
-            const uint32_t hi = (words[wi] >> 4) & 0x0F0F0F0Fu;  // codes 8wi + 2b + 1
-            uint64_t q[4];
-            q[0] = f2_add(f2_pack(__uint_as_float(byte_as_magic<0>(lo)), __uint_as_float(byte_as_magic<0>(hi))), nzz);
-            q[1] = f2_add(f2_pack(__uint_as_float(byte_as_magic<1>(lo)), __uint_as_float(byte_as_magic<1>(hi))), nzz);
-            q[2] = f2_add(f2_pack(__uint_as_float(byte_as_magic<2>(lo)), __uint_as_float(byte_as_magic<2>(hi))), nzz);
-            q[3] = f2_add(f2_pack(__uint_as_float(byte_as_magic<3>(lo)), __uint_as_float(byte_as_magic<3>(hi))), nzz);
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-              const float4 xa = *reinterpret_cast<const float4*>(xc + m * nck * 36 + 8 * wi);
-              const float4 xb = *reinterpret_cast<const float4*>(xc + m * nck * 36 + 8 * wi + 4);
-              part[m] = f2_fma(f2_pack(xa.x, xa.y), q[0], part[m]);
-              part[m] = f2_fma(f2_pack(xa.z, xa.w), q[1], part[m]);
-              part[m] = f2_fma(f2_pack(xb.x, xb.y), q[2], part[m]);
-              part[m] = f2_fma(f2_pack(xb.z, xb.w), q[3], part[m]);
+          for (int r = 0; r < AWQ_RW; ++r) {
+            const int n = min(n0 + r, p.N - 1);  // rows past N recompute row N-1, never stored
+            if (ci < nck) {
+              cw[c][r] = __ldcs(reinterpret_cast<const uint4*>(p.codes + static_cast<size_t>(n) * (p.K / 2)) + ci);
+              gw[c][r] = __ldg(p.gp + static_cast<size_t>(n) * (p.K / AWQ_G) + ci / 2);
+            } else {
+              cw[c][r] = make_uint4(0u, 0u, 0u, 0u);
+              gw[c][r] = 0u;                    // scale 0: contributes nothing
             }
           }
-          const float s = __uint_as_float(gw[r] & 0xFFFF0000u);
+        }
 #pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            const float ps = __fadd_rn(f2_lo(part[m]), f2_hi(part[m]));
-            acc[r][m] = __fmaf_rn(s, ps, acc[r][m]);
+        for (int c = 0; c < AWQ_CB; ++c) {
+          const int ci = min(cb + 32 * c + lane, nck - 1);
+          const float* xc = xs + ci * 36;
+#pragma unroll
+          for (int r = 0; r < AWQ_RW; ++r) {
+            const float nz = -(8388608.0f + static_cast<float>(gw[c][r] & 0xFFu));
+            const uint64_t nzz = f2_pack(nz, nz);
+            uint64_t part[MT];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) part[m] = 0ull;
+            const uint32_t words[4] = {cw[c][r].x, cw[c][r].y, cw[c][r].z, cw[c][r].w};
+#pragma unroll
+            for (int wi = 0; wi < 4; ++wi) {
+              const uint32_t lo = words[wi] & 0x0F0F0F0Fu;         // codes 8wi + 2b
+              const uint32_t hi = (words[wi] >> 4) & 0x0F0F0F0Fu;  // codes 8wi + 2b + 1
+              uint64_t q[4];
+              q[0] = f2_add(f2_pack(__uint_as_float(byte_as_magic<0>(lo)), __uint_as_float(byte_as_magic<0>(hi))), nzz);
+              q[1] = f2_add(f2_pack(__uint_as_float(byte_as_magic<1>(lo)), __uint_as_float(byte_as_magic<1>(hi))), nzz);
+              q[2] = f2_add(f2_pack(__uint_as_float(byte_as_magic<2>(lo)), __uint_as_float(byte_as_magic<2>(hi))), nzz);
+              q[3] = f2_add(f2_pack(__uint_as_float(byte_as_magic<3>(lo)), __uint_as_float(byte_as_magic<3>(hi))), nzz);
+#pragma unroll
+              for (int m = 0; m < MT; ++m) {
+                const float4 xa = *reinterpret_cast<const float4*>(xc + m * nck * 36 + 8 * wi);
+                const float4 xb = *reinterpret_cast<const float4*>(xc + m * nck * 36 + 8 * wi + 4);
+                part[m] = f2_fma(f2_pack(xa.x, xa.y), q[0], part[m]);
+                part[m] = f2_fma(f2_pack(xa.z, xa.w), q[1], part[m]);
+                part[m] = f2_fma(f2_pack(xb.x, xb.y), q[2], part[m]);
+                part[m] = f2_fma(f2_pack(xb.z, xb.w), q[3], part[m]);
+              }
+            }
+            const float sc = __uint_as_float(gw[c][r] & 0xFFFF0000u);
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+              acc[r][m] = __fmaf_rn(sc, __fadd_rn(f2_lo(part[m]), f2_hi(part[m])), acc[r][m]);
           }
         }
       }

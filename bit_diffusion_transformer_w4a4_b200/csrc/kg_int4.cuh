@@ -278,6 +278,11 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 16; ++i) acc[i] = 0ull;
       float sx_next = gm < p.M ? __bfloat162float(sxr[0]) : 0.0f;
+      const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16) + cs * 32;
+      // float(P) for the s32 group product P (a sum of 64 products of 4-bit
+      // codes, |P| <= 4096 < 2^22): bits(P + bits(1.5 * 2^23)) - 1.5 * 2^23,
+      // exact, at the full rate of integer and fp32 adds
+      const uint64_t mag = f2_pack(-12582912.0f, -12582912.0f);
       for (int g = 0; g < ng; ++g, ++gc) {
         const uint32_t b = gc % KGI4_BUFS, use = gc / KGI4_BUFS;
         const float sx = sx_next;
@@ -287,21 +292,21 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         if (!(ok = __all_sync(0xffffffffu, wait_bounded(bar_gfull + 8 * b, use & 1, guard, 0x30a)))) break;
         tc_fence_after();
         uint32_t v[32];
-        tmem_ld_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * KGI4_BN + cs * 32, v);
+        tmem_ld_x32(tq + b * KGI4_BN, v);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_gempty + 8 * b);
-        // acc += (s_x * s_w[n]) * float(P[n]), two columns per instruction
+        // acc += (s_x * s_w[n]) * P[n], two columns per instruction
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
           const float4 w = __ldg(swr + i4);
           const uint64_t s01 = f2_mul(sx2, f2_pack(w.x, w.y));
           const uint64_t s23 = f2_mul(sx2, f2_pack(w.z, w.w));
-          const uint64_t p01 = f2_pack(__int2float_rn(static_cast<int>(v[4 * i4])),
-                                       __int2float_rn(static_cast<int>(v[4 * i4 + 1])));
-          const uint64_t p23 = f2_pack(__int2float_rn(static_cast<int>(v[4 * i4 + 2])),
-                                       __int2float_rn(static_cast<int>(v[4 * i4 + 3])));
+          const uint64_t p01 = f2_add(f2_pack(__uint_as_float(v[4 * i4] + 0x4B400000u),
+                                              __uint_as_float(v[4 * i4 + 1] + 0x4B400000u)), mag);
+          const uint64_t p23 = f2_add(f2_pack(__uint_as_float(v[4 * i4 + 2] + 0x4B400000u),
+                                              __uint_as_float(v[4 * i4 + 3] + 0x4B400000u)), mag);
           acc[2 * i4] = f2_fma(p01, s01, acc[2 * i4]);
           acc[2 * i4 + 1] = f2_fma(p23, s23, acc[2 * i4 + 1]);
         }

@@ -179,6 +179,13 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
+  // E4M3 scale code -> (value, RN(1 / value)) for the NVFP4 quantiser (the
+  // codes of non-negative satfinite scales are 0..126)
+  __shared__ float2 e4lut[128];
+  if (VARIANT == 1 && threadIdx.x < 128) {
+    const float v = e4m3_value(threadIdx.x);
+    e4lut[threadIdx.x] = make_float2(v, v > 0.0f && threadIdx.x < 127 ? __frcp_rn(v) : 0.0f);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -268,10 +275,15 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
       for (int j = 0; j < 8; ++j) {
         const uint4 v = *reinterpret_cast<const uint4*>(xt + swz_off(row, j, 128));
         const float4 f0 = il[2 * j], f1 = il[2 * j + 1];
-        w[4 * j] = pack_bf16x2(__fmul_rn(bf16lo(v.x), f0.x), __fmul_rn(bf16hi(v.x), f0.y));
-        w[4 * j + 1] = pack_bf16x2(__fmul_rn(bf16lo(v.y), f0.z), __fmul_rn(bf16hi(v.y), f0.w));
-        w[4 * j + 2] = pack_bf16x2(__fmul_rn(bf16lo(v.z), f1.x), __fmul_rn(bf16hi(v.z), f1.y));
-        w[4 * j + 3] = pack_bf16x2(__fmul_rn(bf16lo(v.w), f1.z), __fmul_rn(bf16hi(v.w), f1.w));
+        // two round-to-nearest fp32 products per instruction, then bf16 RN
+        const uint64_t p0 = f2_mul(f2_pack(bf16lo(v.x), bf16hi(v.x)), f2_pack(f0.x, f0.y));
+        const uint64_t p1 = f2_mul(f2_pack(bf16lo(v.y), bf16hi(v.y)), f2_pack(f0.z, f0.w));
+        const uint64_t p2 = f2_mul(f2_pack(bf16lo(v.z), bf16hi(v.z)), f2_pack(f1.x, f1.y));
+        const uint64_t p3 = f2_mul(f2_pack(bf16lo(v.w), bf16hi(v.w)), f2_pack(f1.z, f1.w));
+        w[4 * j] = pack_bf16x2(f2_lo(p0), f2_hi(p0));
+        w[4 * j + 1] = pack_bf16x2(f2_lo(p1), f2_hi(p1));
+        w[4 * j + 2] = pack_bf16x2(f2_lo(p2), f2_hi(p2));
+        w[4 * j + 3] = pack_bf16x2(f2_lo(p3), f2_hi(p3));
       }
       // Each thread orders its own shared-memory accesses of this stage before
       // the async proxy (tensor core or the TMA refill) touches it again, and
@@ -296,18 +308,25 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
         for (int g = 0; g < 4; ++g) {
           const float a = bf16_amax<8>(w + 8 * g);
           const uint32_t code = e4m3_rn(div_by_scale(a, 6.0f, kRcp6));
-          const float s_ = e4m3_value(code);
+          const float2 sy = e4lut[code];  // the scale's value and RN(1 / value)
+          const float s_ = sy.x;
           sc |= code << (8 * g);
           if (s_ > 0.0f) {           // E4M3 scales are >= 2^-9: 1/s is finite
-            const float y = __frcp_rn(s_);
+            // div_by_scale on two values per instruction: q0 = x y,
+            // r = fma(q0, -s, x) (= fma(-q0, s, x) exactly), q1 = fma(r, y, q0),
+            // then x's sign put back
+            const uint64_t y2 = f2_pack(sy.y, sy.y), ns2 = f2_pack(-s_, -s_);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               float v[8];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const uint32_t ww = w[8 * g + 4 * h + e];
-                v[2 * e] = div_by_scale(bf16lo(ww), s_, y);
-                v[2 * e + 1] = div_by_scale(bf16hi(ww), s_, y);
+                const uint64_t x2 = f2_pack(bf16lo(ww), bf16hi(ww));
+                const uint64_t q0 = f2_mul(x2, y2);
+                const uint64_t q1 = f2_fma(f2_fma(q0, ns2, x2), y2, q0);
+                v[2 * e] = __uint_as_float(__float_as_uint(f2_lo(q1)) | ((ww << 16) & 0x80000000u));
+                v[2 * e + 1] = __uint_as_float(__float_as_uint(f2_hi(q1)) | (ww & 0x80000000u));
               }
               packed[2 * g + h] = e2m1x8(v);
             }
@@ -330,14 +349,25 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
         const float s_ = __bfloat162float(sb);
         if (s_ >= kMinFastScale && s_ < kMaxFastScale) {
           const float y = __frcp_rn(s_);
+          // div_by_scale on two values per instruction (its sign repair is not
+          // needed: -0 and +0 give the same INT4 code); then rint by adding
+          // 1.5 * 2^23, which leaves the integer in the low mantissa bits.
+          // The clamp to [-8, 7] is not needed here: s = bf16(amax / 7) is at
+          // least (amax / 7)(1 - 2^-9), so |x / s| <= 7.014 and rint is in
+          // [-7, 7].
+          const uint64_t y2 = f2_pack(y, y), ns2 = f2_pack(-s_, -s_);
+          const uint64_t mg2 = f2_pack(12582912.0f, 12582912.0f);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             uint32_t pk = 0;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const uint32_t ww = w[4 * j + e];
-              pk |= int4_rn(div_by_scale(bf16lo(ww), s_, y)) << (8 * e);
-              pk |= int4_rn(div_by_scale(bf16hi(ww), s_, y)) << (8 * e + 4);
+              const uint64_t x2 = f2_pack(bf16lo(ww), bf16hi(ww));
+              const uint64_t q0 = f2_mul(x2, y2);
+              const uint64_t r2 = f2_add(f2_fma(f2_fma(q0, ns2, x2), y2, q0), mg2);
+              pk |= (__float_as_uint(f2_lo(r2)) & 0xFu) << (8 * e);
+              pk |= (__float_as_uint(f2_hi(r2)) & 0xFu) << (8 * e + 4);
             }
             packed[j] = pk;
           }

@@ -646,10 +646,14 @@ void awq_free_all(svdq_awq* h) {
     if (q) cudaFree(q);
 }
 
+constexpr int kAwqSmemCap = 100 * 1024;  // staged tokens per pass are chosen to fit
+
 template <int MT>
 svdq_status launch_awq(svdq_awq* h, const void* x, void* y, int64_t M, cudaStream_t st) {
   const size_t smem = AWQSmem<MT>::bytes(static_cast<int>(h->K));
-  if (svdq_status s = ensure_smem<kawq_kernel<MT>>(static_cast<int>(smem)); s != SVDQ_OK) return s;
+  // the opt-in is the largest size any K can ask for (the cap below), so the
+  // per-device cache stays valid for every later call
+  if (svdq_status s = ensure_smem<kawq_kernel<MT>>(kAwqSmemCap); s != SVDQ_OK) return s;
   AWQParams p;
   p.codes = h->codes;
   p.gp = h->gp;
@@ -660,9 +664,11 @@ svdq_status launch_awq(svdq_awq* h, const void* x, void* y, int64_t M, cudaStrea
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(h->K);
   p.N = static_cast<int>(h->N);
+  // persistent: one or two CTAs per SM (x' is staged once per CTA)
   const int64_t rows_per_cta = (AWQ_THREADS / 32) * AWQ_RW;
   const int64_t want = cdiv(h->N, rows_per_cta);
-  const int grid = static_cast<int>(want < 4 * h->sms ? want : 4 * h->sms);
+  const int64_t resident = static_cast<int64_t>(awq_ctas<MT>()) * h->sms;
+  const int grid = static_cast<int>(want < resident ? want : resident);
   LaunchCfg lc(dim3(grid), dim3(AWQ_THREADS), static_cast<int>(smem), st);
   SVDQ_TRY(cudaLaunchKernelEx(&lc.cfg, kawq_kernel<MT>, p));
   return SVDQ_OK;
@@ -1202,7 +1208,7 @@ svdq_status svdq_awq_load(const svdq_awq_desc* d, svdq_awq_t* out, void* stream)
   if (!d || !out) return SVDQ_ERR_INVALID_ARG;
   *out = nullptr;
   const int64_t K = d->K, N = d->N;
-  if (K < 64 || K % 64 != 0 || K > 32768) return SVDQ_ERR_SHAPE;
+  if (K < 64 || K % 64 != 0 || K > 16384) return SVDQ_ERR_SHAPE;
   if (N < 1 || N > (1 << 24)) return SVDQ_ERR_SHAPE;
   if (d->max_M < 1 || d->max_M > (1ll << 30)) return SVDQ_ERR_SHAPE;
   if (!d->a || !d->codes || !d->scales || !d->zeros) return SVDQ_ERR_INVALID_ARG;
@@ -1266,7 +1272,7 @@ svdq_status svdq_awq_w4a16_forward(svdq_awq_t h, const void* x, void* y, int64_t
   if (dev != h->device) return SVDQ_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // tokens staged per pass: as many as fit, up to 8
-  const size_t cap = 200 * 1024;
+  const size_t cap = kAwqSmemCap;
   if (M >= 5 && AWQSmem<8>::bytes(static_cast<int>(h->K)) <= cap) return launch_awq<8>(h, x, y, M, st);
   if (M >= 3 && AWQSmem<4>::bytes(static_cast<int>(h->K)) <= cap) return launch_awq<4>(h, x, y, M, st);
   if (M >= 2 && AWQSmem<2>::bytes(static_cast<int>(h->K)) <= cap) return launch_awq<2>(h, x, y, M, st);

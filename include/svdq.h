@@ -311,7 +311,7 @@ typedef struct svdq_awq* svdq_awq_t;   /* opaque, library-owned */
  *   scales  bf16 [N x K/64] group scales s
  *   zeros   u8   [N x K/64] integer zero points 0..15 (else INVALID_ARG)
  *   bias    bf16 [N] or NULL
- * Shapes: K % 64 == 0, 64 <= K <= 32768, 1 <= N, 1 <= M <= max_M. */
+ * Shapes: K % 64 == 0, 64 <= K <= 16384, 1 <= N, 1 <= M <= max_M. */
 typedef struct {
   int64_t K, N, max_M;
   const float* a;

@@ -258,3 +258,44 @@ def test_nvfp4_tensor_scale(opts, M, K, N, r):
     PT.check_act(got, ref, r=r, label="tensor scale")
     PT.check_y(got["Y"], ref["y"], ref["Y"], label=f"tensor scale e{pw.w_scale_exp} {opts}")
     h.close()
+
+
+def test_handles_loaded_from_two_threads():
+    """Two threads load handles and run the layer at the same time (first
+    calls race on the per-device shared-memory opt-in); both results equal a
+    single-threaded run."""
+    import threading
+    import torch
+    M, K, N, r = 256, 512, 512, 32
+    cases = []
+    for i, variant in enumerate((NVFP4, INT4)):
+        lay = W.Layer("thr", M=M, K=K, N=N, r=r, variant=variant, config_id=69, layer_id=i)
+        cases.append((lay, W.synthetic_packed(lay), W.activations(lay)))
+    ref = []
+    for lay, pw, x in cases:
+        h = svdq.SVDQWeights(pw, M)
+        ref.append(PT.gpu_forward(h, x, M)["Y"])
+        h.close()
+    out = [None, None]
+    err = []
+
+    def work(i):
+        try:
+            torch.cuda.set_device(0)
+            lay, pw, x = cases[i]
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                h = svdq.SVDQWeights(pw, M)
+                out[i] = PT.gpu_forward(h, x, M)["Y"]
+                h.close()
+        except Exception as e:  # reported below
+            err.append(e)
+
+    th = [threading.Thread(target=work, args=(i,)) for i in range(2)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert not err, err
+    for i in range(2):
+        assert np.array_equal(out[i], ref[i])
