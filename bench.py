@@ -47,6 +47,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-scheme-error", action="store_true",
                     help="skip the (untimed) quantisation-error report")
+    ap.add_argument("--overhead-repeats", type=int, default=0,
+                    help="also time the same single-layer workload at r = 0, alternating with it this "
+                         "many times (each of --steps steps), and report the low-rank branch's "
+                         "overhead t(r) / t(0) - 1 as median and range")
     ap.add_argument("--int4-f16", action="store_true",
                     help="INT4 workloads: kernel 2 as one fp16 GEMM of the dequantised operands "
                          "(SVDQ_INT4_F16) instead of int8 MMAs")
@@ -264,6 +268,45 @@ def scheme_error(layer, f16: bool = False) -> dict:
         if ts:
             out["w_scale_exp"] = e
     return out
+
+
+def lowrank_overhead(d, steps: int, repeats: int, flush) -> dict:
+    """t(r) / t(r = 0) - 1 for one layer: the same shapes, format and inputs
+    with the low-rank branch removed, both timed `repeats` times alternately
+    (each a mean over `steps` flushed steps, CUDA events at step boundaries)."""
+    import dataclasses
+    import statistics
+    import torch
+    from bit_diffusion_transformer_w4a4_b200 import svdq
+    from bit_diffusion_transformer_w4a4_b200 import workloads as W
+    layer = d["layer"]
+    l0 = dataclasses.replace(layer, r=0)
+    pw0 = W.synthetic_packed(l0)
+    h0 = svdq.SVDQWeights(pw0, l0.M, int4_f16=d["f16"])
+    c0, s0, t0 = h0.alloc_act(l0.M)
+    y0 = torch.empty_like(d["y"])
+    stream = torch.cuda.current_stream()
+
+    def timed(h, codes, scales, t, y):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for i in range(steps):
+            flush()
+            ev[i][0].record(stream)
+            h.quantize_act_lowrank_down(d["x"], layer.M, codes, scales, t)
+            h.w4a4_gemm_lowrank_up(codes, scales, t, layer.M, y)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+
+    timed(h0, c0, s0, t0, y0)
+    tr, t0s = [], []
+    for _ in range(repeats):
+        tr.append(timed(d["h"], d["codes"], d["scales"], d["t"], d["y"]))
+        t0s.append(timed(h0, c0, s0, t0, y0))
+    h0.close()
+    ov = [a / b - 1.0 for a, b in zip(tr, t0s)]
+    return {"r": layer.r, "median": statistics.median(ov), "min": min(ov), "max": max(ov),
+            "repeats": repeats, "steps_each": steps, "ms_r": tr, "ms_r0": t0s}
 
 
 def metric_name(workload: str, layers) -> str:
@@ -497,6 +540,8 @@ def run_ours(args, layers):
         line["cpu_baseline"] = cpu_baseline(L[0]["layer"], L[0]["pw"], L[0]["x_bits"], 1024)
     if rank == 0 and world == 1 and not args.no_scheme_error:
         line["scheme_error"] = {d["layer"].name: scheme_error(d["layer"], d["f16"]) for d in L}
+    if args.overhead_repeats > 0 and len(L) == 1 and world == 1:
+        line["lowrank_overhead"] = lowrank_overhead(L[0], args.steps, args.overhead_repeats, flush)
     if rank == 0:
         print(json.dumps(line), flush=True)
     for d in L:
