@@ -21,6 +21,7 @@
 #include "kg_int4.cuh"
 #include "kg_int4h.cuh"
 #include "kg_nvfp4.cuh"
+#include "kg_nvfp4_chain.cuh"
 #include "kg_nvfp4_pair.cuh"
 #include "kq.cuh"
 
@@ -467,6 +468,49 @@ svdq_status launch_kg_v(svdq_weights* h, const CUtensorMap& tma, const uint8_t* 
   return SVDQ_ERR_SHAPE;
 }
 
+
+// fc1's kernel 2 with fc2's activation side fused into the epilogue.
+template <int R, int R2>
+svdq_status launch_chain_t(svdq_weights* h1, svdq_weights* h2, const CUtensorMap& tma, int64_t M,
+                           const uint8_t* sfa, const float* t, void* y1, uint8_t* codes2, uint8_t* scales2,
+                           float* t2, cudaStream_t st) {
+  using C = KGChainSmem<R, R2>;
+  if (svdq_status s = ensure_smem<kg_nvfp4_chain_kernel<R, R2>>(C::TOTAL); s != SVDQ_OK) return s;
+  KGParams p;
+  p.sfa = sfa;
+  p.sfb = h1->wscales;
+  p.t = t;
+  p.bias = h1->bias;
+  p.y = static_cast<uint16_t*>(y1);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(h1->N);
+  p.K = static_cast<int>(h1->K);
+  p.num_m = static_cast<int>(cdiv(M, KG_BM));
+  p.num_n = static_cast<int>(cdiv(h1->N, KG_BN));
+  p.gelu = (h1->flags & SVDQ_EPI_GELU) ? 1 : 0;
+  p.out_scale = h1->out_scale;
+  p.t_scale = h1->t_scale;
+  p.qkv_hd = 0;
+  p.norm_eps = 0.f;
+  p.gq = p.gk = nullptr;
+  p.rope = nullptr;
+  p.err = h1->err;
+  p.debug_mask = 0;
+  p.timeout_ns = h1->timeout_ns;
+  KGChainParams c;
+  c.inv_lam2 = h2->inv_lam;
+  c.codes2 = codes2;
+  c.scales2 = scales2;
+  c.t2 = t2;
+  c.store_y = y1 != nullptr ? 1 : 0;
+  const int tiles = p.num_m * p.num_n;
+  const int grid = tiles < h1->sms ? tiles : h1->sms;
+  LaunchCfg lc(dim3(grid), dim3(KG_THREADS), C::TOTAL, st);
+  SVDQ_TRY(cudaLaunchKernelEx(&lc.cfg, kg_nvfp4_chain_kernel<R, R2>, tma, h1->tm_b, h1->tm_blr, h2->tm_l1t, p, c));
+  return SVDQ_OK;
+}
+
+
 svdq_status get_tm_x(svdq_weights* h, const void* x, int64_t M) {
   if (h->tm_x_ptr == x && h->tm_x_M == M) return SVDQ_OK;
   svdq_status s = make_tmap(&h->tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->K, M, 64, 128,
@@ -499,6 +543,18 @@ svdq_status check_call(svdq_weights* h, int64_t M) {
   if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
   if (dev != h->device) return SVDQ_ERR_INVALID_ARG;
   return SVDQ_OK;
+}
+
+svdq_status check_chain(svdq_weights* h1, svdq_weights* h2, int64_t M) {
+  if (!h1 || !h2) return SVDQ_ERR_INVALID_ARG;
+  if (h1->variant != SVDQ_NVFP4_G16_E4M3 || h2->variant != SVDQ_NVFP4_G16_E4M3) return SVDQ_ERR_INVALID_ARG;
+  if ((h1->flags | h2->flags) & SVDQ_EPI_QKV_NORM_ROPE) return SVDQ_ERR_INVALID_ARG;
+  if (h1->N != h2->K || h1->N % 256 != 0) return SVDQ_ERR_SHAPE;
+  if (!(h1->r == 0 || h1->r == 32) || !(h2->r == 16 || h2->r == 32)) return SVDQ_ERR_SHAPE;
+  if (h1->device != h2->device) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_call(h1, M);
+  if (s != SVDQ_OK) return s;
+  return check_call(h2, M);
 }
 
 // ------------------------------------------------------------- self-test
@@ -1202,6 +1258,52 @@ svdq_status svdq_quantize_act_lowrank_down_static(svdq_variant variant, int64_t 
   return variant == SVDQ_NVFP4_G16_E4M3
              ? launch_kq_static_v<1>(r, tmx, tml, inv_lambda, M, K, sms, act_codes, act_scales, t, scratch, err, st)
              : launch_kq_static_v<0>(r, tmx, tml, inv_lambda, M, K, sms, act_codes, act_scales, t, scratch, err, st);
+}
+
+svdq_status svdq_w4a4_gemm_lowrank_up_chain(svdq_weights_t h1, const uint8_t* act_codes,
+                                            const void* act_scales, const float* t, int64_t M, void* y1,
+                                            svdq_weights_t h2, uint8_t* act_codes2, void* act_scales2,
+                                            float* t2, void* stream) {
+  svdq_status s = check_chain(h1, h2, M);
+  if (s != SVDQ_OK) return s;
+  if (!act_codes || !act_scales || (h1->r > 0 && !t) || !act_codes2 || !act_scales2 || !t2)
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(act_codes) || !aligned16(act_scales) || (t && !aligned16(t)) || (y1 && !aligned16(y1)) ||
+      !aligned16(act_codes2) || !aligned16(act_scales2) || !aligned16(t2))
+    return SVDQ_ERR_ALIGNMENT;
+  if ((s = get_tm_a(h1, act_codes, M)) != SVDQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SVDQ_TRY(cudaMemsetAsync(t2, 0, static_cast<size_t>(M) * h2->r * 4, st));  // T2 is accumulated atomically
+  const uint8_t* sfa = static_cast<const uint8_t*>(act_scales);
+  uint8_t* sc2 = static_cast<uint8_t*>(act_scales2);
+  if (h1->r == 0)
+    return h2->r == 16 ? launch_chain_t<0, 16>(h1, h2, h1->tm_a, M, sfa, t, y1, act_codes2, sc2, t2, st)
+                       : launch_chain_t<0, 32>(h1, h2, h1->tm_a, M, sfa, t, y1, act_codes2, sc2, t2, st);
+  return h2->r == 16 ? launch_chain_t<32, 16>(h1, h2, h1->tm_a, M, sfa, t, y1, act_codes2, sc2, t2, st)
+                     : launch_chain_t<32, 32>(h1, h2, h1->tm_a, M, sfa, t, y1, act_codes2, sc2, t2, st);
+}
+
+svdq_status svdq_linear_forward_chain(svdq_weights_t h1, svdq_weights_t h2, const void* x, void* y2, int64_t M,
+                                      void* stream) {
+  svdq_status s = check_chain(h1, h2, M);
+  if (s != SVDQ_OK) return s;
+  if (!x || !y2) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // T2 is zeroed first, so the three kernels follow one another with
+  // programmatic dependent launch and nothing in between
+  SVDQ_TRY(cudaMemsetAsync(h2->ws_t, 0, static_cast<size_t>(M) * h2->r * 4, st));
+  if ((s = svdq_quantize_act_lowrank_down(h1, x, M, h1->ws_codes, h1->ws_scales, h1->ws_t, stream)) != SVDQ_OK)
+    return s;
+  if ((s = get_tm_a(h1, h1->ws_codes, M)) != SVDQ_OK) return s;
+  const uint8_t* sfa = h1->ws_scales;
+  if (h1->r == 0)
+    s = h2->r == 16 ? launch_chain_t<0, 16>(h1, h2, h1->tm_a, M, sfa, h1->ws_t, nullptr, h2->ws_codes, h2->ws_scales, h2->ws_t, st)
+                    : launch_chain_t<0, 32>(h1, h2, h1->tm_a, M, sfa, h1->ws_t, nullptr, h2->ws_codes, h2->ws_scales, h2->ws_t, st);
+  else
+    s = h2->r == 16 ? launch_chain_t<32, 16>(h1, h2, h1->tm_a, M, sfa, h1->ws_t, nullptr, h2->ws_codes, h2->ws_scales, h2->ws_t, st)
+                    : launch_chain_t<32, 32>(h1, h2, h1->tm_a, M, sfa, h1->ws_t, nullptr, h2->ws_codes, h2->ws_scales, h2->ws_t, st);
+  if (s != SVDQ_OK) return s;
+  return svdq_w4a4_gemm_lowrank_up(h2, h2->ws_codes, h2->ws_scales, h2->ws_t, M, y2, stream);
 }
 
 svdq_status svdq_awq_load(const svdq_awq_desc* d, svdq_awq_t* out, void* stream) {

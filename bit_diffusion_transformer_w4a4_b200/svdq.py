@@ -36,6 +36,7 @@ EXPORTED = [
     "svdq_awq_load", "svdq_awq_free", "svdq_awq_w4a16_forward",
     "svdq_prep_calibrate", "svdq_prep_lowrank", "svdq_prep_residual_quantize",
     "svdq_w4a4_gemm_lowrank_up_qkv", "svdq_linear_forward_qkv",
+    "svdq_w4a4_gemm_lowrank_up_chain", "svdq_linear_forward_chain",
 ]
 
 
@@ -93,6 +94,8 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
     L.svdq_debug_set_fault.argtypes = [vp, ctypes.c_uint32, ctypes.c_uint32]
     L.svdq_selftest_division.argtypes = [ctypes.c_int, ctypes.c_void_p]
     L.svdq_w4a4_gemm_lowrank_up_qkv.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp]
+    L.svdq_w4a4_gemm_lowrank_up_chain.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp]
+    L.svdq_linear_forward_chain.argtypes = [vp, vp, vp, vp, i64, vp]
     L.svdq_linear_forward_qkv.argtypes = [vp, vp, vp, vp, i64, vp]
     L.svdq_awq_load.argtypes = [ctypes.POINTER(AWQDesc), ctypes.POINTER(vp), vp]
     L.svdq_awq_free.argtypes = [vp]
@@ -311,6 +314,20 @@ def prep_residual_quantize(variant, w, lam, L1, L2, K, N, r, codes, scales, tens
                                              _ptr(scales), ctypes.byref(e), _stream(stream)),
            "svdq_prep_residual_quantize")
     return int(e.value)
+
+
+def gemm_lowrank_up_chain(h1, act_codes, act_scales, t, M, y1, h2, codes2, scales2, t2, stream=None):
+    """h1's kernel 2 with h2's activation side in its epilogue (see
+    svdq_w4a4_gemm_lowrank_up_chain); y1 may be None."""
+    _check(lib().svdq_w4a4_gemm_lowrank_up_chain(
+        h1.handle, _ptr(act_codes), _ptr(act_scales), _ptr(t), int(M), _ptr(y1), h2.handle, _ptr(codes2),
+        _ptr(scales2), _ptr(t2), _stream(stream)), "svdq_w4a4_gemm_lowrank_up_chain")
+
+
+def linear_forward_chain(h1, h2, x, y2, M, stream=None):
+    """y2 = fc2(fc1(x)) with fc2's activation side fused into fc1's GEMM."""
+    _check(lib().svdq_linear_forward_chain(h1.handle, h2.handle, _ptr(x), _ptr(y2), int(M), _stream(stream)),
+           "svdq_linear_forward_chain")
 
 
 def untile_nvfp4_scales(buf: np.ndarray, M: int, K: int) -> np.ndarray:

@@ -242,6 +242,38 @@ svdq_status svdq_linear_forward_qkv(svdq_weights_t h, const void* x, const float
                                     int64_t M, void* stream);
 
 /*
+ * Defined by: "Problemas do Nunchaku Qwen ..." (apatero.com), section "O que
+ * e Nunchaku e como acelera modelos Qwen" -- the down projection fused with
+ * the quantisation kernel, the up projection with the 4-bit kernel, the
+ * branches sharing the activations; "Nunchaku Lite ..." (axbrief.com),
+ * section "The Trade-off Between Fused Kernels and Generality" -- fused
+ * paths bundle operations to cut memory traffic.  Here two consecutive
+ * layers (a DiT MLP's fc1 and fc2) share a kernel: fc1's GEMM epilogue
+ * computes fc1's output y1 = bf16(GELU?(acc + bias)), then fc2's activation
+ * side from it -- x2 = bf16(fp32(y1) * (1/lambda2)), fc2's NVFP4 codes and
+ * scales (bit-identical to svdq_quantize_act_lowrank_down on y1) and
+ * T2 = X2' L1_2 (tensor cores, fp32; several CTAs add into one row block
+ * with fp32 atomics, so T2's summation order is not fixed) -- and y1 itself
+ * is only stored when asked for.
+ * Both handles NVFP4 (no QKV epilogue), h1's N == h2's K, N % 256 == 0,
+ * h1's r in {0, 32}, h2's r in {16, 32}, else SVDQ_ERR_SHAPE / INVALID_ARG.
+ *
+ * svdq_w4a4_gemm_lowrank_up_chain: h1's kernel 2 on its activation codes,
+ *   scales and T (as from svdq_quantize_act_lowrank_down on h1), writing
+ *   h2's act_codes2 [M x N1/2], act_scales2 (tiled, svdq_act_scales_bytes of
+ *   h2) and t2 fp32 [M x r2] (zeroed by the call on `stream`, then added
+ *   into), and y1 bf16 [M x N1] unless y1 is NULL.
+ * svdq_linear_forward_chain: y2 = fc2(fc1(x)) through the handles'
+ *   workspaces: fc1's activation kernel, the fused kernel, fc2's GEMM.
+ */
+svdq_status svdq_w4a4_gemm_lowrank_up_chain(svdq_weights_t h1, const uint8_t* act_codes,
+                                            const void* act_scales, const float* t, int64_t M, void* y1,
+                                            svdq_weights_t h2, uint8_t* act_codes2, void* act_scales2,
+                                            float* t2, void* stream);
+svdq_status svdq_linear_forward_chain(svdq_weights_t h1, svdq_weights_t h2, const void* x, void* y2,
+                                      int64_t M, void* stream);
+
+/*
  * Defined by: the same layer as svdq_linear_forward.
  * Same as svdq_linear_forward with HOST input and output (pinned memory is
  * recommended): copies x_host to the device, runs the layer and copies y back
