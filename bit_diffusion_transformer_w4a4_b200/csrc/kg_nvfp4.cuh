@@ -79,8 +79,9 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   const uint32_t bar_drain = smem_u32(bars + 2 * NST + 3);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NST + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  // per stage: A's / B's scale factors are in tensor memory (and the stage's
-  // data has landed); per copy warp: its copies have drained
+  // per stage: the scale factors of the first / second half of the stage's
+  // k-blocks are in tensor memory (and the stage's data has landed); per
+  // copy warp: its copies have drained
   const uint32_t bar_sfa = smem_u32(bars + 2 * NST + 5);
   const uint32_t bar_sfb = smem_u32(bars + 3 * NST + 5);
   const uint32_t bar_sf_drain = smem_u32(bars + 4 * NST + 5);  // two barriers
@@ -187,20 +188,24 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         if (j > 0 && !(ok = wait_bounded(bar_acc_empty, (j - 1) & 1, guard, 0x203))) break;
         tc_fence_after();
         for (int ks = 0; ks < nks; ++ks) {
-          if (!(ok = wait_bounded(bar_sfa + 8 * s, ph, guard, 0x204) &&
-                     wait_bounded(bar_sfb + 8 * s, ph, guard, 0x20a)))
-            break;
-          tc_fence_after();
           const uint64_t so = kStage * s;
           const int kv = min(KB, kblk - KB * ks);
           const uint32_t ca = tmem + S::SFA_COL + KB * 4 * s;
           const uint32_t cb = tmem + S::SFB_COL + KB * 8 * s;
+          // the first half of the k-blocks once warp 2's copies are in, the
+          // second half once warp 3's are
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) {
-            if (kb >= kv) break;
-            mma_nvf4(tmem, dA0 + so + 2 * kb, dB0 + so + 2 * kb, id_f4, ca + 4 * kb, cb + 8 * kb,
-                     (ks | kb) != 0);
+            if (kb == 0 || kb == KB / 2) {
+              if (!(ok = wait_bounded(kb == 0 ? bar_sfa + 8 * s : bar_sfb + 8 * s, ph, guard,
+                                      kb == 0 ? 0x204 : 0x20a)))
+                break;
+              tc_fence_after();
+            }
+            if (kb < kv)
+              mma_nvf4(tmem, dA0 + so + 2 * kb, dB0 + so + 2 * kb, id_f4, ca + 4 * kb, cb + 8 * kb, (ks | kb) != 0);
           }
+          if (!ok) break;
           tc_commit(bar_empty + 8 * s);
           if (++s == NST) { s = 0; ph ^= 1; }
         }
@@ -235,37 +240,36 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     }
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------- scale-factor copies
-    // Warp 2 copies A's atom, warp 3 B's two atoms, per k-block.  Every stage
-    // (k-blocks or low-rank) completes this warp's barrier once, after its
-    // data has landed, so the MMA warp keeps one ring parity for all.
+    // Warp 2 copies the scale atoms (A's and both of B's) of the first half
+    // of each stage's k-blocks, warp 3 those of the second half, so the two
+    // warps issue equal shares.  Every stage (k-blocks or low-rank) completes
+    // each warp's barrier once, after its data has landed, so the MMA warp
+    // keeps one ring parity for all.
     if (lane == 0) {
-      const bool is_a = warp == 2;
-      const uint32_t ready = is_a ? bar_sfa : bar_sfb;
-      const uint64_t d0 = is_a ? smem_desc(sbase + S::A_BYTES + S::B_BYTES, 0, 128, SWZ_NONE)
-                               : smem_desc(sbase + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, 0, 128, SWZ_NONE);
+      const int h = warp - 2;
+      const uint32_t ready = h == 0 ? bar_sfa : bar_sfb;
+      const uint64_t dA = smem_desc(sbase + S::A_BYTES + S::B_BYTES, 0, 128, SWZ_NONE);
+      const uint64_t dB = smem_desc(sbase + S::A_BYTES + S::B_BYTES + S::SFA_BYTES, 0, 128, SWZ_NONE);
       constexpr uint64_t kStage = S::STAGE >> 4;
+      constexpr int KH = KB / 2;
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         for (int ks = 0; ks < nks; ++ks) {
-          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, is_a ? 0x208 : 0x209))) break;
+          if (!(ok = wait_bounded(bar_full + 8 * s, ph, guard, h == 0 ? 0x208 : 0x209))) break;
           tc_fence_after();
-          const uint64_t d = d0 + kStage * s;
           const int kv = min(KB, kblk - KB * ks);
-          if (is_a) {
-            const uint32_t ca = tmem + S::SFA_COL + KB * 4 * s;
+          const uint32_t ca = tmem + S::SFA_COL + KB * 4 * s;
+          const uint32_t cb = tmem + S::SFB_COL + KB * 8 * s;
 #pragma unroll
-            for (int kb = 0; kb < KB; ++kb)
-              if (kb < kv) tmem_cp_32x128b_warpx4(ca + 4 * kb, d + 32 * kb);
-          } else {
-            const uint32_t cb = tmem + S::SFB_COL + KB * 8 * s;
-#pragma unroll
-            for (int kb = 0; kb < KB; ++kb)
-              if (kb < kv) {
-                tmem_cp_32x128b_warpx4(cb + 8 * kb, d + 32 * kb);
-                tmem_cp_32x128b_warpx4(cb + 8 * kb + 4, d + 32 * (KB + kb));
-              }
+          for (int i = 0; i < KH; ++i) {
+            const int kb = h * KH + i;
+            if (kb < kv) {
+              tmem_cp_32x128b_warpx4(ca + 4 * kb, dA + kStage * s + 32 * kb);
+              tmem_cp_32x128b_warpx4(cb + 8 * kb, dB + kStage * s + 32 * kb);
+              tmem_cp_32x128b_warpx4(cb + 8 * kb + 4, dB + kStage * s + 32 * (KB + kb));
+            }
           }
           tc_commit(ready + 8 * s);
           if (++s == NST) { s = 0; ph ^= 1; }
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         }
       }
       // this warp's copies have completed before tensor memory is freed
-      const uint32_t drain = bar_sf_drain + (is_a ? 0 : 8);
+      const uint32_t drain = bar_sf_drain + 8 * h;
       tc_commit(drain);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < p.timeout_ns) {
