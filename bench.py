@@ -51,6 +51,9 @@ def parse():
                     help="also time the same single-layer workload at r = 0, alternating with it this "
                          "many times (each of --steps steps), and report the low-rank branch's "
                          "overhead t(r) / t(0) - 1 as median and range")
+    ap.add_argument("--chain", action="store_true",
+                    help="multi-layer workloads: run each fc1 -> fc2 pair with fc2's activation side fused "
+                         "into fc1's GEMM epilogue (svdq_w4a4_gemm_lowrank_up_chain)")
     ap.add_argument("--int4-f16", action="store_true",
                     help="INT4 workloads: kernel 2 as one fp16 GEMM of the dequantised operands "
                          "(SVDQ_INT4_F16) instead of int8 MMAs")
@@ -383,14 +386,36 @@ def run_ours(args, layers):
         flush_w.zero_()
         flush_r.sum()
 
-    def run_layers(evs=None):
+    # the step as a list of kernel launches (name, call); with --chain an
+    # fc1 -> fc2 pair is fc1's activation kernel, the fused GEMM and fc2's GEMM
+    fused = set()
+    if args.chain:
         for i, d in enumerate(L):
-            d["h"].quantize_act_lowrank_down(d["x"], d["layer"].M, d["codes"], d["scales"], d["t"])
+            if d["chained"] and L[i - 1]["layer"].variant == W.NVFP4 and d["layer"].variant == W.NVFP4:
+                fused.add(i - 1)
+    launches = []
+    for i, d in enumerate(L):
+        pre = d["layer"].name + "." if len(L) > 1 else ""
+        if i - 1 in fused:      # fc2 of a fused pair: its activation side came from fc1's GEMM
+            launches.append((pre + "w4a4_gemm_lowrank_up", lambda d=d: d["h"].w4a4_gemm_lowrank_up(
+                d["codes"], d["scales"], d["t"], d["layer"].M, d["y"])))
+            continue
+        launches.append((pre + "quantize_act_lowrank_down", lambda d=d: d["h"].quantize_act_lowrank_down(
+            d["x"], d["layer"].M, d["codes"], d["scales"], d["t"])))
+        if i in fused:
+            d2 = L[i + 1]
+            launches.append((pre + "w4a4_gemm_lowrank_up_chain", lambda d=d, d2=d2: svdq.gemm_lowrank_up_chain(
+                d["h"], d["codes"], d["scales"], d["t"], d["layer"].M, None, d2["h"], d2["codes"], d2["scales"],
+                d2["t"])))
+        else:
+            launches.append((pre + "w4a4_gemm_lowrank_up", lambda d=d: d["h"].w4a4_gemm_lowrank_up(
+                d["codes"], d["scales"], d["t"], d["layer"].M, d["y"])))
+
+    def run_layers(evs=None):
+        for i, (_, call) in enumerate(launches):
+            call()
             if evs is not None:
-                evs[2 * i + 1].record(stream)
-            d["h"].w4a4_gemm_lowrank_up(d["codes"], d["scales"], d["t"], d["layer"].M, d["y"])
-            if evs is not None:
-                evs[2 * i + 2].record(stream)
+                evs[i + 1].record(stream)
 
     for _ in range(args.warmup):
         flush()
@@ -419,7 +444,7 @@ def run_ours(args, layers):
     clocks.mark(False)
     # timed pass 2: the same steps with an event after every kernel, for the
     # per-kernel durations (the events keep consecutive kernels apart)
-    nk = 2 * len(L)
+    nk = len(launches)
     ev_k = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
@@ -478,7 +503,10 @@ def run_ours(args, layers):
     dl, f16 = L[di]["layer"], L[di]["f16"]
     M, K, N, r = dl.M, dl.K, dl.N, dl.r
     nvfp4 = dl.variant == W.NVFP4
-    ms_kg = per_k[2 * di + 1]
+    names_k = [n for n, _ in launches]
+    pre_d = dl.name + "." if len(L) > 1 else ""
+    kname = pre_d + ("w4a4_gemm_lowrank_up_chain" if di in fused else "w4a4_gemm_lowrank_up")
+    ms_kg = per_k[names_k.index(kname)]
     kg_flops = 2.0 * M * K * N + 2.0 * M * N * r
     achieved = kg_flops / (ms_kg * 1e-3) / 1e12
     ratio = 4.0 if nvfp4 else (1.0 if f16 else 2.0)
@@ -495,11 +523,7 @@ def run_ours(args, layers):
     nominal = 148 * 2 * 128 * 256 * 64 / 128 * sm_mhz * 1e6 / 1e12 / (1.0 if nvfp4 else 2.0)
     traffic_key = args.workload + ("/int4_f16" if f16 else "")
     wl = " + ".join(layer_desc(d["layer"], d["f16"]) for d in L)
-    kernels = {}
-    for i, d in enumerate(L):
-        pre = d["layer"].name + "." if len(L) > 1 else ""
-        kernels[pre + "quantize_act_lowrank_down"] = per_k[2 * i]
-        kernels[pre + "w4a4_gemm_lowrank_up"] = per_k[2 * i + 1]
+    kernels = {n: per_k[i] for i, n in enumerate(names_k)}
     line = {
         "metric": metric_name(args.workload, [d["layer"] for d in L]), "value": value, "unit": "TFLOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -509,6 +533,7 @@ def run_ours(args, layers):
                    "l2": "flushed before every step (256 MB write, then 256 MB read; outside the timed events)",
                    "parallelism": f"replicas x{world}", "tokens_per_step": L[0]["layer"].M * world,
                    "chained": [d["layer"].name for d in L if d["chained"]],
+                   "fused_pairs": [L[i]["layer"].name + "->" + L[i + 1]["layer"].name for i in sorted(fused)],
                    "timing": "ms_per_step: events at step boundaries only (kernels overlap through "
                              "programmatic dependent launch); kernels_ms: a second timed pass with an "
                              "event after every kernel"},
@@ -519,14 +544,14 @@ def run_ours(args, layers):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
                      "traffic": recorded_traffic("w4a4_gemm_lowrank_up", traffic_key),
-                     "peak_source": peak_src, "kernel": f"w4a4_gemm_lowrank_up ({dl.name})",
+                     "peak_source": peak_src, "kernel": kname,
                      "nominal_peak": nominal, "frac_of_nominal": achieved / nominal,
                      "nominal_source": f"{'FP4' if nvfp4 else 'INT8'} dense tcgen05 rate at {sm_mhz:.0f} MHz "
                                        "(128x256x64 per SM per 128 cycles)"},
         "e2e": {"value": job_throughput(world, flops, ms_e2e), "unit": "TFLOPS",
                 "h2d_bytes_per_step": sum(d["layer"].M * d["layer"].K * 2 for d in L),
                 "d2h_bytes_per_step": sum(d["layer"].M * d["layer"].N * 2 for d in L)},
-        "gpu_launches": 2 * len(L) * args.steps,
+        "gpu_launches": len(launches) * args.steps,
         "clocks": clk,
         "kernel_source_hash": kernel_source_hash(),
     }

@@ -34,11 +34,13 @@ namespace svdq {
 
 constexpr int AWQ_THREADS = 256;
 constexpr int AWQ_G = 64;
-constexpr int AWQ_RW = 4;  // weight rows per warp and pass
-// code chunks per lane and row loaded ahead of the arithmetic, and resident
-// CTAs per SM, by tokens per pass (registers: more tokens, more partial sums)
-template <int MT> constexpr int awq_cb() { return MT <= 2 ? 3 : 1; }
-template <int MT> constexpr int awq_ctas() { return MT == 1 ? 2 : 1; }
+// Per tokens-per-pass MT: weight rows per warp and pass (each x' value read
+// from shared memory serves all of them), 16-byte code chunks per lane and
+// row loaded ahead of the arithmetic, and resident CTAs per SM (registers
+// grow with rows x chunks held and with the tokens' partial sums).
+template <int MT> constexpr int awq_rw() { return MT <= 2 ? 4 : 2; }
+template <int MT> constexpr int awq_cb() { return MT == 1 ? 3 : 2; }
+template <int MT> constexpr int awq_ctas() { return MT <= 4 ? 2 : 1; }
 
 // byte `sel` of a, as the fp32 bit pattern 0x4B0000bb (= 2^23 + byte)
 template <int SEL>
@@ -67,11 +69,38 @@ template <int MT>
 __global__ void __launch_bounds__(AWQ_THREADS, awq_ctas<MT>())
     kawq_kernel(AWQParams p) {
   constexpr int AWQ_CB = awq_cb<MT>();
+  constexpr int AWQ_RW = awq_rw<MT>();
   extern __shared__ __align__(16) float xs[];  // [MT][K/32][36]
   const int nck = p.K / 32;                    // 16-byte code chunks per row
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpb = AWQ_THREADS / 32;
   const int gstride = gridDim.x * wpb * AWQ_RW;
+  const int n_first = (blockIdx.x * wpb + warp) * AWQ_RW;
+  // AWQ_CB chunks of each of the RW rows per lane are loaded before any of
+  // them is decoded (up to 12 independent 16-byte loads per lane)
+  uint4 cw[AWQ_CB][AWQ_RW];
+  uint32_t gw[AWQ_CB][AWQ_RW];
+  auto load = [&](int n0, int cb) {
+#pragma unroll
+    for (int c = 0; c < AWQ_CB; ++c) {
+      const int ci = cb + 32 * c + lane;
+#pragma unroll
+      for (int r = 0; r < AWQ_RW; ++r) {
+        const int n = min(n0 + r, p.N - 1);  // rows past N recompute row N-1, never stored
+        if (ci < nck) {
+          cw[c][r] = __ldcs(reinterpret_cast<const uint4*>(p.codes + static_cast<size_t>(n) * (p.K / 2)) + ci);
+          gw[c][r] = __ldg(p.gp + static_cast<size_t>(n) * (p.K / AWQ_G) + ci / 2);
+        } else {
+          cw[c][r] = make_uint4(0u, 0u, 0u, 0u);
+          gw[c][r] = 0u;                    // scale 0: contributes nothing
+        }
+      }
+    }
+  };
+  // the weights are constant: the first chunks are in flight while the
+  // previous kernel of the stream finishes and while x' is staged
+  if (n_first < p.N) load(n_first, 0);
+  bool preloaded = true;
   // x may still be written by the previous kernel of the stream
   griddep_wait();
   griddep_launch_dependents();
@@ -99,48 +128,44 @@ __global__ void __launch_bounds__(AWQ_THREADS, awq_ctas<MT>())
       *reinterpret_cast<float4*>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
     }
     __syncthreads();
-    for (int n0 = (blockIdx.x * wpb + warp) * AWQ_RW; n0 < p.N; n0 += gstride) {
+    for (int n0 = n_first; n0 < p.N; n0 += gstride) {
       float acc[AWQ_RW][MT];
 #pragma unroll
       for (int r = 0; r < AWQ_RW; ++r)
 #pragma unroll
         for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
-      // AWQ_CB chunks of each of the RW rows per lane are loaded before any
-      // of them is decoded (up to 12 independent 16-byte loads per lane)
       for (int cb = 0; cb < nck; cb += 32 * AWQ_CB) {
-        uint4 cw[AWQ_CB][AWQ_RW];
-        uint32_t gw[AWQ_CB][AWQ_RW];
-#pragma unroll
-        for (int c = 0; c < AWQ_CB; ++c) {
-          const int ci = cb + 32 * c + lane;
-#pragma unroll
-          for (int r = 0; r < AWQ_RW; ++r) {
-            const int n = min(n0 + r, p.N - 1);  // rows past N recompute row N-1, never stored
-            if (ci < nck) {
-              cw[c][r] = __ldcs(reinterpret_cast<const uint4*>(p.codes + static_cast<size_t>(n) * (p.K / 2)) + ci);
-              gw[c][r] = __ldg(p.gp + static_cast<size_t>(n) * (p.K / AWQ_G) + ci / 2);
-            } else {
-              cw[c][r] = make_uint4(0u, 0u, 0u, 0u);
-              gw[c][r] = 0u;                    // scale 0: contributes nothing
-            }
-          }
-        }
+        if (!preloaded) load(n0, cb);
+        preloaded = false;
 #pragma unroll
         for (int c = 0; c < AWQ_CB; ++c) {
           const int ci = min(cb + 32 * c + lane, nck - 1);
           const float* xc = xs + ci * 36;
+          uint64_t part[AWQ_RW][MT];
 #pragma unroll
-          for (int r = 0; r < AWQ_RW; ++r) {
-            const float nz = -(8388608.0f + static_cast<float>(gw[c][r] & 0xFFu));
-            const uint64_t nzz = f2_pack(nz, nz);
-            uint64_t part[MT];
+          for (int r = 0; r < AWQ_RW; ++r)
 #pragma unroll
-            for (int m = 0; m < MT; ++m) part[m] = 0ull;
-            const uint32_t words[4] = {cw[c][r].x, cw[c][r].y, cw[c][r].z, cw[c][r].w};
+            for (int m = 0; m < MT; ++m) part[r][m] = 0ull;
 #pragma unroll
-            for (int wi = 0; wi < 4; ++wi) {
-              const uint32_t lo = words[wi] & 0x0F0F0F0Fu;         // codes 8wi + 2b
-              const uint32_t hi = (words[wi] >> 4) & 0x0F0F0F0Fu;  // codes 8wi + 2b + 1
+          for (int wi = 0; wi < 4; ++wi) {
+            // x' of these eight positions, once for all the warp's rows
+            uint64_t xv[MT][4];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              const float4 xa = *reinterpret_cast<const float4*>(xc + m * nck * 36 + 8 * wi);
+              const float4 xb = *reinterpret_cast<const float4*>(xc + m * nck * 36 + 8 * wi + 4);
+              xv[m][0] = f2_pack(xa.x, xa.y);
+              xv[m][1] = f2_pack(xa.z, xa.w);
+              xv[m][2] = f2_pack(xb.x, xb.y);
+              xv[m][3] = f2_pack(xb.z, xb.w);
+            }
+#pragma unroll
+            for (int r = 0; r < AWQ_RW; ++r) {
+              const float nz = -(8388608.0f + static_cast<float>(gw[c][r] & 0xFFu));
+              const uint64_t nzz = f2_pack(nz, nz);
+              const uint32_t word = wi == 0 ? cw[c][r].x : wi == 1 ? cw[c][r].y : wi == 2 ? cw[c][r].z : cw[c][r].w;
+              const uint32_t lo = word & 0x0F0F0F0Fu;         // codes 8wi + 2b
+              const uint32_t hi = (word >> 4) & 0x0F0F0F0Fu;  // codes 8wi + 2b + 1
               uint64_t q[4];
               q[0] = f2_add(f2_pack(__uint_as_float(byte_as_magic<0>(lo)), __uint_as_float(byte_as_magic<0>(hi))), nzz);
               q[1] = f2_add(f2_pack(__uint_as_float(byte_as_magic<1>(lo)), __uint_as_float(byte_as_magic<1>(hi))), nzz);
@@ -148,18 +173,19 @@ __global__ void __launch_bounds__(AWQ_THREADS, awq_ctas<MT>())
               q[3] = f2_add(f2_pack(__uint_as_float(byte_as_magic<3>(lo)), __uint_as_float(byte_as_magic<3>(hi))), nzz);
 #pragma unroll
               for (int m = 0; m < MT; ++m) {
-                const float4 xa = *reinterpret_cast<const float4*>(xc + m * nck * 36 + 8 * wi);
-                const float4 xb = *reinterpret_cast<const float4*>(xc + m * nck * 36 + 8 * wi + 4);
-                part[m] = f2_fma(f2_pack(xa.x, xa.y), q[0], part[m]);
-                part[m] = f2_fma(f2_pack(xa.z, xa.w), q[1], part[m]);
-                part[m] = f2_fma(f2_pack(xb.x, xb.y), q[2], part[m]);
-                part[m] = f2_fma(f2_pack(xb.z, xb.w), q[3], part[m]);
+                part[r][m] = f2_fma(xv[m][0], q[0], part[r][m]);
+                part[r][m] = f2_fma(xv[m][1], q[1], part[r][m]);
+                part[r][m] = f2_fma(xv[m][2], q[2], part[r][m]);
+                part[r][m] = f2_fma(xv[m][3], q[3], part[r][m]);
               }
             }
+          }
+#pragma unroll
+          for (int r = 0; r < AWQ_RW; ++r) {
             const float sc = __uint_as_float(gw[c][r] & 0xFFFF0000u);
 #pragma unroll
             for (int m = 0; m < MT; ++m)
-              acc[r][m] = __fmaf_rn(sc, __fadd_rn(f2_lo(part[m]), f2_hi(part[m])), acc[r][m]);
+              acc[r][m] = __fmaf_rn(sc, __fadd_rn(f2_lo(part[r][m]), f2_hi(part[r][m])), acc[r][m]);
           }
         }
       }

@@ -32,7 +32,11 @@
 // turns writing their X2' values (bf16, 128-byte swizzle, K-major) into one
 // 16 KB shared buffer; after each turn one thread (warp 4, lane 0) issues
 // four bf16 MMAs (M 128, N r2, K 16) with L1_2's slice rows as B, staged per
-// tile by TMA, and commits the buffer back.  Every wait is bounded.
+// tile by TMA, and commits the buffer to the NEXT slice's barrier.  Each
+// slice has its own "buffer free" barrier that completes once per tile, so
+// no waiter is ever more than one phase behind the barrier it polls (with
+// one shared barrier, slices two turns ahead would read the parity of a
+// phase that has not begun as complete).  Every wait is bounded.
 #pragma once
 
 #include "kg_nvfp4.cuh"
@@ -56,7 +60,7 @@ struct KGChainSmem {
   static constexpr int X2_BYTES = 128 * 128;                  // 128 rows x 64 bf16
   static constexpr int L1_OFF = X2_OFF_A + X2_BYTES;
   static constexpr int L1_BYTES = 4 * R2 * 128;               // 4 slices x R2 rows x 64 bf16
-  static constexpr int CBAR_OFF = L1_OFF + L1_BYTES;          // chain barriers
+  static constexpr int CBAR_OFF = L1_OFF + L1_BYTES;          // chain barriers (8 x 8 bytes)
   static constexpr int LUT_OFF = CBAR_OFF + 64;               // E4M3 code -> (value, 1/value)
   static constexpr int TOTAL = LUT_OFF + 128 * 8 + 1024;
   static constexpr int T2_COL = (B::SFB_COL + 8 * B::KB * B::STAGES + 31) / 32 * 32;  // after the scale factors
@@ -93,10 +97,12 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   // chain barriers
   const uint32_t cbar = sbase + C::CBAR_OFF;
   const uint32_t bar_x2_full = cbar;          // a slice's X2' written (128 arrivals)
-  const uint32_t bar_x2_empty = cbar + 8;     // the slice's T2 MMAs have read it (commit)
-  const uint32_t bar_l1_full = cbar + 16;     // the tile's L1_2 rows landed (TMA)
-  const uint32_t bar_t2_drained = cbar + 24;  // T2 accumulator drained (128 arrivals)
-  const uint32_t bar_t2_final = cbar + 32;    // every T2 MMA completed (commit)
+  // bar_x2_free + 8 t: slice t may write the buffer (commit after the MMAs of
+  // the turn before it: slice t - 1's, or the previous tile's slice 3 for t = 0)
+  const uint32_t bar_x2_free = cbar + 8;
+  const uint32_t bar_l1_full = cbar + 40;     // the tile's L1_2 rows landed (TMA)
+  const uint32_t bar_t2_drained = cbar + 48;  // T2 accumulator drained (128 arrivals)
+  const uint32_t bar_t2_final = cbar + 56;    // every T2 MMA completed (commit)
   float2* e4lut = reinterpret_cast<float2*>(smem + C::LUT_OFF);
 
   const int warp = threadIdx.x >> 5;
@@ -126,7 +132,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     mbar_init(bar_sf_drain, 1);
     mbar_init(bar_sf_drain + 8, 1);
     mbar_init(bar_x2_full, 128);
-    mbar_init(bar_x2_empty, 1);
+    for (int t = 0; t < 4; ++t) mbar_init(bar_x2_free + 8 * t, 1);
     mbar_init(bar_l1_full, 1);
     mbar_init(bar_t2_drained, 128);
     mbar_init(bar_t2_final, 1);
@@ -433,10 +439,14 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         *reinterpret_cast<uint32_t*>(sp) = sc;
       }
       // T2 += X2' . L1_2 over this tile's 256 columns: the slices take turns
-      // in the shared buffer (turn t is slice t of this tile)
+      // in the shared buffer (turn t is slice t of this tile).  Slice t's
+      // barrier completes once per tile: for t > 0 this tile's phase j, for
+      // t = 0 the previous tile's (phase j - 1; at j = 0 the preceding phase
+      // of a fresh barrier counts as complete).
       for (int t = 0; t < 4; ++t, ++turn) {
         if (cs == t) {
-          ok = __all_sync(0xffffffffu, wait_bounded(bar_x2_empty, (turn & 1) ^ 1, guard, 0x25d));
+          const uint32_t par = t == 0 ? ((j & 1) ^ 1) : (j & 1);
+          ok = __all_sync(0xffffffffu, wait_bounded(bar_x2_free + 8 * t, par, guard, 0x25d));
           if (ok) {
 #pragma unroll
             for (int j8 = 0; j8 < 8; ++j8)
@@ -457,7 +467,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
               mma_bf16(t2col, dX2 + 2 * kk, dL1 + (t * R2 * 128 >> 4) + 2 * kk, id_t2,
                        (fresh && kk == 0) ? 0u : 1u);
             fresh = false;
-            tc_commit(bar_x2_empty);
+            tc_commit(bar_x2_free + 8 * ((t + 1) & 3));
           }
         }
         __syncwarp();
@@ -468,7 +478,8 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       fresh = __shfl_sync(0xffffffffu, fresh, 0);  // the issuer's view (lane 0 of warp 4)
       if (issuer && tile + 1 < t_end) {
         // L1_2 rows of the next tile, once this tile's T2 MMAs have read them
-        ok = wait_bounded(bar_x2_empty, (turn - 1) & 1, guard, 0x261);
+        // (slice 3's commit is slice 0's barrier, phase j)
+        ok = wait_bounded(bar_x2_free, j & 1, guard, 0x261);
         if (ok) {
           mbar_expect_tx(bar_l1_full, C::L1_BYTES);
           const int nb1 = (tile + 1) % p.num_n;
@@ -482,7 +493,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       if (seg_end) {
         // the row block's T2 accumulation is complete: drain and add into T2
         if (cs == 0) {
-          if (!(ok = __all_sync(0xffffffffu, wait_bounded(bar_x2_empty, (turn - 1) & 1, guard, 0x262)))) break;
+          if (!(ok = __all_sync(0xffffffffu, wait_bounded(bar_x2_free, j & 1, guard, 0x262)))) break;
           tc_fence_after();
           uint32_t tv[R2];
           if constexpr (R2 == 16) tmem_ld_x16(t2col + (static_cast<uint32_t>(q * 32) << 16), tv);

@@ -720,8 +720,8 @@ svdq_status launch_awq(svdq_awq* h, const void* x, void* y, int64_t M, cudaStrea
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(h->K);
   p.N = static_cast<int>(h->N);
-  // persistent: one or two CTAs per SM (x' is staged once per CTA)
-  const int64_t rows_per_cta = (AWQ_THREADS / 32) * AWQ_RW;
+  // persistent: up to three CTAs per SM (x' is staged once per CTA)
+  const int64_t rows_per_cta = (AWQ_THREADS / 32) * awq_rw<MT>();
   const int64_t want = cdiv(h->N, rows_per_cta);
   const int64_t resident = static_cast<int64_t>(awq_ctas<MT>()) * h->sms;
   const int grid = static_cast<int>(want < resident ? want : resident);
@@ -1212,6 +1212,13 @@ svdq_status svdq_device_status(svdq_weights_t h, void* stream) {
     if (h->kq_counters) cudaMemset(h->kq_counters, 0, cdiv(h->max_M, 128) * 4);
     return e == 0x34f ? SVDQ_ERR_RANGE : SVDQ_ERR_DEVICE_TIMEOUT;
   }
+  return SVDQ_OK;
+}
+
+svdq_status svdq_device_error_site(svdq_weights_t h, void* stream, int* site) {
+  if (!h || !site) return SVDQ_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (cudaMemcpy(site, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SVDQ_ERR_CUDA;
   return SVDQ_OK;
 }
 

@@ -36,7 +36,7 @@ EXPORTED = [
     "svdq_awq_load", "svdq_awq_free", "svdq_awq_w4a16_forward",
     "svdq_prep_calibrate", "svdq_prep_lowrank", "svdq_prep_residual_quantize",
     "svdq_w4a4_gemm_lowrank_up_qkv", "svdq_linear_forward_qkv",
-    "svdq_w4a4_gemm_lowrank_up_chain", "svdq_linear_forward_chain",
+    "svdq_w4a4_gemm_lowrank_up_chain", "svdq_linear_forward_chain", "svdq_device_error_site",
 ]
 
 
@@ -96,6 +96,7 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
     L.svdq_w4a4_gemm_lowrank_up_qkv.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp]
     L.svdq_w4a4_gemm_lowrank_up_chain.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp]
     L.svdq_linear_forward_chain.argtypes = [vp, vp, vp, vp, i64, vp]
+    L.svdq_device_error_site.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int)]
     L.svdq_linear_forward_qkv.argtypes = [vp, vp, vp, vp, i64, vp]
     L.svdq_awq_load.argtypes = [ctypes.POINTER(AWQDesc), ctypes.POINTER(vp), vp]
     L.svdq_awq_free.argtypes = [vp]
@@ -226,6 +227,13 @@ class SVDQWeights:
 
     def device_status(self, stream=None) -> int:
         return int(self._lib.svdq_device_status(self.handle, _stream(stream)))
+
+    def device_error_site(self, stream=None) -> int:
+        """Wait-site code of the first expired bounded wait (0 if none)."""
+        v = ctypes.c_int(0)
+        _check(self._lib.svdq_device_error_site(self.handle, _stream(stream), ctypes.byref(v)),
+               "svdq_device_error_site")
+        return int(v.value)
 
     def debug_set_fault(self, mask: int, timeout_us: int) -> None:
         _check(self._lib.svdq_debug_set_fault(self.handle, mask, timeout_us), "svdq_debug_set_fault")

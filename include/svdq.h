@@ -421,6 +421,15 @@ svdq_status svdq_prep_residual_quantize(svdq_variant variant, const void* w, con
 svdq_status svdq_device_status(svdq_weights_t h, void* stream);
 
 /*
+ * Failure reporting (no counterpart on the pages): the wait-site code of the
+ * first bounded wait that expired in a call on this handle since the last
+ * svdq_device_status (0 if none), without clearing it.  The codes identify
+ * the kernel and the wait inside it; they are for diagnosis only.
+ * Synchronises `stream`.
+ */
+svdq_status svdq_device_error_site(svdq_weights_t h, void* stream, int* site);
+
+/*
  * Test hook (no counterpart on the pages): make the next launches wait on a
  * pipeline stage that is never filled (mask bit 0: GEMM producer skips one stage; bit 1: activation
  * kernel producer skips one stage) and use `timeout_us` as the bounded-wait

@@ -105,7 +105,10 @@ def quantize_act_lowrank_down(x_bits, inv_lam, L1_bits, variant):
 def gelu_tanh(x):
     """GELU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))."""
     x = np.asarray(x, dtype=np.float64)
-    return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
+    # x^3 overflows to +-inf for |x| > ~1e102; tanh(+-inf) = +-1 gives the
+    # limits x and 0, so the overflow is harmless and not reported
+    with np.errstate(over="ignore"):
+        return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
 
 
 def gemm_lowrank_up(codes, scales, T, w_codes, w_scales, L2_bits, variant,

@@ -381,3 +381,150 @@ def test_pair_copy_warps_skipping_low_rank_stages_is_caught():
         res = m.run()
         bad += res != "ok" or bool(m.errors)
     assert bad > 0
+
+
+class ChainModel:
+    """The fused MLP pair's epilogue hand-off (fc2's T2 = X2 . L1_2 on the
+    tensor cores): 16 epilogue warps in four 64-column slices of four warps;
+    each tile, the slices take turns writing their X2 rows into one shared
+    buffer (x2_full: four warp arrivals per turn); warp 4 (slice 0) also
+    holds the issuing thread, which waits for the tile's L1_2 rows (TMA) and
+    each turn's rows, issues the turn's MMAs into the T2 accumulator (fresh
+    at a row block's first MMA) and commits the buffer back; it reloads L1_2
+    once the tile's MMAs have read it.  At the end of a row-block segment the
+    four warps of slice 0 drain T2 (t2_drained) before the next segment's
+    first MMA may overwrite it.  `shared_free` plants the single "buffer
+    free" barrier that let slices two turns ahead pass on a stale parity."""
+
+    def __init__(self, t_begin, t_end, num_n, rng, shared_free=False):
+        self.t_begin, self.t_end, self.num_n = t_begin, t_end, num_n
+        self.rng, self.shared = rng, shared_free
+        self.errors = []
+        e = self.errors
+        self.x2_full = MBar(4, e)
+        self.x2_free = [MBar(1, e) for _ in range(1 if shared_free else 4)]
+        self.l1_full = MBar(1, e)
+        self.t2_drained = MBar(4, e)
+        self.buf = [None] * 4        # (tile, slice) whose rows each lane quarter wrote
+        self.l1 = None               # tile whose L1_2 rows are staged
+        self.t2 = set()              # (tile, slice) products accumulated in T2
+        self.tma_ops = []
+        self.tc_ops = []
+
+    def seg_end(self, tile):
+        return tile + 1 == self.t_end or (tile + 1) // self.num_n != tile // self.num_n
+
+    def free_bar(self, t):
+        return self.x2_free[0] if self.shared else self.x2_free[t]
+
+    def load_l1(self, tile):
+        def land():
+            self.l1 = tile
+            self.l1_full.complete_tx(1)
+        self.l1_full.arrive(expect_tx=1)
+        self.tma_ops.append(land)
+
+    def warp(self, cs, q):
+        issuer = cs == 0 and q == 0
+        turn, seg, fresh = 0, 0, True
+        if issuer and self.t_begin < self.t_end:
+            self.load_l1(self.t_begin)
+        for j, tile in enumerate(range(self.t_begin, self.t_end)):
+            for t in range(4):
+                if cs == t:
+                    if self.shared:
+                        yield ("wait", self.x2_free[0], (turn & 1) ^ 1)
+                    else:
+                        yield ("wait", self.x2_free[t], ((j & 1) ^ 1) if t == 0 else (j & 1))
+                    self.buf[q] = (tile, t)
+                    self.x2_full.arrive()
+                if issuer:
+                    if t == 0:
+                        yield ("wait", self.l1_full, j & 1)
+                        if fresh and seg > 0:
+                            yield ("wait", self.t2_drained, (seg - 1) & 1)
+                    yield ("wait", self.x2_full, turn & 1)
+                    f = fresh
+
+                    def mma(tile=tile, t=t, f=f):
+                        if self.buf != [(tile, t)] * 4:
+                            self.errors.append(f"T2 MMA of tile {tile} slice {t} read rows {self.buf}")
+                        if self.l1 != tile:
+                            self.errors.append(f"T2 MMA of tile {tile} read L1_2 of tile {self.l1}")
+                        if f:
+                            self.t2 = set()
+                        self.t2.add((tile, t))
+                        self.free_bar((t + 1) & 3).arrive()
+                    self.tc_ops.append(mma)
+                    fresh = False
+                turn += 1
+            if issuer and tile + 1 < self.t_end:
+                if self.shared:
+                    yield ("wait", self.x2_free[0], (turn - 1) & 1)
+                else:
+                    yield ("wait", self.x2_free[0], j & 1)
+                self.load_l1(tile + 1)
+            if self.seg_end(tile):
+                if cs == 0:
+                    if self.shared:
+                        yield ("wait", self.x2_free[0], (turn - 1) & 1)
+                    else:
+                        yield ("wait", self.x2_free[0], j & 1)
+                    mb = tile // self.num_n
+                    want = {(x, s) for x in range(self.t_begin, tile + 1) if x // self.num_n == mb
+                            for s in range(4)}
+                    if self.t2 != want:
+                        self.errors.append(f"drain of row block {mb} read {sorted(self.t2)}")
+                    self.t2_drained.arrive()
+                seg += 1
+                fresh = True
+
+    def run(self):
+        agents = [self.warp(cs, q) for cs in range(4) for q in range(4)]
+        blocked = {i: None for i in range(len(agents))}
+        live = set(range(len(agents)))
+        steps = 0
+        while live or self.tma_ops or self.tc_ops:
+            steps += 1
+            if steps > 200000:
+                return "livelock"
+            runnable = [i for i in live if blocked[i] is None or blocked[i][0].try_wait(blocked[i][1])]
+            choices = runnable + (["tma"] if self.tma_ops else []) + (["tc"] if self.tc_ops else [])
+            if not choices:
+                return "deadlock"
+            c = self.rng.choice(choices)
+            if c == "tma":
+                self.tma_ops.pop(self.rng.randrange(len(self.tma_ops)))()
+                continue
+            if c == "tc":
+                self.tc_ops.pop(0)()   # the issuer's MMAs and commits complete in order
+                continue
+            blocked[c] = None
+            try:
+                op = next(agents[c])
+                blocked[c] = (op[1], op[2])
+            except StopIteration:
+                live.discard(c)
+        return "ok"
+
+
+CHAIN_CONFIGS = [(t0, n, nn) for nn in (1, 2, 3) for t0 in (0, 1, 2) for n in (1, 2, 4, 5)]
+
+
+@pytest.mark.parametrize("t0,n,num_n", CHAIN_CONFIGS)
+def test_chain_slice_handoff_is_safe(t0, n, num_n):
+    for seed in range(12):
+        m = ChainModel(t0, t0 + n, num_n, random.Random(seed))
+        assert m.run() == "ok"
+        assert not m.errors, m.errors[:3]
+
+
+def test_chain_single_free_barrier_is_caught():
+    """Planted mistake: one shared "buffer free" barrier; slices two turns
+    ahead read the parity of a phase that has not begun as complete."""
+    bad = 0
+    for seed in range(40):
+        m = ChainModel(0, 2, 2, random.Random(seed), shared_free=True)
+        res = m.run()
+        bad += res != "ok" or bool(m.errors)
+    assert bad > 0
