@@ -35,16 +35,25 @@ namespace svdq {
 constexpr int KGI4_BN = 128;   // tile columns (output features)
 constexpr int KGI4_BUFS = 4;   // s32 accumulators of 128 columns in tensor memory
 
+constexpr int KGI4_GC = 16;    // groups per staged chunk of scales
+
 template <int R>
 struct KGI4Smem {
-  static constexpr int STAGES = R >= 128 ? 8 : (R >= 64 ? 9 : 10);
+  static constexpr int STAGES = R >= 128 ? 6 : (R >= 64 ? 8 : 9);
   static constexpr int APK_BYTES = KG_BM * 32;    // 128 rows x 32 B packed (64 codes)
   static constexpr int A8_BYTES = KG_BM * 64;     // 128 rows x 64 int8
   static constexpr int B_BYTES = KGI4_BN * 64;    // 128 rows x 64 int8
   static constexpr int STAGE = APK_BYTES + A8_BYTES + B_BYTES;
   static constexpr int LR_CHUNKS = R > 0 ? (2 * R + 63) / 64 : 0;
   static constexpr int ALR_OFF = STAGES * STAGE;
-  static constexpr int BAR_OFF = ALR_OFF + LR_CHUNKS * 16384;
+  // scale chunks, two buffers: the tile's weight scales [GC][128] fp32 and
+  // activation scales [128 rows][GC] bf16 at a 36-byte row pitch (9 words:
+  // the 32 rows a warp reads fall in 32 distinct banks)
+  static constexpr int SW_BYTES = KGI4_GC * KGI4_BN * 4;
+  static constexpr int SX_PITCH = KGI4_GC * 2 + 4;
+  static constexpr int SC_BUF = SW_BYTES + KG_BM * SX_PITCH;
+  static constexpr int SC_OFF = ALR_OFF + LR_CHUNKS * 16384;
+  static constexpr int BAR_OFF = SC_OFF + 2 * SC_BUF;
   static constexpr int TOTAL = BAR_OFF + 512 + 1024;
   static_assert(STAGE % 1024 == 0, "stages keep the swizzle alignment");
   static_assert(TOTAL <= 232448, "shared memory per CTA");
@@ -81,7 +90,9 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
   const uint32_t bar_gempty = smem_u32(bars + 3 * NST + KGI4_BUFS);     // [KGI4_BUFS]
   const uint32_t bar_lr_full = smem_u32(bars + 3 * NST + 2 * KGI4_BUFS);
   const uint32_t bar_drain = smem_u32(bars + 3 * NST + 2 * KGI4_BUFS + 1);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NST + 2 * KGI4_BUFS + 2);
+  const uint32_t bar_sc_full = smem_u32(bars + 3 * NST + 2 * KGI4_BUFS + 2);  // [2]
+  const uint32_t bar_sc_free = smem_u32(bars + 3 * NST + 2 * KGI4_BUFS + 4);  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * NST + 2 * KGI4_BUFS + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -102,6 +113,10 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     }
     mbar_init(bar_lr_full, KG_EPI_WARPS * 32);
     mbar_init(bar_drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_sc_full + 8 * b, KG_EPI_WARPS * 32);  // one cp.async arrival per epilogue thread
+      mbar_init(bar_sc_free + 8 * b, KG_EPI_WARPS);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -260,6 +275,36 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
     const __nv_bfloat16* sx_all = reinterpret_cast<const __nv_bfloat16*>(p.sfa);
     const float* sw_all = reinterpret_cast<const float*>(p.sfb);
     const int npad = (p.N + 255) / 256 * 256;  // row stride of the weight-scale table
+    const int nchunk = (ng + KGI4_GC - 1) / KGI4_GC;
+    // Scales of a tile come in chunks of GC groups, staged by all epilogue
+    // threads with cp.async one chunk ahead of their use: chunk u goes to
+    // buffer u & 1 once the 16 warps have released that buffer's previous
+    // chunk (u - 2), and its barrier completes when every thread's copies
+    // have landed.  Zero fill past M and past the last group.
+    auto stage = [&](int tile, int c, uint32_t u) -> bool {
+      const uint32_t b = u & 1, k = u >> 1;
+      if (!__all_sync(0xffffffffu, wait_bounded(bar_sc_free + 8 * b, (k & 1) ^ 1, guard, 0x30e))) return false;
+      const uint32_t buf = sbase + S::SC_OFF + b * S::SC_BUF;
+      const int mb = tile % p.num_m, nb = tile / p.num_m;
+      const int g0 = c * KGI4_GC;
+      {  // weight scales: GC rows of 512 contiguous bytes, one 16-byte piece per thread
+        const int gi = etid >> 5, c4 = etid & 31;
+        const bool in = g0 + gi < ng;
+        const float* src = sw_all + static_cast<size_t>(in ? g0 + gi : 0) * npad + nb * KGI4_BN + 4 * c4;
+        cp_async_16(buf + gi * (KGI4_BN * 4) + 16 * c4, src, in ? 16u : 0u);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // activation scales: 128 rows x GC/2 words, two per thread
+        const int it = etid + 512 * h;
+        const int r = it >> 3, w = it & 7;
+        const int gm = mb * KG_BM + r;
+        const bool in = gm < p.M && g0 + 2 * w < ng;  // ng is even: a word is both groups or neither
+        const __nv_bfloat16* src = sx_all + (in ? static_cast<size_t>(gm) * ng + g0 + 2 * w : 0);
+        cp_async_4(buf + S::SW_BYTES + r * S::SX_PITCH + 4 * w, src, in ? 4u : 0u);
+      }
+      cp_async_mbar_arrive(bar_sc_full + 8 * b);
+      return true;
+    };
     if constexpr (R > 0) {
       if (static_cast<int>(blockIdx.x) < num_tiles) {
         prep_lowrank_a<R>(alr, p.t, (blockIdx.x % p.num_m) * KG_BM, p.M, etid);
@@ -268,27 +313,36 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       }
     }
     uint32_t gc = 0;
-    bool ok = true;
+    uint32_t u = 0;  // scale chunks consumed so far
+    bool ok = static_cast<int>(blockIdx.x) >= num_tiles || stage(blockIdx.x, 0, 0);
     for (int tile = blockIdx.x, j = 0; tile < num_tiles && ok; tile += gridDim.x, ++j) {
       const int mb = tile % p.num_m, nb = tile / p.num_m;
-      const int gm = mb * KG_BM + row;
       const int n_base = nb * KGI4_BN + cs * 32;
-      const __nv_bfloat16* sxr = sx_all + static_cast<size_t>(gm < p.M ? gm : 0) * ng;
       uint64_t acc[16];  // 32 fp32 sums, in pairs
 #pragma unroll
       for (int i = 0; i < 16; ++i) acc[i] = 0ull;
-      float sx_next = gm < p.M ? __bfloat162float(sxr[0]) : 0.0f;
       const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16) + cs * 32;
       // float(P) for the s32 group product P (a sum of 64 products of 4-bit
       // codes, |P| <= 4096 < 2^22): bits(P + bits(1.5 * 2^23)) - 1.5 * 2^23,
       // exact, at the full rate of integer and fp32 adds
       const uint64_t mag = f2_pack(-12582912.0f, -12582912.0f);
+      const uint8_t* scb = nullptr;
       for (int g = 0; g < ng; ++g, ++gc) {
+        const int gi = g % KGI4_GC;
+        if (gi == 0) {
+          // the next chunk (this tile's, or the next tile's first) into the other buffer
+          const int c = g / KGI4_GC;
+          if (c + 1 < nchunk) ok = stage(tile, c + 1, u + 1);
+          else if (tile + static_cast<int>(gridDim.x) < num_tiles) ok = stage(tile + gridDim.x, 0, u + 1);
+          if (!ok) break;
+          if (!(ok = __all_sync(0xffffffffu, wait_bounded(bar_sc_full + 8 * (u & 1), (u >> 1) & 1, guard, 0x30f))))
+            break;
+          scb = smem + S::SC_OFF + (u & 1) * S::SC_BUF;
+        }
         const uint32_t b = gc % KGI4_BUFS, use = gc / KGI4_BUFS;
-        const float sx = sx_next;
-        if (g + 1 < ng) sx_next = gm < p.M ? __bfloat162float(sxr[g + 1]) : 0.0f;
+        const float sx = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(scb + S::SW_BYTES + row * S::SX_PITCH + 2 * gi));
         const uint64_t sx2 = f2_pack(sx, sx);
-        const float4* swr = reinterpret_cast<const float4*>(sw_all + static_cast<size_t>(g) * npad + n_base);
+        const float4* swr = reinterpret_cast<const float4*>(scb + gi * (KGI4_BN * 4) + cs * 128);
         if (!(ok = __all_sync(0xffffffffu, wait_bounded(bar_gfull + 8 * b, use & 1, guard, 0x30a)))) break;
         tc_fence_after();
         uint32_t v[32];
@@ -300,7 +354,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
         // acc += (s_x * s_w[n]) * P[n], two columns per instruction
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 w = __ldg(swr + i4);
+          const float4 w = swr[i4];
           const uint64_t s01 = f2_mul(sx2, f2_pack(w.x, w.y));
           const uint64_t s23 = f2_mul(sx2, f2_pack(w.z, w.w));
           const uint64_t p01 = f2_add(f2_pack(__uint_as_float(v[4 * i4] + 0x4B400000u),
@@ -309,6 +363,12 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
                                               __uint_as_float(v[4 * i4 + 3] + 0x4B400000u)), mag);
           acc[2 * i4] = f2_fma(p01, s01, acc[2 * i4]);
           acc[2 * i4 + 1] = f2_fma(p23, s23, acc[2 * i4 + 1]);
+        }
+        if (gi == KGI4_GC - 1 || g == ng - 1) {
+          // this warp is done with the chunk's buffer
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_sc_free + 8 * (u & 1));
+          ++u;
         }
       }
       if (!ok) break;
@@ -343,6 +403,7 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       }
       store_rows32_coalesced(p, mb * KG_BM + q * 32, n_base, out, lane);
     }
+    cp_async_wait_all();  // no copy into this CTA's shared memory outlives it
   }
 
   tc_fence_before();
