@@ -148,21 +148,18 @@ __global__ void prep_gram_f64_kernel(const float* __restrict__ Y, int64_t rows, 
   }
 }
 
-// Y[rows x l] := Y . T for a small T [l x l] (fp64, row-major), in place:
-// a thread per row (the row is read fully before it is written).
-__global__ void prep_rmul_small_kernel(float* __restrict__ Y, int64_t rows, int l, const double* __restrict__ T) {
-  extern __shared__ double ts[];
-  for (int e = threadIdx.x; e < l * l; e += blockDim.x) ts[e] = T[e];
-  __syncthreads();
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= rows) return;
-  double row[64];
-  for (int a = 0; a < l; ++a) row[a] = Y[i * l + a];
-  for (int b = 0; b < l; ++b) {
-    double s = 0.0;
-    for (int a = 0; a < l; ++a) s = fma(row[a], ts[a * l + b], s);
-    Y[i * l + b] = static_cast<float>(s);
-  }
+// Yo[rows x l] = Y . T for a small T [l x l] (fp64, row-major), out of
+// place: a thread per output element; T's row a is read by a whole warp at
+// once (one broadcast load per step) through the read-only cache.
+__global__ void prep_rmul_small_kernel(const float* __restrict__ Y, int64_t rows, int l,
+                                       const double* __restrict__ T, float* __restrict__ Yo) {
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= rows * l) return;
+  const int64_t i = e / l;
+  const int b = static_cast<int>(e % l);
+  double s = 0.0;
+  for (int a = 0; a < l; ++a) s = fma(static_cast<double>(Y[i * l + a]), __ldg(T + a * l + b), s);
+  Yo[e] = static_cast<float>(s);
 }
 
 // --------------------------------------------------- residual quantisation

@@ -12,9 +12,13 @@
 //
 // CTA tile: 128 tokens x (K / ksplit) input channels.  The K range of a row
 // block is split over `ksplit` CTAs so that a 4608-token layer still fills
-// the 148 SMs in one wave; their partial T tiles go to a scratch buffer and
-// the last CTA of the row block to finish sums them in split order
-// (deterministic), with a per-block arrival counter that it resets.
+// the 148 SMs in one wave.  Their partial T tiles are added into T with
+// fp32 vector reductions (split 0 clears the row block's T at its start and
+// raises a per-launch flag that the others check before adding), or -- for
+// the entry point
+// that allocates nothing and keeps T deterministic -- go to a scratch buffer
+// that the last CTA of the row block to finish sums in split order, with a
+// per-block arrival counter that it resets.
 //
 // Warp roles (576 threads):
 //   warps 0-15 quantisers, one token row per thread; warp w covers rows
@@ -114,6 +118,12 @@ struct KQParams {
   float* t;              // [M x R]
   float* tpart;          // scratch: partial T tiles [ksplit x num_m x 128 x R] (ksplit > 1)
   int* counters;         // scratch: arrivals per 128-row block, zero between launches
+  int t_accumulate;      // ksplit > 1: add the partial tiles into T with fp32
+                         // reductions instead of the scratch pass; split 0 of a row
+                         // block zeroes its rows of T first and publishes
+                         // tflags[row block] = epoch, which the other splits await
+  unsigned int* tflags;  // [row blocks]
+  unsigned int epoch;    // nonzero, new for every launch on the same flags
   int M, K, ksplit, chunks;  // chunks of 64 columns per CTA
   int* err;
   uint32_t debug_mask;
@@ -122,13 +132,23 @@ struct KQParams {
 
 template <int VARIANT, int R>
 struct KQSmem {
-  static constexpr int STAGES = R <= 32 ? 8 : (R == 64 ? 7 : 6);
   static constexpr int X_BYTES = 128 * KQ_CHUNK * 2;  // 16 KB
   static constexpr int L_BYTES = R * KQ_CHUNK * 2;    // r x 128 B
   static constexpr int IL_BYTES = KQ_CHUNK * 4;       // 1/lambda for the chunk
-  static constexpr int STAGE = X_BYTES + L_BYTES + 1024;  // 1/lambda padded to keep 1 KB alignment
-  static constexpr int BAR_OFF = STAGES * STAGE;
+  // a stage holds the X and L1^T tiles (1 KB multiples, so every stage keeps
+  // the 128-byte swizzle's alignment); the chunk's 1/lambda sits in a ring
+  // of its own.  As many stages as shared memory holds (static shared
+  // memory -- the E4M3 table and the reduction flag -- takes up to 2 KB once
+  // the 1 KB-aligned dynamic region follows it): a CTA's chunks are mostly in
+  // flight at once.
+  static constexpr int STAGE = X_BYTES + L_BYTES;
+  static constexpr int FREE = 232448 - 2048 - 512 - 1024;
+  static constexpr int STAGES = FREE / (STAGE + IL_BYTES) < 16 ? FREE / (STAGE + IL_BYTES) : 16;
+  static constexpr int IL_OFF = STAGES * STAGE;
+  static constexpr int BAR_OFF = IL_OFF + STAGES * IL_BYTES;
   static constexpr int TOTAL = BAR_OFF + 512 + 1024;  // barriers + slack for 1 KB alignment
+  static_assert(TOTAL + 2048 <= 232448, "shared memory per CTA");
+  static_assert(STAGES * 3 + 2 <= 64, "barriers");
 };
 
 // 1/6 and 1/7 rounded to nearest: scale = amax / 6 (NVFP4) or amax / 7 (INT4)
@@ -194,6 +214,17 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
   // the outputs may still be read by it: see griddep_wait()
   griddep_wait();
   griddep_launch_dependents();
+  if (R > 0 && p.t_accumulate && ks == 0 && warp == MMA) {
+    // split 0 clears the row block's T (read by the previous kernel of the
+    // stream until griddep_wait) before any split adds into it: the MMA
+    // warp, idle until the first chunk is quantised, does it
+    const int rows = min(128, p.M - m0);
+    float4* dst = reinterpret_cast<float4*>(p.t + static_cast<size_t>(m0) * R);
+    for (int i = lane; i < rows * (R / 4); i += 32) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) st_release_gpu(p.tflags + blockIdx.y, p.epoch);
+  }
 
   if (warp == PRODUCER) {
     // ---------------------------------------------------------------- producer
@@ -212,7 +243,7 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
         mbar_expect_tx(bar_full + 8 * s, S::X_BYTES + S::L_BYTES + S::IL_BYTES);
         tma_load_2d(st, &tm_x, bar_full + 8 * s, k0, m0);
         if (R > 0) tma_load_2d(st + S::X_BYTES, &tm_l1t, bar_full + 8 * s, k0, 0);
-        bulk_load(st + S::X_BYTES + S::L_BYTES, p.inv_lam + k0, S::IL_BYTES, bar_full + 8 * s);
+        bulk_load(sbase + S::IL_OFF + s * S::IL_BYTES, p.inv_lam + k0, S::IL_BYTES, bar_full + 8 * s);
         issued |= 1u << s;
         issued_par = (issued_par & ~(1u << s)) | (ph << s);
       }
@@ -267,7 +298,7 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
       const uint32_t ph = (c / NST) & 1;
       if (!wait_bounded(bar_full + 8 * s, ph, guard, 0x104)) break;
       uint8_t* xt = smem + s * S::STAGE;
-      const float4* il = reinterpret_cast<const float4*>(xt + S::X_BYTES + S::L_BYTES);
+      const float4* il = reinterpret_cast<const float4*>(smem + S::IL_OFF + s * S::IL_BYTES);
       const int k0 = kbase + c * KQ_CHUNK;
       // 64 bf16 of this row (de-swizzled), smoothed: x' = bf16(x * inv_lambda)
       uint32_t w[32];
@@ -407,8 +438,26 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
     if (warp < 4) {  // one warp per 32-lane group of tensor memory
       const int row = warp * 32 + lane;
       const int grow = m0 + row;
-      const bool ok = wait_bounded(bar_tfull, 0, guard, 0x105);
+      bool ok = wait_bounded(bar_tfull, 0, guard, 0x105);
       if (ok) tc_fence_after();
+      if (p.ksplit > 1 && p.t_accumulate && ks != 0) {
+        // split 0 has cleared this row block's T (long ago, in practice)
+        bool seen = true;
+        if (lane == 0) {
+          const uint64_t t0 = global_timer_ns();
+          while (ld_acquire_gpu(p.tflags + blockIdx.y) != p.epoch) {
+            if (*abort_flag || global_timer_ns() - t0 > p.timeout_ns) {
+              if (!*abort_flag) {
+                *abort_flag = 1;
+                atomicCAS(p.err, 0, 0x106);
+              }
+              seen = false;
+              break;
+            }
+          }
+        }
+        ok = ok && __shfl_sync(0xffffffffu, seen, 0);
+      }
       const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
       // stream the row's R fp32 values out of tensor memory 16 or 32 columns at a time
       constexpr int CW = R < 32 ? R : 32;
@@ -421,18 +470,28 @@ __global__ void __launch_bounds__(KQ_THREADS, 1)
           tmem_ld_wait();
         }
         if (ok && grow < p.M) {
-          float* drow = p.ksplit == 1
-                            ? p.t + static_cast<size_t>(grow) * R
-                            : p.tpart + ((static_cast<size_t>(ks) * num_m + blockIdx.y) * 128 + row) * R;
-          float4* dst = reinterpret_cast<float4*>(drow + c0);
+          if (p.ksplit > 1 && p.t_accumulate) {
+            // the split partials meet in T itself (fire-and-forget vector
+            // reductions; their order across the splits is not fixed)
+            float4* dst = reinterpret_cast<float4*>(p.t + static_cast<size_t>(grow) * R + c0);
 #pragma unroll
-          for (int j = 0; j < CW / 4; ++j)
-            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+            for (int j = 0; j < CW / 4; ++j)
+              atomicAdd(dst + j, make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+          } else {
+            float* drow = p.ksplit == 1
+                              ? p.t + static_cast<size_t>(grow) * R
+                              : p.tpart + ((static_cast<size_t>(ks) * num_m + blockIdx.y) * 128 + row) * R;
+            float4* dst = reinterpret_cast<float4*>(drow + c0);
+#pragma unroll
+            for (int j = 0; j < CW / 4; ++j)
+              dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          }
         }
       }
     }
-    if (p.ksplit > 1) {
+    if (p.ksplit > 1 && !p.t_accumulate) {
       // The last split CTA of this row block to arrive sums the partial tiles
       // in split order (deterministic) and resets the block's counter.
       __shared__ int last;

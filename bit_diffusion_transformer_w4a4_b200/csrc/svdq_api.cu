@@ -183,10 +183,15 @@ struct svdq_weights {
   uint8_t* wscales = nullptr;  // NVFP4 tiled E4M3; INT4 fp32 [K/64 x npad]
   uint16_t* wh = nullptr;      // INT4 with SVDQ_INT4_F16: fp16 s_w q_w [N x K]
   uint16_t* bias = nullptr;
-  // activation-kernel scratch: partial T tiles of split row blocks and their
-  // arrival counters (zero between launches)
+  // bit-reproducible T (svdq_set_deterministic): split partial T tiles and
+  // their per-row-block arrival counters (zero between launches)
+  int deterministic = 0;
   float* kq_tpart = nullptr;
   int* kq_counters = nullptr;
+  // split partials added into T: per-row-block flags (zeroed at load) and
+  // the launch counter whose value split 0 publishes in them
+  unsigned int* kq_flags = nullptr;
+  unsigned int kq_epoch = 0;
   // forward workspace (sized for max_M)
   uint8_t* ws_codes = nullptr;
   uint8_t* ws_scales = nullptr;
@@ -223,8 +228,8 @@ size_t act_scale_bytes(const svdq_weights* h, int64_t M) {
 
 void free_all(svdq_weights* h) {
   void* ptrs[] = {h->inv_lam, h->l1t, h->l2dup, h->wcodes, h->wscales, h->wh, h->bias, h->ws_codes,
-                  h->ws_scales, h->ws_t, h->x_dev, h->y_dev, h->err, h->kq_tpart, h->kq_counters,
-                  h->gq, h->gk};
+                  h->ws_scales, h->ws_t, h->x_dev, h->y_dev, h->err, h->gq, h->gk,
+                  h->kq_tpart, h->kq_counters, h->kq_flags};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -243,13 +248,21 @@ svdq_status launch_kq_t(svdq_weights* h, const CUtensorMap& tmx, int64_t M, uint
     while (ksplit < 8 && num_m * ksplit * 2 <= h->sms && kch % (ksplit * 2) == 0) ksplit *= 2;
   else
     while (ksplit < 8 && num_m * ksplit * 2 <= h->sms && kch % (ksplit * 2) == 0) ksplit *= 2;
+  // split partials are added into T (split 0 clears it first, see kq.cuh);
+  // in deterministic mode they go through the scratch and are summed in
+  // split order
+  const bool accumulate = R > 0 && ksplit > 1 && !h->deterministic;
   KQParams p;
+  p.tflags = h->kq_flags;
+  if (accumulate && ++h->kq_epoch == 0) h->kq_epoch = 1;  // 0 is the flags' initial value
+  p.epoch = h->kq_epoch;
   p.inv_lam = h->inv_lam;
   p.codes = codes;
   p.scales = scales;
   p.t = t;
   p.tpart = h->kq_tpart;
   p.counters = h->kq_counters;
+  p.t_accumulate = accumulate ? 1 : 0;
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(h->K);
   p.ksplit = ksplit;
@@ -656,6 +669,9 @@ svdq_status launch_kq_static(const CUtensorMap& tmx, const CUtensorMap& tml, con
   p.t = t;
   p.tpart = reinterpret_cast<float*>(scratch);
   p.counters = counters;
+  p.t_accumulate = 0;  // deterministic split-order sum through the static scratch
+  p.tflags = nullptr;
+  p.epoch = 0;
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(K);
   p.ksplit = ksplit;
@@ -857,6 +873,8 @@ svdq_status gemm_f32(const float* A, int64_t as0, int64_t as1, const float* B, i
 // Y [rows x l] := an orthonormal basis of its column span, by two rounds of
 // Cholesky QR (Gram matrix in fp64 on the GPU, its factor on the host).
 svdq_status orthonormalize(float* Y, int64_t rows, int l, double* G_dev, cudaStream_t st) {
+  DevBuf yo;
+  if (!yo.alloc(static_cast<size_t>(rows) * l * 4)) return SVDQ_ERR_OOM;
   for (int round = 0; round < 2; ++round) {
     prep_gram_f64_kernel<<<dim3(l, l), 256, 0, st>>>(Y, rows, l, G_dev);
     SVDQ_TRY(cudaGetLastError());
@@ -865,8 +883,10 @@ svdq_status orthonormalize(float* Y, int64_t rows, int l, double* G_dev, cudaStr
     SVDQ_TRY(cudaStreamSynchronize(st));
     if (!cholesky_inv(G, l, Rinv)) return SVDQ_ERR_RANGE;
     SVDQ_TRY(cudaMemcpyAsync(G_dev, Rinv.data(), Rinv.size() * 8, cudaMemcpyHostToDevice, st));
-    prep_rmul_small_kernel<<<static_cast<unsigned>(cdiv(rows, 128)), 128, l * l * 8, st>>>(Y, rows, l, G_dev);
+    prep_rmul_small_kernel<<<static_cast<unsigned>(cdiv(rows * l, 256)), 256, 0, st>>>(Y, rows, l, G_dev,
+                                                                                      yo.as<float>());
     SVDQ_TRY(cudaGetLastError());
+    SVDQ_TRY(cudaMemcpyAsync(Y, yo.p, static_cast<size_t>(rows) * l * 4, cudaMemcpyDeviceToDevice, st));
     SVDQ_TRY(cudaStreamSynchronize(st));  // Rinv (host) outlives the copy
   }
   return SVDQ_OK;
@@ -1029,11 +1049,11 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
     h->norm_eps = d->norm_eps;
   }
   if (!wh.empty() && !dmalloc(reinterpret_cast<void**>(&h->wh), wh.size() * 2)) return fail(SVDQ_ERR_OOM);
-  if (r > 0 && (!dmalloc(reinterpret_cast<void**>(&h->kq_tpart), static_cast<size_t>(sms) * 128 * r * 4) ||
-                !dmalloc(reinterpret_cast<void**>(&h->kq_counters), cdiv(h->max_M, 128) * 4)))
-    return fail(SVDQ_ERR_OOM);
-  if (h->kq_counters && cudaMemset(h->kq_counters, 0, cdiv(h->max_M, 128) * 4) != cudaSuccess)
-    return fail(SVDQ_ERR_CUDA);
+  if (r > 0) {
+    const size_t nf = static_cast<size_t>(cdiv(h->max_M, 128)) * 4;
+    if (!dmalloc(reinterpret_cast<void**>(&h->kq_flags), nf)) return fail(SVDQ_ERR_OOM);
+    if (cudaMemset(h->kq_flags, 0, nf) != cudaSuccess) return fail(SVDQ_ERR_CUDA);
+  }
 
   // synchronous copies: the host vectors go out of scope on return
   if (cudaMemcpy(h->inv_lam, inv.data(), K * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
@@ -1212,6 +1232,31 @@ svdq_status svdq_device_status(svdq_weights_t h, void* stream) {
     if (h->kq_counters) cudaMemset(h->kq_counters, 0, cdiv(h->max_M, 128) * 4);
     return e == 0x34f ? SVDQ_ERR_RANGE : SVDQ_ERR_DEVICE_TIMEOUT;
   }
+  return SVDQ_OK;
+}
+
+svdq_status svdq_set_deterministic(svdq_weights_t h, int on) {
+  if (!h || (on != 0 && on != 1)) return SVDQ_ERR_INVALID_ARG;
+  if (on && h->r > 0 && !h->kq_tpart) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+    if (dev != h->device) return SVDQ_ERR_INVALID_ARG;
+    const size_t nc = static_cast<size_t>(cdiv(h->max_M, 128)) * 4;
+    if (cudaMalloc(&h->kq_tpart, static_cast<size_t>(h->sms) * 128 * h->r * 4) != cudaSuccess) {
+      cudaGetLastError();
+      h->kq_tpart = nullptr;
+      return SVDQ_ERR_OOM;
+    }
+    if (cudaMalloc(&h->kq_counters, nc) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(h->kq_tpart);
+      h->kq_tpart = nullptr;
+      h->kq_counters = nullptr;
+      return SVDQ_ERR_OOM;
+    }
+    if (cudaMemset(h->kq_counters, 0, nc) != cudaSuccess) return SVDQ_ERR_CUDA;
+  }
+  h->deterministic = on;
   return SVDQ_OK;
 }
 
@@ -1415,7 +1460,7 @@ svdq_status svdq_prep_lowrank(const void* w, const float* lambda, int64_t K, int
                               void* stream) {
   if (!w || !lambda || !omega || !L1 || !L2) return SVDQ_ERR_INVALID_ARG;
   if (K < 1 || N < 1 || K > (1 << 20) || N > (1 << 20)) return SVDQ_ERR_SHAPE;
-  if (r < 1 || l < r || l > 64 || l > K || l > N) return SVDQ_ERR_SHAPE;
+  if (r < 1 || l < r || l > 192 || l > K || l > N) return SVDQ_ERR_SHAPE;
   if (power_iters < 0 || power_iters > 8) return SVDQ_ERR_INVALID_ARG;
   int sms = 0;
   svdq_status s = check_device(nullptr, &sms);

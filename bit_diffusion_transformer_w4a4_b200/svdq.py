@@ -37,6 +37,7 @@ EXPORTED = [
     "svdq_prep_calibrate", "svdq_prep_lowrank", "svdq_prep_residual_quantize",
     "svdq_w4a4_gemm_lowrank_up_qkv", "svdq_linear_forward_qkv",
     "svdq_w4a4_gemm_lowrank_up_chain", "svdq_linear_forward_chain", "svdq_device_error_site",
+    "svdq_set_deterministic",
 ]
 
 
@@ -97,6 +98,7 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
     L.svdq_w4a4_gemm_lowrank_up_chain.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp]
     L.svdq_linear_forward_chain.argtypes = [vp, vp, vp, vp, i64, vp]
     L.svdq_device_error_site.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int)]
+    L.svdq_set_deterministic.argtypes = [vp, ctypes.c_int]
     L.svdq_linear_forward_qkv.argtypes = [vp, vp, vp, vp, i64, vp]
     L.svdq_awq_load.argtypes = [ctypes.POINTER(AWQDesc), ctypes.POINTER(vp), vp]
     L.svdq_awq_free.argtypes = [vp]
@@ -234,6 +236,11 @@ class SVDQWeights:
         _check(self._lib.svdq_device_error_site(self.handle, _stream(stream), ctypes.byref(v)),
                "svdq_device_error_site")
         return int(v.value)
+
+    def set_deterministic(self, on: bool = True) -> None:
+        """Sum kernel 1's split partial T tiles in a fixed order (bit-reproducible
+        T and Y) instead of with fp32 reductions."""
+        _check(self._lib.svdq_set_deterministic(self.handle, 1 if on else 0), "svdq_set_deterministic")
 
     def debug_set_fault(self, mask: int, timeout_us: int) -> None:
         _check(self._lib.svdq_debug_set_fault(self.handle, mask, timeout_us), "svdq_debug_set_fault")

@@ -184,7 +184,12 @@ svdq_status svdq_act_scales_bytes(svdq_weights_t h, int64_t M, size_t* bytes);
  *              tiles; inside tile b, K-block j (64 elements = 4 scales) of
  *              row m sits at byte
  *                b*(K/64)*512 + j*512 + (m%32)*16 + ((m/32)%4)*4 + (k/16)%4
- *   t          fp32 [M x r]  T = X' L1 (written; untouched when r == 0)
+ *   t          fp32 [M x r]  T = X' L1 (written; untouched when r == 0).
+ *              When a row block's K range is split over several CTAs (M
+ *              below about 74 * 128 tokens) the partial sums are added into
+ *              t with fp32 reductions (the kernel clears t first), so
+ *              its last bits (and through it Y's) may differ between calls
+ *              on the same input -- unless svdq_set_deterministic is on.
  * Per element (round to nearest even throughout):
  *   x' = bf16(fp32(x) * inv_lambda);  a = max|x'| over the group;
  *   INT4 s = bf16(a / 7), q = rint(x'/s);  NVFP4 s = e4m3_satfinite(a / 6),
@@ -299,8 +304,9 @@ svdq_status svdq_linear_forward_host(svdq_weights_t h, const void* x_host, void*
  *               wait expires (never cleared by the library).  May be NULL:
  *               such a failure is then reported to no one, and the outputs
  *               of that call may be incomplete without any sign of it
- * The split-K scratch (partial T tiles and per-row-block arrival counters)
- * lives in a static device array of the library: 10 MiB of partial tiles
+ * Unlike svdq_quantize_act_lowrank_down, T is summed over the K split in a
+ * fixed order (bit-reproducible).  The split-K scratch (partial T tiles and
+ * per-row-block arrival counters) lives in a static device array of the library: 10 MiB of partial tiles
  * plus counters for M <= 524288 tokens, held by every GPU that loads the
  * library until the process exits.  Calls whose split needs more, or with
  * M > 524288, return SVDQ_ERR_SHAPE before any work is enqueued.  The first
@@ -392,7 +398,7 @@ svdq_status svdq_prep_calibrate(const void* x, int64_t M, const void* w, int64_t
 
 /* Rank-r factors of W_hat = diag(lambda) w by a randomized SVD: the range
  * of W_hat Omega (omega fp32 [N x l], the caller's Gaussian test matrix,
- * r <= l <= 64, l <= min(K, N)) refined by `power_iters` power iterations
+ * r <= l <= 192, l <= min(K, N)) refined by `power_iters` power iterations
  * with re-orthonormalisation (Cholesky QR twice, fp64 Gram matrices), then
  * the small SVD of Q^T W_hat on the host in fp64.  The singular values are
  * split evenly: L1 = Q U_r S_r^(1/2) bf16 [K x r], L2 = S_r^(1/2) V_r^T bf16
@@ -419,6 +425,18 @@ svdq_status svdq_prep_residual_quantize(svdq_variant variant, const void* w, con
  * calls on this handle (SVDQ_ERR_DEVICE_TIMEOUT), clearing the record.
  */
 svdq_status svdq_device_status(svdq_weights_t h, void* stream);
+
+/*
+ * Bit-reproducible T (no counterpart on the pages): with on = 1 the split
+ * partial T tiles of kernel 1 are summed in a fixed order through a scratch
+ * buffer owned by the handle (allocated here, sms * 128 * r floats plus one
+ * counter per 128-row block), so T and Y are the same bits on every call
+ * with the same input; with on = 0 (the default) they are added into T with
+ * fp32 reductions, which is faster.  Codes and scales are bit-exact either
+ * way.  Returns SVDQ_ERR_OOM if the scratch cannot be allocated, and
+ * SVDQ_ERR_INVALID_ARG for on other than 0 / 1 or a different current device.
+ */
+svdq_status svdq_set_deterministic(svdq_weights_t h, int on);
 
 /*
  * Failure reporting (no counterpart on the pages): the wait-site code of the

@@ -71,6 +71,8 @@ def test_null_arguments():
     assert L.svdq_w4a4_gemm_lowrank_up(None, None, None, None, 1, None, None) == 1
     assert L.svdq_device_status(None, None) == 1
     assert L.svdq_debug_set_fault(None, 1, 10) == 1
+    assert L.svdq_set_deterministic(None, 1) == 1
+    assert L.svdq_device_error_site(None, None, None) == 1
     n = ctypes.c_size_t(0)
     assert L.svdq_act_scales_bytes(None, 1, ctypes.byref(n)) == 1
 

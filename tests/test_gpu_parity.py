@@ -79,6 +79,7 @@ def test_forward_small(variant, opts, gelu, with_bias, M, K, N, r):
     """Ragged M and N (partial tiles), several K tiles, bias and GELU."""
     lay, x, pw = _prepped(M, K, N, r, variant, gelu=gelu, with_bias=with_bias)
     h = svdq.SVDQWeights(pw, M, **opts)
+    h.set_deterministic()  # the two entry points are compared bit for bit below
     got = PT.gpu_forward(h, x, M)
     ref = O.linear_forward(x, pw)
     PT.check_act(got, ref, r=r, label="fwd")
@@ -131,6 +132,7 @@ def test_host_entry_point_matches_device(variant):
     pw = W.synthetic_packed(lay)
     x = W.activations(lay)
     h = svdq.SVDQWeights(pw, M)
+    h.set_deterministic()
     dev = PT.gpu_forward(h, x, M, two_calls=False)
     xh = torch.from_numpy(x.view(np.int16)).pin_memory()
     yh = torch.empty((M, N), dtype=torch.int16).pin_memory()
@@ -149,6 +151,7 @@ def test_bounded_wait_reports_timeout(variant, opts, mask):
     pw = W.synthetic_packed(lay)
     x = W.activations(lay)
     h = svdq.SVDQWeights(pw, M, **opts)
+    h.set_deterministic()
     ok = PT.gpu_forward(h, x, M)
     h.debug_set_fault(mask, 20000)                 # 20 ms limit
     import torch
@@ -274,6 +277,7 @@ def test_handles_loaded_from_two_threads():
     ref = []
     for lay, pw, x in cases:
         h = svdq.SVDQWeights(pw, M)
+        h.set_deterministic()
         ref.append(PT.gpu_forward(h, x, M)["Y"])
         h.close()
     out = [None, None]
@@ -286,6 +290,7 @@ def test_handles_loaded_from_two_threads():
             s = torch.cuda.Stream()
             with torch.cuda.stream(s):
                 h = svdq.SVDQWeights(pw, M)
+                h.set_deterministic()
                 out[i] = PT.gpu_forward(h, x, M)["Y"]
                 h.close()
         except Exception as e:  # reported below
@@ -299,3 +304,34 @@ def test_handles_loaded_from_two_threads():
     assert not err, err
     for i in range(2):
         assert np.array_equal(out[i], ref[i])
+
+
+@pytest.mark.parametrize("variant", [NVFP4, INT4])
+def test_split_t_reduction_modes(variant):
+    """Kernel 1's split partial T tiles added into T with fp32 reductions (the
+    default) against the fixed-order sum (svdq_set_deterministic): codes and
+    scales identical, T within the fp32 accumulation bound of the oracle's
+    exact T, and the deterministic mode repeats its bits."""
+    import torch
+    M, K, N, r = 1000, 3072, 512, 32   # 8 row blocks: the K range is split
+    lay = W.Layer("tsum", M=M, K=K, N=N, r=r, variant=variant, config_id=70)
+    pw = W.synthetic_packed(lay)
+    x = W.activations(lay)
+    h = svdq.SVDQWeights(pw, M)
+    fast = PT.gpu_forward(h, x, M)
+    h.set_deterministic()
+    det1 = PT.gpu_forward(h, x, M)
+    det2 = PT.gpu_forward(h, x, M)
+    h.set_deterministic(False)
+    fast2 = PT.gpu_forward(h, x, M)
+    h.close()
+    assert np.array_equal(fast["codes"], det1["codes"]) and np.array_equal(fast["scales"], det1["scales"])
+    assert np.array_equal(det1["T"], det2["T"]) and np.array_equal(det1["Y"], det2["Y"])
+    xp = O.smooth_activations(x, (np.float32(1) / pw.lam).astype(np.float32)).astype(np.float64)
+    l1 = W.bf16_bits_to_f32(pw.L1).astype(np.float64)
+    tb = PT.t_bound(xp, l1)
+    texact = xp @ l1
+    for got, label in ((fast, "reductions"), (det1, "fixed order"), (fast2, "reductions again")):
+        d = float(np.linalg.norm(got["T"].astype(np.float64) - texact))
+        PT.record(f"T {label} v{variant}", "||dT|| / fp32 bound", d / tb, 1.0)
+        assert d <= tb, (label, d, tb)

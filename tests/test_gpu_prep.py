@@ -77,13 +77,14 @@ def test_residual_quantize_matches_oracle(variant, tensor_scale, r):
     assert bad_c == 0 and bad_s == 0, (bad_c, bad_s)
 
 
-@pytest.mark.parametrize("power_iters", [1, 2])
-def test_randomized_svd_near_optimal(power_iters):
+@pytest.mark.parametrize("r,power_iters", [(32, 1), (32, 2), (128, 2)])
+def test_randomized_svd_near_optimal(r, power_iters):
     """lowrank128 weights (singular values 48/i plus noise): the GPU factors'
     residual ||W_hat - L1 L2||_F is within 2% of the exact truncated SVD's
-    (the oracle's prepare(), bf16 factors as well)."""
+    (the oracle's prepare(), bf16 factors as well); r = 128 runs a sketch of
+    144 columns."""
     import torch
-    lay = W.Layer("rs", M=512, K=1024, N=768, r=32, variant=NVFP4, weight_kind="lowrank128", config_id=97)
+    lay = W.Layer("rs", M=512, K=1024, N=768, r=r, variant=NVFP4, weight_kind="lowrank128", config_id=97)
     x = W.activations(lay)
     w = W.weight(lay)
     pw = P.prepare(x, w, lay.r, NVFP4)
@@ -99,7 +100,7 @@ def test_randomized_svd_near_optimal(power_iters):
     res_gpu = np.linalg.norm(pw.w_hat - l1 @ l2)
     res_ora = np.linalg.norm(pw.R)
     opt = np.sqrt(np.sum(pw.S[lay.r:] ** 2))
-    PT.record(f"rsvd q{power_iters}", "residual / optimum", res_gpu / opt, 1.02)
+    PT.record(f"rsvd r{r} q{power_iters}", "residual / optimum", res_gpu / opt, 1.02)
     assert res_ora <= 1.001 * opt
     assert res_gpu <= 1.02 * opt, (res_gpu / opt, res_ora / opt)
 
