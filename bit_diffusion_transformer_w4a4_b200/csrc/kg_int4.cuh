@@ -23,7 +23,8 @@
 //   warp 0      TMA producer: packed activation codes (32B swizzle) and int8
 //               weight codes (64B swizzle) for one 64-group per stage
 //   warp 1      MMA issuer (two k-steps of 32 per group), tensor-memory owner
-//   warps 2-3   unpack activation nibbles to int8 in the MMA operand layout
+//   warps 2-3   unpack activation nibbles to int8 (16 x the code) in the MMA
+//               operand layout
 //   warps 4-19  epilogue: per-group rescale into fp32 registers, low-rank
 //               add, next tile's low-rank operand, bias + GELU + bf16 stores
 #pragma once
@@ -59,13 +60,14 @@ struct KGI4Smem {
   static_assert(TOTAL <= 232448, "shared memory per CTA");
 };
 
-// 8 two's-complement nibbles (element 0 in the low nibble) -> 8 int8 bytes.
-__device__ __forceinline__ uint2 unpack_s4x8(uint32_t w) {
-  uint32_t lo = w & 0x0F0F0F0Fu;          // elements 0, 2, 4, 6
-  uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;   // elements 1, 3, 5, 7
-  // per byte: n -> n - 16 when n >= 8 (no carries: every byte stays < 136)
-  lo = ((lo ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
-  hi = ((hi ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+// 8 two's-complement nibbles (element 0 in the low nibble) -> 8 int8 bytes
+// holding 16 x each value: the nibble moves to the byte's high half, so its
+// sign bit is the byte's and no sign extension is needed.  The group products
+// come out as 16 P; the weight-scale table holds s_w / 16 (exact: a power of
+// two), so the rescale below is unchanged.
+__device__ __forceinline__ uint2 unpack_s4x8_x16(uint32_t w) {
+  const uint32_t lo = (w << 4) & 0xF0F0F0F0u;  // elements 0, 2, 4, 6
+  const uint32_t hi = w & 0xF0F0F0F0u;         // elements 1, 3, 5, 7
   uint2 r;
   r.x = __byte_perm(lo, hi, 0x5140);
   r.y = __byte_perm(lo, hi, 0x7362);
@@ -246,8 +248,8 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const uint4 v = *reinterpret_cast<const uint4*>(apk + swz_off(row, c, 32));
-            const uint2 o0 = unpack_s4x8(v.x), o1 = unpack_s4x8(v.y);
-            const uint2 o2 = unpack_s4x8(v.z), o3 = unpack_s4x8(v.w);
+            const uint2 o0 = unpack_s4x8_x16(v.x), o1 = unpack_s4x8_x16(v.y);
+            const uint2 o2 = unpack_s4x8_x16(v.z), o3 = unpack_s4x8_x16(v.w);
             *reinterpret_cast<uint4*>(a8 + swz_off(row, 2 * c, 64)) = make_uint4(o0.x, o0.y, o1.x, o1.y);
             *reinterpret_cast<uint4*>(a8 + swz_off(row, 2 * c + 1, 64)) = make_uint4(o2.x, o2.y, o3.x, o3.y);
           }
@@ -322,9 +324,9 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 16; ++i) acc[i] = 0ull;
       const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16) + cs * 32;
-      // float(P) for the s32 group product P (a sum of 64 products of 4-bit
-      // codes, |P| <= 4096 < 2^22): bits(P + bits(1.5 * 2^23)) - 1.5 * 2^23,
-      // exact, at the full rate of integer and fp32 adds
+      // float(P) for the s32 group product P (16 x a sum of 64 products of
+      // 4-bit codes, |P| <= 65536 < 2^22): bits(P + bits(1.5 * 2^23)) -
+      // 1.5 * 2^23, exact, at the full rate of integer and fp32 adds
       const uint64_t mag = f2_pack(-12582912.0f, -12582912.0f);
       const uint8_t* scb = nullptr;
       for (int g = 0; g < ng; ++g, ++gc) {

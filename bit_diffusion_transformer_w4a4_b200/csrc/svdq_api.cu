@@ -1028,6 +1028,12 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
   }
 
   // ---- device allocations and copies
+  if (d->variant == SVDQ_INT4_G64_BF16) {
+    // the int8 GEMM's activation operand holds 16 x the codes: its weight
+    // scales are stored as s_w / 16 (exact), after the host uses above
+    float* sf = reinterpret_cast<float*>(scales.data());
+    for (size_t i = 0; i < scales.size() / 4; ++i) sf[i] *= 0.0625f;
+  }
   if (!dmalloc(reinterpret_cast<void**>(&h->inv_lam), K * 4) ||
       !dmalloc(reinterpret_cast<void**>(&h->wcodes), codes.size()) ||
       !dmalloc(reinterpret_cast<void**>(&h->wscales), scales.size()) ||
