@@ -158,6 +158,9 @@ def test_bounded_wait_reports_timeout(variant, opts, mask):
     xd = PT.to_dev(x.view(np.int16)).view(torch.bfloat16)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     h.linear_forward(xd, y, M)
+    # the wait that expired first: kernel 1's sites are 0x1xx, kernel 2's 0x2xx / 0x3xx
+    site = h.device_error_site()
+    assert (site >> 8) == 1 if mask == 2 else (site >> 8) in (2, 3), hex(site)
     assert h.device_status() == 7                 # SVDQ_ERR_DEVICE_TIMEOUT
     h.debug_set_fault(0, 0)
     again = PT.gpu_forward(h, x, M)
