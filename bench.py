@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--int4-f16", action="store_true",
                     help="INT4 workloads: kernel 2 as one fp16 GEMM of the dequantised operands "
                          "(SVDQ_INT4_F16) instead of int8 MMAs")
+    ap.add_argument("--qkv-epilogue", action="store_true",
+                    help="NVFP4 qkv layers: kernel 2 with the fused Q/K RMS norm + rotary epilogue "
+                         "(svdq_w4a4_gemm_lowrank_up_qkv; a seeded 2-D position table)")
     ap.add_argument("--l2-warm", action="store_true",
                     help="layer workloads: no L2 flush between steps (steps back to back; the "
                          "layers' inputs and outputs together exceed the 126 MB L2)")
@@ -152,10 +155,11 @@ def layer_bytes(layer) -> int:
             + K * r * 2 + r * N * 2 + 2 * M * r * 4 + M * N * 2)
 
 
-def layer_desc(layer, f16: bool = False) -> str:
+def layer_desc(layer, f16: bool = False, qkv: bool = False) -> str:
     from bit_diffusion_transformer_w4a4_b200 import workloads as W
     return (f"{layer.name} M{layer.M} K{layer.K} N{layer.N} r{layer.r}{' GELU' if layer.gelu else ''} "
-            f"{W.VARIANT_NAME[layer.variant]}{' fp16-operand GEMM' if f16 else ''}")
+            f"{W.VARIANT_NAME[layer.variant]}{' fp16-operand GEMM' if f16 else ''}"
+            f"{' + QK-norm + RoPE epilogue' if qkv else ''}")
 
 
 def cpu_baseline(layer, pw, x_bits, nrows: int, one_core: bool = True):
@@ -368,7 +372,14 @@ def run_ours(args, layers):
         f16 = bool(args.int4_f16) and layer.variant == W.INT4
         pw = W.synthetic_packed(layer, seed=rank)
         x_bits = W.activations(layer, seed=rank)
-        h = svdq.SVDQWeights(pw, layer.M, int4_f16=f16)
+        qkv = bool(args.qkv_epilogue) and layer.name.endswith("qkv") and layer.variant == W.NVFP4
+        rope = None
+        if qkv:
+            gq, gk, rope_h = W.qkv_epilogue_inputs(layer.M, rank)
+            h = svdq.SVDQWeights(pw, layer.M, qkv_norm=(gq, gk, 1e-6))
+            rope = torch.from_numpy(rope_h).cuda()
+        else:
+            h = svdq.SVDQWeights(pw, layer.M, int4_f16=f16)
         chained = layer.name.endswith("fc2") and any(n.endswith("fc1") for n in names[:i])
         if chained:
             x = L[names.index(names[i - 1])]["y"]
@@ -377,7 +388,7 @@ def run_ours(args, layers):
         y = torch.empty((layer.M, layer.N), dtype=torch.bfloat16, device="cuda")
         codes, scales, t = h.alloc_act(layer.M)
         L.append(dict(layer=layer, pw=pw, x_bits=x_bits, h=h, x=x, y=y, codes=codes, scales=scales,
-                      t=t, f16=f16, chained=chained))
+                      t=t, f16=f16, chained=chained, rope=rope))
     # L2 flush before every step, outside the timed events: a 256 MB write,
     # then a 256 MB read of another buffer, so that L2 holds neither the inputs
     # nor dirty lines whose write-back would land inside the next step
@@ -412,6 +423,9 @@ def run_ours(args, layers):
             launches.append((pre + "w4a4_gemm_lowrank_up_chain", lambda d=d, d2=d2: svdq.gemm_lowrank_up_chain(
                 d["h"], d["codes"], d["scales"], d["t"], d["layer"].M, None, d2["h"], d2["codes"], d2["scales"],
                 d2["t"])))
+        elif d["rope"] is not None:
+            launches.append((pre + "w4a4_gemm_lowrank_up_qkv", lambda d=d: d["h"].w4a4_gemm_lowrank_up_qkv(
+                d["codes"], d["scales"], d["t"], d["layer"].M, d["rope"], d["y"])))
         else:
             launches.append((pre + "w4a4_gemm_lowrank_up", lambda d=d: d["h"].w4a4_gemm_lowrank_up(
                 d["codes"], d["scales"], d["t"], d["layer"].M, d["y"])))
@@ -481,7 +495,14 @@ def run_ours(args, layers):
 
     def host_step():
         for d, xh, yh in zip(L, hx, hy):
-            d["h"].linear_forward_host(xh, yh, d["layer"].M)
+            if d["rope"] is None:
+                d["h"].linear_forward_host(xh, yh, d["layer"].M)
+                continue
+            # the QKV-epilogue layer has no host-buffer entry point: the same
+            # copies around the device entry point
+            d["x"].view(torch.int16).copy_(xh, non_blocking=True)
+            d["h"].linear_forward_qkv(d["x"], d["rope"], d["y"], d["layer"].M)
+            yh.copy_(d["y"].view(torch.int16), non_blocking=True)
 
     for _ in range(2):
         host_step()
@@ -527,7 +548,7 @@ def run_ours(args, layers):
     sm_mhz = clk.get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
     nominal = 148 * 2 * 128 * 256 * 64 / 128 * sm_mhz * 1e6 / 1e12 / (1.0 if nvfp4 else 2.0)
     traffic_key = args.workload + ("/int4_f16" if f16 else "")
-    wl = " + ".join(layer_desc(d["layer"], d["f16"]) for d in L)
+    wl = " + ".join(layer_desc(d["layer"], d["f16"], d["rope"] is not None) for d in L)
     kernels = {n: per_k[i] for i, n in enumerate(names_k)}
     line = {
         "metric": metric_name(args.workload, [d["layer"] for d in L]), "value": value, "unit": "TFLOPS",
@@ -541,6 +562,7 @@ def run_ours(args, layers):
                    "parallelism": f"replicas x{world}", "tokens_per_step": L[0]["layer"].M * world,
                    "chained": [d["layer"].name for d in L if d["chained"]],
                    "fused_pairs": [L[i]["layer"].name + "->" + L[i + 1]["layer"].name for i in sorted(fused)],
+                   "qkv_epilogue": [d["layer"].name for d in L if d["rope"] is not None],
                    "timing": "ms_per_step: events at step boundaries only (kernels overlap through "
                              "programmatic dependent launch); kernels_ms: a second timed pass with an "
                              "event after every kernel"},

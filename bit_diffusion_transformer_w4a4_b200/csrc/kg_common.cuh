@@ -34,7 +34,8 @@ struct KGParams {
   float out_scale, t_scale;
   // fused QKV epilogue (qkv_hd > 0): columns [Q | K | V] of qkv_hd each; Q
   // and K heads (128 features) RMS-normalised (times gq / gk, bf16 [128]) and
-  // rotated pairwise by rope (fp32 [M x 64 x 2]: cos, sin per token and pair)
+  // rotated pairwise by rope: the row-blocked table of rope_block_kernel
+  // (float4 [rows / 32][32 two-pair chunks][32 rows] of cos, sin, cos, sin)
   int qkv_hd;
   float norm_eps;
   const uint16_t* gq;
@@ -215,7 +216,8 @@ __device__ __forceinline__ void store_rows32_coalesced(const KGParams& p, int ro
 // Kernels and Generality": the QKV projection, the Q/K normalisation and the
 // rotary embedding in one kernel.  Per value: v = acc * out_scale (+ bias);
 // for Q and K columns, per 128-feature head: v <- v / sqrt(mean(v^2) + eps)
-// * g, then pairs (2i, 2i+1) rotated by token row's (cos, sin) of pair i.
+// * g, then pairs (2i, 2i+1) rotated by token row's (cos, sin) of pair i
+// (read from the row-blocked copy of the caller's table).
 // A head spans two warps (slices cs and cs ^ 1 of the same lane quarter q).
 // Each publishes its rows' partial sums of squares in red ([4][4][32]
 // floats) and the pair exchanges them through mbarrier xbar[q + 4 (cs/2)]
@@ -266,12 +268,14 @@ __device__ __forceinline__ bool epilogue_qkv64(const KGParams& p, int row0, int 
         v[8 * c8 + 2 * e + 1] = __fmul_rn(__fmul_rn(v[8 * c8 + 2 * e + 1], inv), bf16hi(gw[e]));
       }
     }
-    const int row = row0 + lane;
-    const float4* cs4 =
-        reinterpret_cast<const float4*>(p.rope + (static_cast<size_t>(row < p.M ? row : 0) * 64 + d0 / 2) * 2);
+    // row0 is a multiple of 32 and the blocked table covers every row of
+    // every tile (rows past M hold the identity rotation): each load reads
+    // the 32 rows' chunk d0 / 4 + i2, 512 contiguous bytes
+    const float4* cs4 = reinterpret_cast<const float4*>(p.rope) +
+                        (static_cast<size_t>(row0 / 32) * 32 + d0 / 4) * 32 + lane;
 #pragma unroll
     for (int i2 = 0; i2 < 16; ++i2) {  // two pairs per 16-byte load: (cos, sin, cos, sin)
-      const float4 t = row < p.M ? __ldg(cs4 + i2) : make_float4(1.f, 0.f, 1.f, 0.f);
+      const float4 t = __ldg(cs4 + 32 * i2);
       const float a0 = v[4 * i2], b0 = v[4 * i2 + 1], a1 = v[4 * i2 + 2], b1 = v[4 * i2 + 3];
       v[4 * i2] = __fsub_rn(__fmul_rn(a0, t.x), __fmul_rn(b0, t.y));
       v[4 * i2 + 1] = __fadd_rn(__fmul_rn(a0, t.y), __fmul_rn(b0, t.x));

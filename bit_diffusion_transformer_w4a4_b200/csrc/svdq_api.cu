@@ -24,6 +24,7 @@
 #include "kg_nvfp4_chain.cuh"
 #include "kg_nvfp4_pair.cuh"
 #include "kq.cuh"
+#include "krope.cuh"
 
 using namespace svdq;
 
@@ -169,11 +170,14 @@ struct svdq_weights {
   uint32_t flags;
   int device, sms;
   float out_scale = 1.0f, t_scale = 1.0f;  // 2^e and 2^-e of the NVFP4 per-tensor scale
-  // fused QKV epilogue (SVDQ_EPI_QKV_NORM_ROPE): norm weights, epsilon, and
-  // the rotary table of the call being launched
+  // fused QKV epilogue (SVDQ_EPI_QKV_NORM_ROPE): norm weights, epsilon, the
+  // row-blocked rotary table (library-owned, cdiv(max_M, 256) * 256 rows of
+  // 512 bytes, rewritten by every call), and the table of the call being
+  // launched (rope_blk while the GEMM is launched, else null)
   uint16_t* gq = nullptr;
   uint16_t* gk = nullptr;
   float norm_eps = 0.f;
+  float* rope_blk = nullptr;
   const float* rope = nullptr;
   // device weights (library-owned)
   float* inv_lam = nullptr;
@@ -228,7 +232,7 @@ size_t act_scale_bytes(const svdq_weights* h, int64_t M) {
 
 void free_all(svdq_weights* h) {
   void* ptrs[] = {h->inv_lam, h->l1t, h->l2dup, h->wcodes, h->wscales, h->wh, h->bias, h->ws_codes,
-                  h->ws_scales, h->ws_t, h->x_dev, h->y_dev, h->err, h->gq, h->gk,
+                  h->ws_scales, h->ws_t, h->x_dev, h->y_dev, h->err, h->gq, h->gk, h->rope_blk,
                   h->kq_tpart, h->kq_counters, h->kq_flags};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -1047,7 +1051,8 @@ svdq_status svdq_weights_load(const svdq_weight_desc* d, svdq_weights_t* out, vo
     return fail(SVDQ_ERR_OOM);
   if (d->bias && !dmalloc(reinterpret_cast<void**>(&h->bias), N * 2)) return fail(SVDQ_ERR_OOM);
   if (d->flags & SVDQ_EPI_QKV_NORM_ROPE) {
-    if (!dmalloc(reinterpret_cast<void**>(&h->gq), 256) || !dmalloc(reinterpret_cast<void**>(&h->gk), 256))
+    if (!dmalloc(reinterpret_cast<void**>(&h->gq), 256) || !dmalloc(reinterpret_cast<void**>(&h->gk), 256) ||
+        !dmalloc(reinterpret_cast<void**>(&h->rope_blk), static_cast<size_t>(cdiv(h->max_M, 256)) * 256 * 512))
       return fail(SVDQ_ERR_OOM);
     if (cudaMemcpy(h->gq, d->q_norm, 256, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(h->gk, d->k_norm, 256, cudaMemcpyHostToDevice) != cudaSuccess)
@@ -1190,9 +1195,20 @@ svdq_status svdq_w4a4_gemm_lowrank_up_qkv(svdq_weights_t h, const uint8_t* act_c
                                           const void* act_scales, const float* t, int64_t M,
                                           const float* rope, void* y, void* stream) {
   if (!h || !(h->flags & SVDQ_EPI_QKV_NORM_ROPE) || !rope) return SVDQ_ERR_INVALID_ARG;
-  if (!aligned16(rope)) return SVDQ_ERR_ALIGNMENT;
-  h->rope = rope;
-  const svdq_status s = svdq_w4a4_gemm_lowrank_up(h, act_codes, act_scales, t, M, y, stream);
+  svdq_status s = check_call(h, M);
+  if (s != SVDQ_OK) return s;
+  if (!act_codes || !act_scales || !y || (h->r > 0 && !t)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(rope) || !aligned16(act_codes) || !aligned16(act_scales) || !aligned16(y) ||
+      (t && !aligned16(t)))
+    return SVDQ_ERR_ALIGNMENT;
+  // the row-blocked table for every row of every GEMM tile (256-row tiles on
+  // SM pairs, 128 on single SMs), then the GEMM reading it
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LaunchCfg lc(dim3(static_cast<unsigned>(cdiv(M, 256) * 8)), dim3(256), 0, st);
+  SVDQ_TRY(cudaLaunchKernelEx(&lc.cfg, rope_block_kernel, reinterpret_cast<const float4*>(rope),
+                              static_cast<int>(M), reinterpret_cast<float4*>(h->rope_blk)));
+  h->rope = h->rope_blk;
+  s = svdq_w4a4_gemm_lowrank_up(h, act_codes, act_scales, t, M, y, stream);
   h->rope = nullptr;
   return s;
 }

@@ -206,6 +206,24 @@ def synthetic_packed(layer: Layer, seed: int = 0, int4_min: int = -7) -> PackedW
                          bias(layer, seed), layer.gelu, {"source": "synthetic"})
 
 
+def qkv_epilogue_inputs(M: int, seed: int = 0):
+    """Inputs of the fused QKV epilogue for M tokens: the Q and K norm
+    weights (bf16 bits [128], around 1) and the caller's rotary table
+    [M, 128] fp32 of (cos, sin) per interleaved pair.  Angles: token m sits
+    at (m // 64, m % 64) on a 2-D grid; pair i turns at 10000^(-(i mod 32)/32)
+    per unit of the row coordinate (pairs 0-31) or the column (32-63)."""
+    g = _rng(seed, 91, 0)
+    gq = to_bf16_bits(np.float32(1) + np.float32(0.2) * g.standard_normal(128, dtype=np.float32))
+    gk = to_bf16_bits(np.float32(1) + np.float32(0.2) * g.standard_normal(128, dtype=np.float32))
+    i = np.arange(64)
+    freq = 10000.0 ** (-(i % 32) / 32.0)
+    m = np.arange(M)
+    pos = np.where(i[None, :] < 32, (m // 64)[:, None], (m % 64)[:, None]).astype(np.float64)
+    ang = pos * freq[None, :]
+    rope = np.stack([np.cos(ang), np.sin(ang)], axis=-1).reshape(M, 128).astype(np.float32)
+    return gq, gk, rope
+
+
 # ------------------------------------------------------------ AWQ W4A16 layers
 @dataclass(frozen=True)
 class AWQLayer:

@@ -238,7 +238,12 @@ svdq_status svdq_linear_forward(svdq_weights_t h, const void* x, void* y, int64_
  *   rope  device fp32 [M x 64 x 2], 16-byte aligned: (cos, sin) of the
  *         rotary angle of token m for pair i at rope[(m * 64 + i) * 2]
  * Other arguments as svdq_w4a4_gemm_lowrank_up / svdq_linear_forward.  The
- * table is read while the kernel runs (it must stay valid until then).
+ * GEMM is preceded by one small kernel that copies the table, row-blocked
+ * (32 tokens per block, so that the epilogue's loads are contiguous), into
+ * a buffer the handle owns (cdiv(max_M, 256) * 256 * 512 bytes, allocated at
+ * load); the caller's table is read by that kernel and must stay valid until
+ * it has run.  Calls on one handle from different streams at once race on
+ * that buffer as on the workspace.
  */
 svdq_status svdq_w4a4_gemm_lowrank_up_qkv(svdq_weights_t h, const uint8_t* act_codes,
                                           const void* act_scales, const float* t, int64_t M,

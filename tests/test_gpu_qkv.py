@@ -2,7 +2,7 @@
 RMS normalisation of Q and K, rotary embedding of their interleaved pairs,
 V untouched) against the oracle: NVFP4 on SM pairs and on single SMs, with
 bias, ragged M, several tiles per CTA, and the layer's own all-row check at
-a 2048-px block's qkv shape."""
+a 2048-px block's qkv shape with the benchmark's inputs."""
 import math
 
 import numpy as np
@@ -83,3 +83,27 @@ def test_qkv_plain_calls_refused():
     with pytest.raises(svdq.SvdqError):
         h.linear_forward(x, y, 128)
     h.close()
+
+
+def test_qkv_epilogue_block_full_size():
+    """The 2048-px block's qkv layer (M16896 K3072 N9216 r32, NVFP4, SM pairs)
+    with the benchmark's norm weights and rotary table, in the launch
+    configuration the benchmark times: every row against the oracle."""
+    import torch
+    lay = W.workloads()["block_2048px"][0]
+    assert lay.name.endswith("qkv") and lay.variant == W.NVFP4
+    x = W.activations(lay)
+    pw = W.synthetic_packed(lay)
+    gq, gk, rope = W.qkv_epilogue_inputs(lay.M, 0)
+    h = svdq.SVDQWeights(pw, lay.M, qkv_norm=(gq, gk, 1e-6))
+    xd = PT.to_dev(x.view(np.int16)).view(torch.bfloat16)
+    y = torch.empty((lay.M, lay.N), dtype=torch.bfloat16, device="cuda")
+    h.linear_forward_qkv(xd, PT.to_dev(rope), y, lay.M)
+    torch.cuda.synchronize()
+    assert h.device_status() == 0
+    Y = PT.from_dev(y.view(torch.int16)).view(np.uint16)
+    h.close()
+    act = PT.oracle_act_all(pw, x)
+    acc, _ = PT.oracle_y_all(pw, act)
+    yq, Yq = Q.qkv_epilogue(acc, gq, gk, rope[:, 0::2].astype(np.float64), rope[:, 1::2].astype(np.float64))
+    PT.check_y(Y, yq, Yq, label="qkv block 2048px")

@@ -37,3 +37,17 @@ def test_synthetic_packed_shapes():
         assert pw.scales.shape == (64, 256 // G)
         assert pw.L1.shape == (256, 32) and pw.L2.shape == (32, 64)
         assert pw.lam.dtype == np.float32 and np.all(pw.lam > 0)
+
+
+def test_qkv_epilogue_inputs():
+    gq, gk, rope = W.qkv_epilogue_inputs(300)
+    assert gq.dtype == np.uint16 and gq.shape == (128,) and not np.array_equal(gq, gk)
+    g = W.bf16_bits_to_f32(gq)
+    assert 0.3 < g.min() and g.max() < 1.8
+    assert rope.shape == (300, 128) and rope.dtype == np.float32
+    c, s = rope[:, 0::2].astype(np.float64), rope[:, 1::2].astype(np.float64)
+    assert np.abs(c * c + s * s - 1).max() < 1e-6
+    # token 65 sits at grid (1, 1): pair 0 turns by 1 radian, pair 32 too
+    assert abs(c[65, 0] - np.cos(1.0)) < 1e-7 and abs(s[65, 32] - np.sin(1.0)) < 1e-7
+    assert np.all(c[0] == 1) and np.all(s[0] == 0)
+    assert np.array_equal(W.qkv_epilogue_inputs(300)[2], rope)
