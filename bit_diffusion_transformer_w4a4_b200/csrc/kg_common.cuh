@@ -46,13 +46,52 @@ struct KGParams {
   uint64_t timeout_ns;
 };
 
-// GELU, tanh form: 0.5 x (1 + tanh(u)) = x / (1 + exp(-2u)),
-// u = sqrt(2/pi) (x + 0.044715 x^3).
-__device__ __forceinline__ float gelu_tanh(float x) {
-  const float u = __fmul_rn(__fmul_rn(x, __fmaf_rn(0.044715f * x, x, 1.0f)), 0.7978845608028654f);
-  float e;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-2.8853900817779268f * u));
-  return __fdividef(x, 1.0f + e);
+// GELU, tanh form, of two values with paired fp32 arithmetic:
+//   0.5 x (1 + tanh(u)) = x / (1 + exp(-2u)) = x / (1 + 2^a),
+//   u = sqrt(2/pi) (x + 0.044715 x^3),  a = x (c1 + c2 x^2),
+//   c1 = -2 log2(e) sqrt(2/pi),  c2 = 0.044715 c1,
+// with the hardware's approximate base-2 exponential and reciprocal (both
+// within a few fp32 ulps; x / (1 + 2^a) -> -0 or 0 as 2^a overflows).
+__device__ __forceinline__ uint64_t gelu_tanh2(uint64_t x) {
+  const uint64_t t = f2_fma(f2_mul(x, x), f2_pack(-0.10294324160f, -0.10294324160f),
+                            f2_pack(-2.3022081852f, -2.3022081852f));
+  const uint64_t a = f2_mul(x, t);
+  float e0, e1, r0, r1;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(f2_lo(a)));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(f2_hi(a)));
+  const uint64_t d = f2_add(f2_pack(e0, e1), f2_pack(1.0f, 1.0f));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(f2_lo(d)));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r1) : "f"(f2_hi(d)));
+  return f2_mul(x, f2_pack(r0, r1));
+}
+// In place on 2n values.
+template <int N2>
+__device__ __forceinline__ void gelu_tanh_pairs(float* v) {
+#pragma unroll
+  for (int e = 0; e < 2 * N2; e += 2) {
+    const uint64_t g = gelu_tanh2(f2_pack(v[e], v[e + 1]));
+    v[e] = f2_lo(g);
+    v[e + 1] = f2_hi(g);
+  }
+}
+
+// v[0..7] (columns n..n+7) <- v * out_scale (+ bias), in pairs.
+__device__ __forceinline__ void scale_bias_pairs(const KGParams& p, int n, float* v) {
+  const uint64_t os2 = f2_pack(p.out_scale, p.out_scale);
+  uint64_t x[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = f2_mul(f2_pack(v[2 * e], v[2 * e + 1]), os2);
+  if (p.bias != nullptr && n < p.N) {
+    const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
+    const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = f2_add(x[e], f2_pack(bf16lo(bw[e]), bf16hi(bw[e])));
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    v[2 * e] = f2_lo(x[e]);
+    v[2 * e + 1] = f2_hi(x[e]);
+  }
 }
 
 // Write [T_hi | T_lo] of rows m0..m0+127 into the A operand buffer of the
@@ -111,19 +150,10 @@ __device__ __forceinline__ void store_rows64_coalesced(const KGParams& p, int ro
     const int n = n_base + 8 * j8;
     float v[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = FINAL ? acc[8 * j8 + e] : __fmul_rn(acc[8 * j8 + e], p.out_scale);
-    if (!FINAL && p.bias != nullptr && n < p.N) {
-      const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
-      const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[2 * e] = __fadd_rn(v[2 * e], bf16lo(bw[e]));
-        v[2 * e + 1] = __fadd_rn(v[2 * e + 1], bf16hi(bw[e]));
-      }
-    }
-    if (!FINAL && p.gelu) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = gelu_tanh(v[e]);
+    for (int e = 0; e < 8; ++e) v[e] = acc[8 * j8 + e];
+    if (!FINAL) {
+      scale_bias_pairs(p, n, v);
+      if (p.gelu) gelu_tanh_pairs<4>(v);
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) w[4 * j8 + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
@@ -166,20 +196,9 @@ __device__ __forceinline__ void store_rows32_coalesced(const KGParams& p, int ro
     const int n = n_base + 8 * j8;
     float v[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(acc[8 * j8 + e], p.out_scale);
-    if (p.bias != nullptr && n < p.N) {
-      const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
-      const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[2 * e] = __fadd_rn(v[2 * e], bf16lo(bw[e]));
-        v[2 * e + 1] = __fadd_rn(v[2 * e + 1], bf16hi(bw[e]));
-      }
-    }
-    if (p.gelu) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = gelu_tanh(v[e]);
-    }
+    for (int e = 0; e < 8; ++e) v[e] = acc[8 * j8 + e];
+    scale_bias_pairs(p, n, v);
+    if (p.gelu) gelu_tanh_pairs<4>(v);
 #pragma unroll
     for (int e = 0; e < 4; ++e) w[4 * j8 + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
   }

@@ -375,20 +375,9 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       for (int c8 = 0; c8 < 8; ++c8) {
         float y[8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) y[t] = __fmul_rn(f[8 * c8 + t], p.out_scale);
-        if (p.bias != nullptr) {
-          const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n_base + 8 * c8));
-          const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            y[2 * t] = __fadd_rn(y[2 * t], bf16lo(bw[t]));
-            y[2 * t + 1] = __fadd_rn(y[2 * t + 1], bf16hi(bw[t]));
-          }
-        }
-        if (p.gelu) {
-#pragma unroll
-          for (int t = 0; t < 8; ++t) y[t] = gelu_tanh(y[t]);
-        }
+        for (int t = 0; t < 8; ++t) y[t] = f[8 * c8 + t];
+        scale_bias_pairs(p, n_base + 8 * c8, y);
+        if (p.gelu) gelu_tanh_pairs<4>(y);
         const float4 i0 = __ldg(reinterpret_cast<const float4*>(c.inv_lam2 + n_base + 8 * c8));
         const float4 i1 = __ldg(reinterpret_cast<const float4*>(c.inv_lam2 + n_base + 8 * c8 + 4));
         const float il[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
