@@ -580,7 +580,8 @@ def run_ours(args, layers):
         "e2e": {"value": job_throughput(world, flops, ms_e2e), "unit": "TFLOPS",
                 "h2d_bytes_per_step": sum(d["layer"].M * d["layer"].K * 2 for d in L),
                 "d2h_bytes_per_step": sum(d["layer"].M * d["layer"].N * 2 for d in L)},
-        "gpu_launches": len(launches) * args.steps,
+        # the qkv-epilogue call launches the rotary-table copy and the GEMM
+        "gpu_launches": sum(2 if n.endswith("_qkv") else 1 for n, _ in launches) * args.steps,
         "clocks": clk,
         "kernel_source_hash": kernel_source_hash(),
     }
