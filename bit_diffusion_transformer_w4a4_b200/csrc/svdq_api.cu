@@ -203,6 +203,11 @@ struct svdq_weights {
   // host-call staging
   void* x_dev = nullptr;
   void* y_dev = nullptr;
+  // svdq_linear_forward_host: copy streams (in, out) and per-chunk events,
+  // created on first use; the K split its row chunks share (0 = automatic)
+  cudaStream_t host_in = nullptr, host_out = nullptr;
+  cudaEvent_t host_ev[2 * 8 + 1] = {};
+  int kq_ksplit_force = 0;
   int* err = nullptr;
   uint32_t debug_mask = 0;
   uint64_t timeout_ns = kDefaultTimeoutNs;
@@ -236,9 +241,23 @@ void free_all(svdq_weights* h) {
                   h->kq_tpart, h->kq_counters, h->kq_flags};
   for (void* p : ptrs)
     if (p) cudaFree(p);
+  for (cudaEvent_t e : h->host_ev)
+    if (e) cudaEventDestroy(e);
+  if (h->host_in) cudaStreamDestroy(h->host_in);
+  if (h->host_out) cudaStreamDestroy(h->host_out);
 }
 
 // ------------------------------------------------------------------ launches
+// K splits of the activation kernel for M rows: the most (up to 8, dividing
+// the K / 64 chunks) that keep the grid within one wave of the SMs.
+int kq_auto_ksplit(const svdq_weights* h, int64_t M) {
+  const int num_m = static_cast<int>(cdiv(M, 128));
+  const int kch = static_cast<int>(h->K / 64);
+  int ksplit = 1;
+  while (ksplit < 8 && num_m * ksplit * 2 <= h->sms && kch % (ksplit * 2) == 0) ksplit *= 2;
+  return ksplit;
+}
+
 template <int V, int R>
 svdq_status launch_kq_t(svdq_weights* h, const CUtensorMap& tmx, int64_t M, uint8_t* codes,
                         void* scales, float* t, cudaStream_t st) {
@@ -246,12 +265,9 @@ svdq_status launch_kq_t(svdq_weights* h, const CUtensorMap& tmx, int64_t M, uint
   if (svdq_status s = ensure_smem<kq_kernel<V, R>>(S::TOTAL); s != SVDQ_OK) return s;
   const int num_m = static_cast<int>(cdiv(M, 128));
   const int kch = static_cast<int>(h->K / 64);
-  // split the K range so that the grid fills the SMs in one wave
-  int ksplit = 1;
-  if (R > 0)
-    while (ksplit < 8 && num_m * ksplit * 2 <= h->sms && kch % (ksplit * 2) == 0) ksplit *= 2;
-  else
-    while (ksplit < 8 && num_m * ksplit * 2 <= h->sms && kch % (ksplit * 2) == 0) ksplit *= 2;
+  // split the K range so that the grid fills the SMs in one wave (or as the
+  // host-buffer entry point fixes it for its row chunks)
+  const int ksplit = h->kq_ksplit_force > 0 ? h->kq_ksplit_force : kq_auto_ksplit(h, M);
   // split partials are added into T (split 0 clears it first, see kq.cuh);
   // in deterministic mode they go through the scratch and are summed in
   // split order
@@ -1233,13 +1249,59 @@ svdq_status svdq_linear_forward_host(svdq_weights_t h, const void* x_host, void*
       return SVDQ_ERR_OOM;
     }
   }
+  if (!h->host_in) {
+    if (cudaStreamCreateWithFlags(&h->host_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&h->host_out, cudaStreamNonBlocking) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+    for (cudaEvent_t& e : h->host_ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return SVDQ_ERR_CUDA;
+  }
+  // Row chunks of at least 256 rows (at most 8; a last chunk of 128 rows or
+  // fewer joins the one before, so every chunk runs on the same GEMM kernel
+  // as the whole M would): chunk c's input copy (stream host_in) overlaps
+  // the layer on earlier chunks (the caller's stream) and their output copies
+  // (host_out), whose two directions run at once.  Each chunk's activation
+  // kernel uses the K split of the whole M, so the chunks produce exactly
+  // what one call over M would.  The workspace is reused chunk after chunk
+  // (the layer's launches are ordered on the caller's stream).
+  const int64_t C = std::max<int64_t>(256, cdiv(cdiv(M, 6), 256) * 256);
+  int64_t bounds[9];
+  int nc = 0;
+  for (int64_t r0 = 0; r0 < M && nc < 8; r0 += C) bounds[nc++] = r0;
+  if (nc > 1 && M - bounds[nc - 1] <= 128) --nc;
+  bounds[nc] = M;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  SVDQ_TRY(cudaMemcpyAsync(h->x_dev, x_host, static_cast<size_t>(M) * h->K * 2,
-                           cudaMemcpyHostToDevice, st));
-  if ((s = svdq_linear_forward(h, h->x_dev, h->y_dev, M, stream)) != SVDQ_OK) return s;
-  SVDQ_TRY(cudaMemcpyAsync(y_host, h->y_dev, static_cast<size_t>(M) * h->N * 2,
-                           cudaMemcpyDeviceToHost, st));
-  return SVDQ_OK;
+  cudaEvent_t* ev = h->host_ev;  // [0, nc) inputs copied, [8, 8 + nc) chunks computed, [16] entry / exit
+  const size_t xrow = static_cast<size_t>(h->K) * 2, yrow = static_cast<size_t>(h->N) * 2;
+  // the staging buffers are free once the caller's stream reaches this call
+  SVDQ_TRY(cudaEventRecord(ev[16], st));
+  SVDQ_TRY(cudaStreamWaitEvent(h->host_in, ev[16], 0));
+  SVDQ_TRY(cudaStreamWaitEvent(h->host_out, ev[16], 0));
+  h->kq_ksplit_force = kq_auto_ksplit(h, M);
+  for (int c = 0; c < nc; ++c) {
+    const int64_t r0 = bounds[c], mc = bounds[c + 1] - r0;
+    uint8_t* xd = static_cast<uint8_t*>(h->x_dev) + r0 * xrow;
+    uint8_t* yd = static_cast<uint8_t*>(h->y_dev) + r0 * yrow;
+    if (cudaMemcpyAsync(xd, static_cast<const uint8_t*>(x_host) + r0 * xrow, mc * xrow,
+                        cudaMemcpyHostToDevice, h->host_in) != cudaSuccess ||
+        cudaEventRecord(ev[c], h->host_in) != cudaSuccess || cudaStreamWaitEvent(st, ev[c], 0) != cudaSuccess) {
+      s = SVDQ_ERR_CUDA;
+      break;
+    }
+    if ((s = svdq_linear_forward(h, xd, yd, mc, stream)) != SVDQ_OK) break;
+    if (cudaEventRecord(ev[8 + c], st) != cudaSuccess || cudaStreamWaitEvent(h->host_out, ev[8 + c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t*>(y_host) + r0 * yrow, yd, mc * yrow, cudaMemcpyDeviceToHost,
+                        h->host_out) != cudaSuccess) {
+      s = SVDQ_ERR_CUDA;
+      break;
+    }
+  }
+  h->kq_ksplit_force = 0;
+  // the caller's stream completes after the last output copy (also on an
+  // error above, after the copies already enqueued)
+  if (cudaEventRecord(ev[16], h->host_out) != cudaSuccess || cudaStreamWaitEvent(st, ev[16], 0) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  return s;
 }
 
 svdq_status svdq_device_status(svdq_weights_t h, void* stream) {

@@ -286,9 +286,18 @@ svdq_status svdq_linear_forward_chain(svdq_weights_t h1, svdq_weights_t h2, cons
 /*
  * Defined by: the same layer as svdq_linear_forward.
  * Same as svdq_linear_forward with HOST input and output (pinned memory is
- * recommended): copies x_host to the device, runs the layer and copies y back
- * on `stream`.  Returns after enqueueing; synchronise the stream before
- * reading y_host.  Device staging buffers are owned by the handle.
+ * recommended; pageable memory works but its copies do not overlap): copies
+ * x_host to the device, runs the layer and copies y back.  The rows go in
+ * chunks (at least 256 rows, at most 8 chunks): a chunk's input copy and the
+ * output copies of earlier chunks run on two streams of the handle while the
+ * layer runs on `stream`, so the two copy directions and the kernels
+ * overlap.  Y is the same as one svdq_linear_forward over all M rows (the
+ * chunks use the activation kernel's K split of the whole M; with
+ * svdq_set_deterministic, bit for bit).  Returns after enqueueing; `stream`
+ * completes after the last output copy, so synchronise it before reading
+ * y_host.  Device staging buffers, the two streams and their events are
+ * owned by the handle (created on first use); calls on one handle must not
+ * overlap.
  */
 svdq_status svdq_linear_forward_host(svdq_weights_t h, const void* x_host, void* y_host,
                                      int64_t M, void* stream);

@@ -125,9 +125,13 @@ def test_quantizer_edge_values():
 
 
 @pytest.mark.parametrize("variant", [INT4, NVFP4])
-def test_host_entry_point_matches_device(variant):
+@pytest.mark.parametrize("M", [256, 1300])
+def test_host_entry_point_matches_device(variant, M):
+    """The host-buffer entry point (row chunks with overlapped copies at
+    M = 1300: five chunks, the last of 276 rows) gives the device entry
+    point's Y bit for bit (deterministic T)."""
     import torch
-    M, K, N, r = 256, 512, 512, 32
+    K, N, r = 512, 512, 32
     lay = W.Layer("host", M=M, K=K, N=N, r=r, variant=variant, config_id=61)
     pw = W.synthetic_packed(lay)
     x = W.activations(lay)
