@@ -325,9 +325,10 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
       for (int i = 0; i < 16; ++i) acc[i] = 0ull;
       const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16) + cs * 32;
       // float(P) for the s32 group product P (16 x a sum of 64 products of
-      // 4-bit codes, |P| <= 65536 < 2^22): bits(P + bits(1.5 * 2^23)) -
-      // 1.5 * 2^23, exact, at the full rate of integer and fp32 adds
-      const uint64_t mag = f2_pack(-12582912.0f, -12582912.0f);
+      // 4-bit codes, |P| <= 65536 < 2^24): the hardware conversion, exact.
+      // (The magic-number form, bits(P + bits(1.5 * 2^23)) - 1.5 * 2^23 in an
+      // integer add and a paired fp32 add, measured 612 against 547 us for
+      // qkv's kernel 2.)
       const uint8_t* scb = nullptr;
       for (int g = 0; g < ng; ++g, ++gc) {
         const int gi = g % KGI4_GC;
@@ -359,10 +360,10 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
           const float4 w = swr[i4];
           const uint64_t s01 = f2_mul(sx2, f2_pack(w.x, w.y));
           const uint64_t s23 = f2_mul(sx2, f2_pack(w.z, w.w));
-          const uint64_t p01 = f2_add(f2_pack(__uint_as_float(v[4 * i4] + 0x4B400000u),
-                                              __uint_as_float(v[4 * i4 + 1] + 0x4B400000u)), mag);
-          const uint64_t p23 = f2_add(f2_pack(__uint_as_float(v[4 * i4 + 2] + 0x4B400000u),
-                                              __uint_as_float(v[4 * i4 + 3] + 0x4B400000u)), mag);
+          const uint64_t p01 = f2_pack(__int2float_rn(static_cast<int>(v[4 * i4])),
+                                       __int2float_rn(static_cast<int>(v[4 * i4 + 1])));
+          const uint64_t p23 = f2_pack(__int2float_rn(static_cast<int>(v[4 * i4 + 2])),
+                                       __int2float_rn(static_cast<int>(v[4 * i4 + 3])));
           acc[2 * i4] = f2_fma(p01, s01, acc[2 * i4]);
           acc[2 * i4 + 1] = f2_fma(p23, s23, acc[2 * i4 + 1]);
         }
