@@ -74,7 +74,7 @@ typedef enum {
  * default, when M > 128, it runs on pairs of SMs: a two-CTA cluster per
  * 256 x 256 tile, one M = 256 tensor-core MMA stream per pair, which halves
  * the B bytes each SM stages and so deepens the pipeline (B200, fc1
- * 4608 x 3072 x 12288: 108.5 vs 118.8 us).  Both compute the same y up to
+ * 4608 x 3072 x 12288: 108.5 vs 118.8 us side by side).  Both compute the same y up to
  * fp32 summation order.  For comparison and tests. */
 #define SVDQ_GEMM_SINGLE_SM 2u
 /* INT4 only: run kernel 2 as one fp16 GEMM of the dequantised operands
