@@ -124,18 +124,20 @@ def test_quantizer_edge_values():
         PT.check_act(got, ref, r=r, label=f"edge v{variant}")
 
 
-@pytest.mark.parametrize("variant", [INT4, NVFP4])
-@pytest.mark.parametrize("M", [256, 1300])
-def test_host_entry_point_matches_device(variant, M):
-    """The host-buffer entry point (row chunks with overlapped copies at
-    M = 1300: five chunks, the last of 276 rows) gives the device entry
-    point's Y bit for bit (deterministic T)."""
+@pytest.mark.parametrize("variant,opts", [(INT4, {}), (NVFP4, {}), (INT4, {"int4_f16": True})],
+                         ids=["int4", "nvfp4", "int4-f16"])
+@pytest.mark.parametrize("M", [100, 256, 1300, 1536])
+def test_host_entry_point_matches_device(variant, opts, M):
+    """The host-buffer entry point gives the device entry point's Y bit for
+    bit (deterministic T): one chunk on single SMs (M = 100), one chunk
+    (256), five chunks with a last one of 276 rows (1300), six chunks of 256
+    rows (1536)."""
     import torch
     K, N, r = 512, 512, 32
     lay = W.Layer("host", M=M, K=K, N=N, r=r, variant=variant, config_id=61)
     pw = W.synthetic_packed(lay)
     x = W.activations(lay)
-    h = svdq.SVDQWeights(pw, M)
+    h = svdq.SVDQWeights(pw, M, **opts)
     h.set_deterministic()
     dev = PT.gpu_forward(h, x, M, two_calls=False)
     xh = torch.from_numpy(x.view(np.int16)).pin_memory()

@@ -58,7 +58,7 @@ def _run(M, H, r, opts, with_bias=True, seed=0, pw_kind="prep"):
 
 
 @pytest.mark.parametrize("opts", [{}, {"single_sm": True}], ids=["pair", "1sm"])
-@pytest.mark.parametrize("M,H,r", [(300, 2, 32), (129, 1, 16), (640, 3, 0)])
+@pytest.mark.parametrize("M,H,r", [(300, 2, 32), (129, 1, 16), (640, 3, 0), (1, 1, 32)])
 def test_qkv_epilogue(opts, M, H, r):
     Y, yq, Yq = _run(M, H, r, opts)
     PT.check_y(Y, yq, Yq, label=f"qkv M{M} H{H} r{r} {opts}")
