@@ -77,10 +77,14 @@ __device__ __forceinline__ void gelu_tanh_pairs(float* v) {
 
 // v[0..7] (columns n..n+7) <- v * out_scale (+ bias), in pairs.
 __device__ __forceinline__ void scale_bias_pairs(const KGParams& p, int n, float* v) {
-  const uint64_t os2 = f2_pack(p.out_scale, p.out_scale);
   uint64_t x[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) x[e] = f2_mul(f2_pack(v[2 * e], v[2 * e + 1]), os2);
+  for (int e = 0; e < 4; ++e) x[e] = f2_pack(v[2 * e], v[2 * e + 1]);
+  if (p.out_scale != 1.0f) {  // 2^e, only with an NVFP4 per-tensor weight scale (x 1 is exact)
+    const uint64_t os2 = f2_pack(p.out_scale, p.out_scale);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = f2_mul(x[e], os2);
+  }
   if (p.bias != nullptr && n < p.N) {
     const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
     const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};

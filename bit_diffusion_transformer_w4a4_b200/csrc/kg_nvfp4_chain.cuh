@@ -384,7 +384,8 @@ __global__ void __launch_bounds__(KG_THREADS, 1)
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const uint32_t y1 = pack_bf16x2(y[2 * t], y[2 * t + 1]);  // fc1's bf16 output
-          w[4 * c8 + t] = pack_bf16x2(__fmul_rn(bf16lo(y1), il[2 * t]), __fmul_rn(bf16hi(y1), il[2 * t + 1]));
+          const uint64_t x2 = f2_mul(f2_pack(bf16lo(y1), bf16hi(y1)), f2_pack(il[2 * t], il[2 * t + 1]));
+          w[4 * c8 + t] = pack_bf16x2(f2_lo(x2), f2_hi(x2));
         }
       }
       // fc2's NVFP4 group quantisation of the 64 values (4 groups of 16),
