@@ -528,3 +528,80 @@ def test_chain_single_free_barrier_is_caught():
         res = m.run()
         bad += res != "ok" or bool(m.errors)
     assert bad > 0
+
+
+class QkvExchangeModel:
+    """The fused QKV epilogue's per-head exchange: the two warps that hold
+    the two 64-column halves of a head (same 32 rows) publish their partial
+    sums of squares in shared memory and meet on one mbarrier (two warps'
+    arrivals per phase), twice per tile: after writing (then each reads the
+    partner's partial) and after reading (so that the next tile's write
+    cannot overtake the partner's read).  Tiles whose columns are V skip the
+    exchange in both warps.  `one_phase` plants the version without the
+    second phase."""
+
+    def __init__(self, tiles, rng, one_phase=False):
+        self.tiles, self.rng, self.one_phase = tiles, rng, one_phase
+        self.errors = []
+        self.bar = MBar(2, self.errors)
+        self.red = [None, None]
+
+    def warp(self, w):
+        xph = 0
+        for j, is_v in enumerate(self.tiles):
+            if is_v:
+                yield None
+                continue
+            self.red[w] = (j, w)
+            self.bar.arrive()
+            yield (self.bar, xph & 1)
+            if self.red[1 - w] != (j, 1 - w):
+                self.errors.append(f"warp {w} tile {j} read the partner's {self.red[1 - w]}")
+            if self.one_phase:
+                xph += 1
+                continue
+            self.bar.arrive()
+            yield (self.bar, (xph + 1) & 1)
+            xph += 2
+
+    def run(self):
+        agents = [self.warp(0), self.warp(1)]
+        blocked = [None, None]
+        live = {0, 1}
+        steps = 0
+        while live:
+            steps += 1
+            if steps > 100000:
+                return "livelock"
+            runnable = [i for i in live if blocked[i] is None or blocked[i][0].try_wait(blocked[i][1])]
+            if not runnable:
+                return "deadlock"
+            c = self.rng.choice(runnable)
+            blocked[c] = None
+            try:
+                op = next(agents[c])
+                blocked[c] = op
+            except StopIteration:
+                live.discard(c)
+        return "ok"
+
+
+@pytest.mark.parametrize("n", [1, 2, 5, 9])
+def test_qkv_exchange_is_safe(n):
+    for seed in range(30):
+        rng = random.Random(seed)
+        tiles = [rng.random() < 0.3 for _ in range(n)]
+        m = QkvExchangeModel(tiles, rng)
+        assert m.run() == "ok"
+        assert not m.errors, m.errors[:3]
+
+
+def test_qkv_exchange_single_phase_is_caught():
+    """Planted mistake: one phase per tile; a warp that runs a tile ahead
+    overwrites its partial before the partner has read it."""
+    bad = 0
+    for seed in range(40):
+        m = QkvExchangeModel([False] * 4, random.Random(seed), one_phase=True)
+        res = m.run()
+        bad += res != "ok" or bool(m.errors)
+    assert bad > 0
